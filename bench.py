@@ -1,0 +1,422 @@
+"""Benchmark of the BPT layer forward on B200: tokens/s and TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one whole layer forward (QKV projection, blockwise attention over
+every query block, output projection, residuals and FFN) over one batch of
+synthetic inputs already resident in HBM. N > 1 runs under torchrun, one rank
+per GPU: every rank runs its own sequence(s) (independent units, no collective
+on the data path); the timed region is bracketed by a barrier and a device
+sync on every rank and the reported time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (a deliberately slow program) on a
+bounded sample of the same workload, on the host cores, rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import bpt_inputs as bi  # noqa: E402
+
+METRIC = "BPT layer fwd tokens/s and TFLOP/s (% BF16 peak) on 1 B200, vs fp64 oracle"
+DEFAULT_WORKLOAD = "gpt7b_s32768_h4096"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# work accounting (matmul flops; causal attention counted as half)
+# ---------------------------------------------------------------------------
+
+def layer_flops(shape: bi.LayerShape) -> dict:
+    b, s, h = shape.b, shape.s, shape.h
+    tok = b * s
+    att = 4.0 * b * s * s * h * (0.5 if shape.causal else 1.0)
+    return {
+        "gemm_qkv": 2.0 * tok * h * 3 * h,
+        "attention": att,
+        "gemm_outproj": 2.0 * tok * h * h,
+        "gemm_ffn_up": 2.0 * tok * h * 4 * h,
+        "gemm_ffn_down": 2.0 * tok * 4 * h * h,
+    }
+
+
+def measured_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str, world: int):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """Max of a float over all ranks (every rank takes this step)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64,
+                     device=device if (device is not None and dist.get_backend() == "nccl") else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own sequence(s): independent units of work."""
+    return rank
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="bpt_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(shape: bi.LayerShape, inp: dict, budget_s: float = 10.0, max_rows: int | None = None):
+    """Time the oracle on the first n rows of sequence 0 (n doubled until the
+    budget is spent). Returns (tokens/s, rows, seconds)."""
+    import oracle
+    args = bi.oracle_args(inp)
+    n = 64
+    cap = min(shape.s, max_rows or shape.s)
+    best = None
+    while True:
+        rows = np.arange(min(n, cap), dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.layer_rows(*args, heads=shape.heads, causal=shape.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        best = (rows.size / dt, int(rows.size), dt)
+        if dt >= budget_s or rows.size >= cap:
+            return best
+        n = min(cap, max(n * 2, int(n * budget_s / max(dt, 1e-3) * 0.6)))
+
+
+def reference_arm(args, shape, name):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = bi.make_inputs(shape, seed=0)
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample(shape, inp, budget_s=2.0, max_rows=256)
+    for _ in range(args.steps):
+        per_step.append(oracle_sample(shape, inp, budget_s=args.ref_budget))
+    tps = float(np.mean([p[0] for p in per_step]))
+    rows = per_step[-1][1]
+    secs = float(sum(p[2] for p in per_step))
+    cores = blas_threads()
+    sample = (f"oracle rows t=0..{rows - 1} of sequence 0 (their keys/values projected), fp64 numpy/BLAS; "
+              f"early causal rows attend to short prefixes, so this favours the CPU")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases)",
+        "config": config_of(shape, name),
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(shape: bi.LayerShape, name: str) -> dict:
+    return {"workload": name, "batch": shape.b, "seq_len": shape.s, "d_model": shape.h, "heads": shape.heads,
+            "head_dim": shape.dh, "ffn_hidden": shape.f, "causal": shape.causal, "q_block": shape.q_block,
+            "kv_block": shape.kv_block, "input_dtype": shape.dtype,
+            "l2": "inputs larger than L2 (x, K/V and weights each exceed 126 MB)"
+            if shape.b * shape.s * shape.h * 2 > L2_BYTES else "L2 flushed between steps",
+            "parallelism": "independent sequences per GPU"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def our_arm(args, shape, name):
+    import torch
+
+    import blockwise_attn_ffn_bpt_b200 as bpt
+
+    world, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist("nccl", world)
+
+    inp = bi.make_inputs(shape, seed=rank_seed(rank))
+    x = bi.to_torch(inp["x"], device)
+    params = {k: bi.to_torch(inp[k], device) for k in bi.PARAM_NAMES}
+    out = torch.empty((shape.b, shape.s, shape.h), dtype=torch.float32, device=device)
+    dtype_code = bpt.BPT_DTYPE_F32 if shape.dtype == "f32" else bpt.BPT_DTYPE_BF16
+    ws_bytes = bpt.workspace_bytes(dtype_code, shape.b, shape.s, shape.h, shape.heads, shape.q_block,
+                                   shape.kv_block)
+    flush = None
+    if shape.b * shape.s * shape.h * 2 <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal, out=out,
+                          stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if bpt.device_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    torch.cuda.reset_peak_memory_stats(device)
+    mem0 = torch.cuda.memory_allocated(device)
+    free0, _ = torch.cuda.mem_get_info(device)
+    bpt.set_kernel_timing(True)
+    bpt.kernel_times()
+    launches0 = bpt.launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                      int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+    launches = bpt.launch_count() - launches0
+    ktimes = bpt.kernel_times()
+    bpt.set_kernel_timing(False)
+    if bpt.device_status() != 0:
+        raise RuntimeError("device error during the timed region")
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, dist, device)
+
+    # ---- end to end through the public API from pinned host memory
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    out_host = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+    x_dev = torch.empty_like(x)
+    for _ in range(max(1, args.warmup // 2)):
+        bpt.layer_forward_from_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+                                    out_host=out_host, x_dev=x_dev, out_dev=out, stream=stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(e2e_steps):
+        with torch.cuda.stream(stream):
+            x_dev.copy_(x_host, non_blocking=True)
+            bpt.layer_forward(x_dev, params, shape.heads, shape.q_block, shape.kv_block, shape.causal, out=out,
+                              stream=stream)
+            out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+
+    peak_bytes = torch.cuda.max_memory_allocated(device) - mem0
+
+    # ---- CPU baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, rows, secs = oracle_sample(shape, inp, budget_s=args.ref_budget)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {rows} rows of sequence 0 with their keys/values, fp64 numpy/BLAS, {secs:.1f} s"}
+
+    if dist is not None:
+        barrier(dist, device)
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    tokens = shape.b * shape.s
+    flops = layer_flops(shape)
+    total_flops = sum(flops.values())
+    value = tokens * args.steps * world / (ms_max / 1e3)
+    tflops = total_flops * args.steps * world / (ms_max / 1e3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+
+    # dominant kernel: largest share of the timed kernel time
+    dom = max(ktimes.items(), key=lambda kv: kv[1][1]) if ktimes else None
+    roof = None
+    if dom is not None:
+        kname, (nl, kms) = dom
+        kflops = flops.get(kname, 0.0) * args.steps
+        achieved = kflops / (kms / 1e3) / 1e12 if kms > 0 else 0.0
+        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "launches": nl, "avg_launch_ms": kms / nl,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"}
+    kernel_table = {k: {"launches": n, "ms": t, "share": t / sum(v[1] for v in ktimes.values())}
+                    for k, (n, t) in ktimes.items()}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases; random-init layer)",
+        "config": config_of(shape, name),
+        "tflops": tflops, "frac_of_bf16_peak": tflops / peak,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens * e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+        "gpu_launches": int(launches),
+        "kernels": kernel_table,
+        "clocks": clocks.summary(),
+        "memory": {"workspace_bytes": ws_bytes, "ratio_bytes_vs_2bsh": ws_bytes / (2 * tokens * shape.h),
+                   "ratio_elems_vs_2bsh": ws_bytes / 2 / (2 * tokens * shape.h),
+                   "peak_torch_alloc_bytes_in_step": int(peak_bytes),
+                   "free_bytes_before": int(free0)},
+    }
+    print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="one of: " + ", ".join(list(bi.WORKLOADS) + ["sweep_<block>_<causal|noncausal>"]))
+    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    name = args.workload
+    if name.startswith("sweep_"):
+        _, blk, c = name.split("_")
+        shape = bi.sweep_shape(int(blk), c == "causal")
+    else:
+        shape = bi.WORKLOADS[name]
+    world, _, _ = dist_env()
+    if world != args.gpus:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        return reference_arm(args, shape, name)
+    return our_arm(args, shape, name)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,212 @@
+"""Python binding of the B200 BPT layer-forward library (libbpt.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. torch is used for device memory and streams. There is no fallback:
+if the built library is missing, or a call returns an error status, these
+functions raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbpt.so")
+
+BPT_DTYPE_BF16 = 0
+BPT_DTYPE_F32 = 1
+
+EXPORTED = (
+    "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
+    "bpt_layer_forward_ws", "bpt_qkv_projection", "bpt_attention", "bpt_device_status",
+    "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
+)
+
+
+class BPTError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m blockwise_attn_ffn_bpt_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.bpt_status_string.restype = ctypes.c_char_p
+    L.bpt_status_string.argtypes = [i]
+    L.bpt_layer_forward.restype = i
+    L.bpt_layer_forward.argtypes = [vp] * 9 + [i] * 7 + [vp, vp]
+    L.bpt_layer_forward_f32.restype = i
+    L.bpt_layer_forward_f32.argtypes = [vp] * 9 + [i] * 7 + [vp, vp]
+    L.bpt_layer_workspace_bytes.restype = sz
+    L.bpt_layer_workspace_bytes.argtypes = [i] * 8
+    L.bpt_layer_forward_ws.restype = i
+    L.bpt_layer_forward_ws.argtypes = [i] + [vp] * 9 + [i] * 8 + [vp, sz, vp, vp]
+    L.bpt_qkv_projection.restype = i
+    L.bpt_qkv_projection.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
+    L.bpt_attention.restype = i
+    L.bpt_attention.argtypes = [vp] * 3 + [i] * 7 + [vp, vp]
+    L.bpt_device_status.restype = i
+    L.bpt_device_status.argtypes = []
+    L.bpt_launch_count.restype = ctypes.c_uint64
+    L.bpt_launch_count.argtypes = []
+    L.bpt_set_kernel_timing.restype = i
+    L.bpt_set_kernel_timing.argtypes = [i]
+    L.bpt_kernel_times.restype = i
+    L.bpt_kernel_times.argtypes = [ctypes.POINTER(KernelTime), i]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().bpt_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise BPTError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+PARAM_NAMES = ("Wqkv", "bqkv", "Wo", "bo", "W1", "b1", "W2", "b2")
+
+
+def workspace_bytes(dtype: int, b: int, s: int, h: int, heads: int, q_block: int, kv_block: int,
+                    wave_rows: int = 0) -> int:
+    return int(lib().bpt_layer_workspace_bytes(dtype, b, s, h, heads, q_block, kv_block, wave_rows))
+
+
+def layer_forward(x: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int, causal: bool,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  wave_rows: int = 0, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One BPT layer forward; x [b, s, h] (bf16 or fp32) on the GPU, params a
+    dict of Wqkv [h,3h], bqkv, Wo [h,h], bo, W1 [h,4h], b1, W2 [4h,h], b2 of
+    x's dtype. Returns out, fp32 [b, s, h].
+
+    With workspace=None the library allocates its workspace stream-ordered;
+    otherwise `workspace` (a uint8 CUDA tensor of at least workspace_bytes(...))
+    is used and nothing is allocated.
+    """
+    b, s, h = x.shape
+    if out is None:
+        out = torch.empty((b, s, h), dtype=torch.float32, device=x.device)
+    ps = [_ptr(params[k]) for k in PARAM_NAMES]
+    if x.dtype == torch.bfloat16:
+        dtype = BPT_DTYPE_BF16
+    elif x.dtype == torch.float32:
+        dtype = BPT_DTYPE_F32
+    else:
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    for k in PARAM_NAMES:
+        if params[k].dtype != x.dtype:
+            raise TypeError(f"{k} must have dtype {x.dtype}")
+    st = _stream(stream)
+    if workspace is None and wave_rows == 0:
+        fn = lib().bpt_layer_forward if dtype == BPT_DTYPE_BF16 else lib().bpt_layer_forward_f32
+        r = fn(_ptr(x), *ps, b, s, h, heads, q_block, kv_block, int(bool(causal)), _ptr(out), st)
+    else:
+        if workspace is None:
+            nbytes = workspace_bytes(dtype, b, s, h, heads, q_block, kv_block, wave_rows)
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        r = lib().bpt_layer_forward_ws(dtype, _ptr(x), *ps, b, s, h, heads, q_block, kv_block, int(bool(causal)),
+                                       wave_rows, _ptr(workspace), workspace.numel(), _ptr(out), st)
+    _check(r, "bpt_layer_forward")
+    return out
+
+
+def layer_forward_from_host(x_host: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int,
+                            causal: bool, out_host: Optional[torch.Tensor] = None,
+                            x_dev: Optional[torch.Tensor] = None, out_dev: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """End-to-end call from host memory: copy x (pinned host) to the device,
+    run the layer (weights already resident on the device), copy out back to
+    (pinned) host memory. Returns out_host after the stream has finished."""
+    b, s, h = x_host.shape
+    dev = params["Wqkv"].device
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    if x_dev is None:
+        x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device=dev)
+    if out_dev is None:
+        out_dev = torch.empty((b, s, h), dtype=torch.float32, device=dev)
+    if out_host is None:
+        out_host = torch.empty((b, s, h), dtype=torch.float32, pin_memory=True)
+    with torch.cuda.stream(st):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer_forward(x_dev, params, heads, q_block, kv_block, causal, out=out_dev, stream=st)
+        out_host.copy_(out_dev, non_blocking=True)
+    st.synchronize()
+    return out_host
+
+
+def qkv_projection(x: torch.Tensor, Wqkv: torch.Tensor, bqkv: torch.Tensor,
+                   stream: Optional[torch.cuda.Stream] = None):
+    """Algorithm 1 step 1 alone: bf16 Q, K, V [b, s, h] from bf16 x [b, s, h]."""
+    b, s, h = x.shape
+    q = torch.empty((b, s, h), dtype=torch.bfloat16, device=x.device)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    r = lib().bpt_qkv_projection(_ptr(x), _ptr(Wqkv), _ptr(bqkv), b, s, h, _ptr(q), _ptr(k), _ptr(v),
+                                 _stream(stream))
+    _check(r, "bpt_qkv_projection")
+    return q, k, v
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int, q_block: int, kv_block: int,
+              causal: bool, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Algorithm 1 steps 2-10 alone: bf16 O [b, s, h] (heads concatenated)."""
+    b, s, h = q.shape
+    o = torch.empty((b, s, h), dtype=torch.bfloat16, device=q.device)
+    r = lib().bpt_attention(_ptr(q), _ptr(k), _ptr(v), b, s, h, heads, q_block, kv_block, int(bool(causal)),
+                            _ptr(o), _stream(stream))
+    _check(r, "bpt_attention")
+    return o
+
+
+def device_status() -> int:
+    return int(lib().bpt_device_status())
+
+
+def launch_count() -> int:
+    return int(lib().bpt_launch_count())
+
+
+def set_kernel_timing(enable: bool) -> None:
+    _check(lib().bpt_set_kernel_timing(int(bool(enable))), "bpt_set_kernel_timing")
+
+
+def kernel_times(max_kinds: int = 32) -> dict:
+    """{kernel name: (launches, total ms)} since timing was enabled or last read."""
+    arr = (KernelTime * max_kinds)()
+    n = lib().bpt_kernel_times(arr, max_kinds)
+    if n < 0:
+        raise BPTError(n, "bpt_kernel_times")
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}

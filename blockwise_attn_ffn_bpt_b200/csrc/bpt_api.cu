@@ -1,0 +1,618 @@
+// C ABI of the BPT layer forward: argument checks, workspace layout, TMA
+// descriptors, the wave schedule and the kernel launches.
+//
+// Schedule of one call (Algorithm 1 of the BPT paper review, section 3):
+//   1. QKV projection over the whole sequence (step 1): K and V go to the
+//      workspace, Q is parked inside `out` (a bf16 Q row fits in the first half
+//      of its fp32 output row and is consumed before that row is written).
+//   2. For each wave of query blocks (a whole number of q_block rows, about
+//      4096 by default): blockwise attention of the wave's query tiles over all
+//      key/value tiles (steps 4-10), then Wo + bo + x (first residual, fp32 into
+//      `out`), W1 + b1 + ReLU (bf16 U) and W2 + b2 + hid (second residual) on
+//      the wave's rows (step 11). Scratch is bounded by the wave, not by s: the
+//      full-sequence 4h FFN intermediate and the s x s scores never exist.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attention.cuh"
+#include "bpt.h"
+#include "gemm.cuh"
+
+namespace bpt {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// ------------------------------------------------------------- timing log
+struct TimedLaunch {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+bool g_timing = false;
+std::vector<TimedLaunch> g_timed;
+
+struct LaunchScope {
+  TimedLaunch rec{};
+  bool on = false;
+  cudaStream_t stream;
+  LaunchScope(const char* name, cudaStream_t st) : stream(st) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    if (!g_timing) return;
+    on = true;
+    rec.name = name;
+    cudaEventCreate(&rec.start);
+    cudaEventCreate(&rec.stop);
+    cudaEventRecord(rec.start, stream);
+  }
+  ~LaunchScope() {
+    if (!on) return;
+    cudaEventRecord(rec.stop, stream);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timed.push_back(rec);
+  }
+};
+
+// ------------------------------------------------------------- driver entry
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first,
+// strides in bytes for dims 1.. (dim 0 is contiguous).
+bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides[i];
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// [rows, cols] bf16 row-major with `ld` elements between rows, loaded as
+// [box_rows][64] boxes.
+bool map_rows(CUtensorMap* m, const void* base, long long rows, long long cols, long long ld, uint32_t box_rows) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)ld * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return make_map(m, base, 2, dims, strides, box);
+}
+
+// [b, s, cols] bf16 with `ld` elements between rows, [128 rows][64] boxes;
+// rows past s of a sequence read as zero.
+bool map_seq(CUtensorMap* m, const void* base, int b, int s, int cols, long long ld) {
+  const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)s, (uint64_t)b};
+  const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)ld * 2 * (uint64_t)s};
+  const uint32_t box[3] = {64, 128, 1};
+  return make_map(m, base, 3, dims, strides, box);
+}
+
+// ------------------------------------------------------------- device info
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int check_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0);
+    d.sms = n;
+    if (d.ok) {
+      bool attrs = cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_OUTPROJ>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_FFN_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_FFN_DOWN>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnCfg<64>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnCfg<128>::SMEM_BYTES) == cudaSuccess;
+      if (!attrs) return BPT_ERR_CUDA;
+    }
+    d.checked = true;
+  }
+  if (!d.ok) return BPT_ERR_UNSUPPORTED;
+  *sms = d.sms;
+  return BPT_OK;
+}
+
+// ------------------------------------------------------------- argument checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo < a.hi && b.lo < b.hi; }
+Range rng(const void* p, size_t bytes) {
+  return Range{reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + bytes};
+}
+
+int check_shape(int b, int s, int h, int heads) {
+  if (b < 0 || s < 0 || h <= 0 || heads <= 0) return BPT_ERR_SHAPE;
+  if (h % heads) return BPT_ERR_SHAPE;
+  const int dh = h / heads;
+  if (dh != 64 && dh != 128) return BPT_ERR_SHAPE;
+  if ((long long)b * s > 0x7fffffffLL) return BPT_ERR_SHAPE;
+  if ((long long)h * 4 > 0x7fffffffLL / 4) return BPT_ERR_SHAPE;
+  return BPT_OK;
+}
+
+int check_blocks(int s, int q_block, int kv_block) {
+  if (s == 0) return BPT_OK;
+  if (q_block <= 0 || kv_block <= 0 || q_block > s || kv_block > s) return BPT_ERR_BLOCK;
+  if (s % q_block || s % kv_block) return BPT_ERR_BLOCK;
+  return BPT_OK;
+}
+
+// ------------------------------------------------------------- wave plan
+struct Wave {
+  long long row0;  // flat row of the wave's first row
+  int beta0, n_seq, t_start, t_len;
+  long long rows() const { return (long long)n_seq * t_len; }
+};
+
+constexpr int kDefaultWaveRows = 4096;
+
+int wave_rows_for(int b, int s, int q_block, int wave_rows) {
+  long long wr = wave_rows > 0 ? wave_rows : kDefaultWaveRows;
+  wr = std::max<long long>(q_block, (wr / q_block) * q_block);
+  if (wr >= s) {
+    const long long g = std::max<long long>(1, std::min<long long>(b, wr / s));
+    return (int)std::min<long long>(g * s, 0x7fffffffLL);
+  }
+  return (int)wr;
+}
+
+std::vector<Wave> plan_waves(int b, int s, int q_block, int wave_rows) {
+  std::vector<Wave> w;
+  const int wr = wave_rows_for(b, s, q_block, wave_rows);
+  if (wr >= s) {
+    const int g = wr / s;
+    for (int beta = 0; beta < b; beta += g) w.push_back(Wave{(long long)beta * s, beta, std::min(g, b - beta), 0, s});
+  } else {
+    for (int beta = 0; beta < b; ++beta)
+      for (int ts = 0; ts < s; ts += wr)
+        w.push_back(Wave{(long long)beta * s + ts, beta, 1, ts, std::min(wr, s - ts)});
+  }
+  return w;
+}
+
+// ------------------------------------------------------------- workspace layout
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+  size_t k, v, hb, ou, xb, wqkv, wo, w1, w2, total;
+  int wave_rows;
+};
+
+Layout layout_for(int dtype, int b, int s, int h, int q_block, int wave_rows) {
+  Layout L{};
+  const size_t tok = (size_t)b * s;
+  const int wr = wave_rows_for(b, s, q_block, wave_rows);
+  L.wave_rows = wr;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes, 1024);
+    return at;
+  };
+  L.k = take(tok * h * 2);
+  L.v = take(tok * h * 2);
+  L.hb = take((size_t)wr * h * 2);
+  L.ou = take((size_t)wr * 4 * h * 2);
+  if (dtype == BPT_DTYPE_F32) {
+    L.xb = take(tok * h * 2);
+    L.wqkv = take((size_t)h * 3 * h * 2);
+    L.wo = take((size_t)h * h * 2);
+    L.w1 = take((size_t)h * 4 * h * 2);
+    L.w2 = take((size_t)4 * h * h * 2);
+  }
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------- launches
+template <int MODE>
+int launch_gemm(const void* A, long long M, long long K, long long lda, const void* B, long long N,
+                GemmArgs args, int sms, cudaStream_t st, const char* name) {
+  if (M <= 0) return BPT_OK;
+  CUtensorMap ta, tb;
+  if (!map_rows(&ta, A, M, K, lda, GEMM_BM)) return BPT_ERR_CUDA;
+  if (!map_rows(&tb, B, K, N, N, 64)) return BPT_ERR_CUDA;
+  args.M = (int)M;
+  args.N = (int)N;
+  args.K = (int)K;
+  args.m_tiles = (int)((M + GEMM_BM - 1) / GEMM_BM);
+  args.n_tiles = (int)((N + GEMM_BN - 1) / GEMM_BN);
+  const int tiles = args.m_tiles * args.n_tiles;
+  const int grid = std::min(tiles, sms);
+  {
+    LaunchScope ls(name, st);
+    gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+// Attention of the query rows [t_start, t_start + t_len) of sequences
+// beta0 .. beta0 + n_seq - 1; q rows have `ldq` elements between them.
+int launch_attention(const void* q, long long ldq, const void* k, const void* v, int b, int s, int h, int heads,
+                     int causal, int beta0, int n_seq, int t_start, int t_len, __nv_bfloat16* o, long long ldo,
+                     cudaStream_t st) {
+  const int dh = h / heads;
+  CUtensorMap tq, tk, tv;
+  if (!map_seq(&tq, q, b, s, h, ldq) || !map_seq(&tk, k, b, s, h, h) || !map_seq(&tv, v, b, s, h, h))
+    return BPT_ERR_CUDA;
+  AttnArgs a{};
+  a.s = s;
+  a.heads = heads;
+  a.causal = causal ? 1 : 0;
+  a.t_start = t_start;
+  a.t_len = t_len;
+  a.n_qtiles = (t_len + ATT_BM - 1) / ATT_BM;
+  a.ldo = ldo;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  for (int z0 = 0; z0 < n_seq; z0 += 65535) {
+    const int nz = std::min(65535, n_seq - z0);
+    a.beta0 = beta0 + z0;
+    a.o = o + (long long)z0 * t_len * ldo;
+    dim3 grid(heads, a.n_qtiles, nz);
+    LaunchScope ls("attention", st);
+    if (dh == 64)
+      attention_fwd_tcgen05<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+    else
+      attention_fwd_tcgen05<128><<<grid, ATT_THREADS, AttnCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, long long n) {
+  const long long n4 = n / 4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 f = reinterpret_cast<const float4*>(src)[i];
+    uint2 o;
+    o.x = pack_bf16x2(f.x, f.y);
+    o.y = pack_bf16x2(f.z, f.w);
+    reinterpret_cast<uint2*>(dst)[i] = o;
+  }
+  for (long long i = n4 * 4 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+int launch_convert(const float* src, void* dst, long long n, int sms, cudaStream_t st) {
+  if (n <= 0) return BPT_OK;
+  const long long blocks = std::min<long long>((n / 4 + 255) / 256 + 1, (long long)sms * 8);
+  LaunchScope ls("f32_to_bf16", st);
+  f32_to_bf16_kernel<<<(int)blocks, 256, 0, st>>>(src, reinterpret_cast<__nv_bfloat16*>(dst), n);
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+#define BPT_TRY(expr)            \
+  do {                           \
+    int _r = (expr);             \
+    if (_r != BPT_OK) return _r; \
+  } while (0)
+
+struct LayerPtrs {
+  const void *x, *Wqkv, *bqkv, *Wo, *bo, *W1, *b1, *W2, *b2;
+};
+
+int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int kv_block,
+                   const float* out) {
+  if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return BPT_ERR_DTYPE;
+  BPT_TRY(check_shape(b, s, h, heads));
+  BPT_TRY(check_blocks(s, q_block, kv_block));
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[10] = {p.x, p.Wqkv, p.bqkv, p.Wo, p.bo, p.W1, p.b1, p.W2, p.b2, out};
+  for (const void* q : ptrs)
+    if (!q) return BPT_ERR_NULL;
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return BPT_ERR_ALIGN;
+  const size_t es = dtype == BPT_DTYPE_F32 ? 4 : 2;
+  const size_t tok = (size_t)b * s;
+  const Range ro = rng(out, tok * h * 4);
+  const Range in[9] = {rng(p.x, tok * h * es),      rng(p.Wqkv, (size_t)h * 3 * h * es), rng(p.bqkv, 3 * (size_t)h * es),
+                       rng(p.Wo, (size_t)h * h * es), rng(p.bo, (size_t)h * es),          rng(p.W1, (size_t)h * 4 * h * es),
+                       rng(p.b1, 4 * (size_t)h * es), rng(p.W2, (size_t)4 * h * h * es),    rng(p.b2, (size_t)h * es)};
+  for (const Range& r : in)
+    if (overlap(ro, r)) return BPT_ERR_ALIAS;
+  return BPT_OK;
+}
+
+int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int causal,
+              int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms) {
+  const Layout L = layout_for(dtype, b, s, h, q_block, wave_rows);
+  const long long tok = (long long)b * s;
+  __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(ws + L.k);
+  __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(ws + L.v);
+  __nv_bfloat16* HB = reinterpret_cast<__nv_bfloat16*>(ws + L.hb);
+  __nv_bfloat16* OU = reinterpret_cast<__nv_bfloat16*>(ws + L.ou);
+  __nv_bfloat16* Q = reinterpret_cast<__nv_bfloat16*>(out);  // bf16 row r at out row r
+  const long long ldq = 2LL * h;
+
+  const void *xa = p.x, *wqkv = p.Wqkv, *wo = p.Wo, *w1 = p.W1, *w2 = p.W2;
+  const int f32 = dtype == BPT_DTYPE_F32 ? 1 : 0;
+  if (f32) {
+    BPT_TRY(launch_convert((const float*)p.x, ws + L.xb, tok * h, sms, st));
+    BPT_TRY(launch_convert((const float*)p.Wqkv, ws + L.wqkv, 3LL * h * h, sms, st));
+    BPT_TRY(launch_convert((const float*)p.Wo, ws + L.wo, 1LL * h * h, sms, st));
+    BPT_TRY(launch_convert((const float*)p.W1, ws + L.w1, 4LL * h * h, sms, st));
+    BPT_TRY(launch_convert((const float*)p.W2, ws + L.w2, 4LL * h * h, sms, st));
+    xa = ws + L.xb;
+    wqkv = ws + L.wqkv;
+    wo = ws + L.wo;
+    w1 = ws + L.w1;
+    w2 = ws + L.w2;
+  }
+
+  // step 1: projection of the whole sequence
+  {
+    GemmArgs a{};
+    a.bias = p.bqkv;
+    a.bias_f32 = f32;
+    a.q = Q;
+    a.ldq = ldq;
+    a.k = K;
+    a.v = V;
+    a.ldkv = h;
+    a.h = h;
+    BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, "gemm_qkv"));
+  }
+
+  // steps 4-11 per wave of query blocks
+  for (const Wave& w : plan_waves(b, s, q_block, wave_rows)) {
+    const long long rows = w.rows();
+    BPT_TRY(launch_attention(Q, ldq, K, V, b, s, h, heads, causal, w.beta0, w.n_seq, w.t_start, w.t_len, OU, h, st));
+    GemmArgs a{};
+    a.resid = p.x;
+    a.resid_f32 = f32;
+    a.ld_resid = h;
+    a.out = out;
+    a.ld_out = h;
+    a.row0 = w.row0;
+    a.bias_f32 = f32;
+    a.bias = p.bo;
+    a.dst = HB;
+    a.ld_dst = h;
+    BPT_TRY(launch_gemm<EPI_OUTPROJ>(OU, rows, h, h, wo, h, a, sms, st, "gemm_outproj"));
+    a.bias = p.b1;
+    a.dst = OU;
+    a.ld_dst = 4LL * h;
+    BPT_TRY(launch_gemm<EPI_FFN_UP>(HB, rows, h, h, w1, 4LL * h, a, sms, st, "gemm_ffn_up"));
+    a.bias = p.b2;
+    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(OU, rows, 4LL * h, 4LL * h, w2, h, a, sms, st, "gemm_ffn_down"));
+  }
+  return BPT_OK;
+}
+
+int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
+                int wave_rows, void* workspace, size_t ws_bytes, bool caller_ws, float* out, void* stream) {
+  BPT_TRY(validate_layer(dtype, p, b, s, h, heads, q_block, kv_block, out));
+  if ((long long)b * s == 0) return BPT_OK;
+  const Layout L = layout_for(dtype, b, s, h, q_block, wave_rows);
+  if (caller_ws) {
+    if (!workspace) return BPT_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BPT_ERR_ALIGN;
+    if (ws_bytes < L.total) return BPT_ERR_NOMEM;
+    const size_t es = dtype == BPT_DTYPE_F32 ? 4 : 2;
+    const size_t tok = (size_t)b * s;
+    const Range rw = rng(workspace, L.total);
+    const Range others[10] = {rng(out, tok * h * 4),      rng(p.x, tok * h * es),        rng(p.Wqkv, (size_t)3 * h * h * es),
+                              rng(p.bqkv, (size_t)3 * h * es), rng(p.Wo, (size_t)h * h * es), rng(p.bo, (size_t)h * es),
+                              rng(p.W1, (size_t)4 * h * h * es), rng(p.b1, (size_t)4 * h * es), rng(p.W2, (size_t)4 * h * h * es),
+                              rng(p.b2, (size_t)h * es)};
+    for (const Range& r : others)
+      if (overlap(rw, r)) return BPT_ERR_ALIAS;
+  }
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (!caller_ws) {
+    void* m = nullptr;
+    if (cudaMallocAsync(&m, L.total, st) != cudaSuccess) {
+      cudaGetLastError();
+      return BPT_ERR_NOMEM;
+    }
+    ws = reinterpret_cast<uint8_t*>(m);
+  }
+  const int r = run_layer(dtype, p, b, s, h, heads, q_block, causal, wave_rows, ws, out, st, sms);
+  if (!caller_ws) cudaFreeAsync(ws, st);
+  return r;
+}
+
+}  // namespace
+}  // namespace bpt
+
+using namespace bpt;
+
+extern "C" {
+
+const char* bpt_status_string(int status) {
+  switch (status) {
+    case BPT_OK: return "BPT_OK";
+    case BPT_ERR_NULL: return "BPT_ERR_NULL: a required pointer is NULL";
+    case BPT_ERR_SHAPE: return "BPT_ERR_SHAPE: bad b, s, h or heads (dh = h/heads must be 64 or 128)";
+    case BPT_ERR_BLOCK: return "BPT_ERR_BLOCK: q_block/kv_block must be in [1, s] and divide s";
+    case BPT_ERR_ALIGN: return "BPT_ERR_ALIGN: pointers must be 16-byte aligned (workspace 256-byte)";
+    case BPT_ERR_ALIAS: return "BPT_ERR_ALIAS: out or workspace overlaps another argument";
+    case BPT_ERR_NOMEM: return "BPT_ERR_NOMEM: workspace allocation failed or ws_bytes too small";
+    case BPT_ERR_CUDA: return "BPT_ERR_CUDA: a CUDA call failed";
+    case BPT_ERR_TIMEOUT: return "BPT_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case BPT_ERR_UNSUPPORTED: return "BPT_ERR_UNSUPPORTED: the current device is not sm_100";
+    case BPT_ERR_DTYPE: return "BPT_ERR_DTYPE: unknown dtype";
+    default: return "unknown bpt status";
+  }
+}
+
+int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                      const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                      int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  return layer_entry(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, kv_block, causal, 0, nullptr, 0, false, out, stream);
+}
+
+int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, const float* Wo, const float* bo,
+                          const float* W1, const float* b1, const float* W2, const float* b2, int b, int s, int h,
+                          int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  return layer_entry(BPT_DTYPE_F32, p, b, s, h, heads, q_block, kv_block, causal, 0, nullptr, 0, false, out, stream);
+}
+
+size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
+                                 int wave_rows) {
+  if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return 0;
+  if (check_shape(b, s, h, heads) != BPT_OK || check_blocks(s, q_block, kv_block) != BPT_OK) return 0;
+  if ((long long)b * s == 0) return 0;
+  return layout_for(dtype, b, s, h, q_block, wave_rows).total;
+}
+
+int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
+                         const void* bo, const void* W1, const void* b1, const void* W2, const void* b2, int b,
+                         int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
+                         void* workspace, size_t ws_bytes, float* out, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  return layer_entry(dtype, p, b, s, h, heads, q_block, kv_block, causal, wave_rows, workspace, ws_bytes, true, out,
+                     stream);
+}
+
+int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,
+                       void* v, void* stream) {
+  if (b < 0 || s < 0 || h <= 0 || h % 64 || (long long)b * s > 0x7fffffffLL) return BPT_ERR_SHAPE;
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[6] = {x, Wqkv, bqkv, q, k, v};
+  for (const void* p : ptrs)
+    if (!p) return BPT_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return BPT_ERR_ALIGN;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  GemmArgs a{};
+  a.bias = bqkv;
+  a.q = reinterpret_cast<__nv_bfloat16*>(q);
+  a.ldq = h;
+  a.k = reinterpret_cast<__nv_bfloat16*>(k);
+  a.v = reinterpret_cast<__nv_bfloat16*>(v);
+  a.ldkv = h;
+  a.h = h;
+  return launch_gemm<EPI_QKV>(x, (long long)b * s, h, h, Wqkv, 3LL * h, a, sms,
+                              reinterpret_cast<cudaStream_t>(stream), "gemm_qkv");
+}
+
+int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int q_block,
+                  int kv_block, int causal, void* o, void* stream) {
+  BPT_TRY(check_shape(b, s, h, heads));
+  BPT_TRY(check_blocks(s, q_block, kv_block));
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[4] = {q, k, v, o};
+  for (const void* p : ptrs)
+    if (!p) return BPT_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return BPT_ERR_ALIGN;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  return launch_attention(q, h, k, v, b, s, h, heads, causal, 0, b, 0, s, reinterpret_cast<__nv_bfloat16*>(o), h,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bpt_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return BPT_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return BPT_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BPT_ERR_CUDA;
+  return v;
+}
+
+uint64_t bpt_launch_count(void) { return g_launches.load(); }
+
+int bpt_set_kernel_timing(int enable) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  g_timing = enable != 0;
+  return BPT_OK;
+}
+
+int bpt_kernel_times(bpt_kernel_time* out, int max) {
+  std::vector<TimedLaunch> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    recs.swap(g_timed);
+  }
+  std::map<std::string, std::pair<int, double>> agg;
+  std::vector<std::string> order;
+  int rc = BPT_OK;
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+      rc = BPT_ERR_CUDA;
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+    auto it = agg.find(r.name);
+    if (it == agg.end()) {
+      order.push_back(r.name);
+      agg[r.name] = {1, ms};
+    } else {
+      it->second.first += 1;
+      it->second.second += ms;
+    }
+  }
+  if (rc != BPT_OK) return rc;
+  int n = 0;
+  for (const auto& name : order) {
+    if (n >= max || !out) break;
+    std::memset(out[n].name, 0, sizeof(out[n].name));
+    std::strncpy(out[n].name, name.c_str(), sizeof(out[n].name) - 1);
+    out[n].launches = agg[name].first;
+    out[n].total_ms = agg[name].second;
+    ++n;
+  }
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,306 @@
+// Persistent tcgen05 GEMM with fused epilogues for the projections of the BPT
+// layer: D[M, N] = A[M, K] * B[K, N] with A bf16 row-major (K-major operand),
+// B bf16 row-major [in, out] weights (MN-major operand), fp32 accumulation in
+// tensor memory.
+//
+// Roles (192 threads): warp 0 issues TMA tile loads into a STAGES-deep ring,
+// one thread of warp 1 issues tcgen05.mma into one of two TMEM accumulators,
+// warps 2-5 read the finished accumulator (warp w owns TMEM lanes
+// 32*(w%4) .. +31, one output row per thread) and run the epilogue while the
+// next tile's MMAs proceed into the other accumulator.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace bpt {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB, one 128B-swizzle atom column
+constexpr int GEMM_B_BOX_BYTES = GEMM_BK * 64 * 2;   // 8 KB: 64 K-rows x 64 N-columns
+constexpr int GEMM_B_BYTES = GEMM_BK * GEMM_BN * 2;  // 32 KB: four boxes along N
+constexpr int GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
+constexpr int GEMM_TMEM_COLS = 2 * GEMM_BN;          // two fp32 accumulators
+constexpr int GEMM_GROUP_M = 16;                     // raster: 16 M-tiles share B tiles in L2
+constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + 256;
+
+enum EpiMode {
+  EPI_QKV = 0,       // + bqkv -> bf16 Q | K | V
+  EPI_OUTPROJ = 1,   // + bo + x (first residual) -> fp32 hid into out, bf16 copy for the FFN
+  EPI_FFN_UP = 2,    // + b1, ReLU -> bf16 U
+  EPI_FFN_DOWN = 3,  // + b2 + hid (second residual, read from out) -> fp32 out
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int m_tiles, n_tiles;
+  const void* bias;  // [N], bf16 or fp32
+  int bias_f32;
+  // EPI_QKV
+  __nv_bfloat16* q;
+  long long ldq;     // elements between Q rows
+  __nv_bfloat16* k;
+  __nv_bfloat16* v;
+  long long ldkv;
+  int h;
+  // EPI_OUTPROJ residual input x
+  const void* resid;
+  int resid_f32;
+  long long ld_resid;
+  // fp32 out (OUTPROJ writes hid, FFN_DOWN reads hid and writes the result)
+  float* out;
+  long long ld_out;
+  long long row0;    // flat row of local row 0 (for x and out)
+  // bf16 destination of OUTPROJ (hid copy) and FFN_UP (U)
+  __nv_bfloat16* dst;
+  long long ld_dst;
+};
+
+__device__ __forceinline__ float load_vec_elem(const void* p, int f32, long long i) {
+  return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+// 32 consecutive values (columns col .. col+31) of one row.
+__device__ __forceinline__ void load32(const void* p, int f32, long long off, float (&v)[32]) {
+  if (f32) {
+    const float4* s = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + off);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 t = s[i];
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 t = s[i];
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+        float2 f = __bfloat1622float2(b2);
+        v[8 * i + 2 * j] = f.x;
+        v[8 * i + 2 * j + 1] = f.y;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    st_global_v4(dst + 8 * i, pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                 pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+__device__ __forceinline__ void store32_f32(float* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    st_global_v4(dst + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]), __float_as_uint(v[4 * i + 2]),
+                 __float_as_uint(v[4 * i + 3]));
+}
+
+template <int MODE>
+__device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int col, float (&v)[32]) {
+  float bias[32];
+  load32(a.bias, a.bias_f32, col, bias);
+  if constexpr (MODE == EPI_QKV) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += bias[i];
+    const int part = col / a.h;
+    const int c = col - part * a.h;
+    __nv_bfloat16* dst = part == 0 ? a.q + (long long)row * a.ldq + c
+                                   : (part == 1 ? a.k : a.v) + (long long)row * a.ldkv + c;
+    store32_bf16(dst, v);
+  } else if constexpr (MODE == EPI_OUTPROJ) {
+    float x[32];
+    const long long grow = a.row0 + row;
+    load32(a.resid, a.resid_f32, grow * a.ld_resid + col, x);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += bias[i] + x[i];
+    store32_f32(a.out + grow * a.ld_out + col, v);
+    store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
+  } else if constexpr (MODE == EPI_FFN_UP) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i] + bias[i], 0.0f);
+    store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
+  } else {
+    float hid[32];
+    const long long grow = a.row0 + row;
+    float* o = a.out + grow * a.ld_out + col;
+    load32(o, 1, 0, hid);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += bias[i] + hid[i];
+    store32_f32(o, v);
+  }
+}
+
+__device__ __forceinline__ void gemm_tile_coords(int t, int m_tiles, int n_tiles, int& mt, int& nt) {
+  const int group_size = GEMM_GROUP_M * n_tiles;
+  const int group = t / group_size;
+  const int first_m = group * GEMM_GROUP_M;
+  const int gm = min(GEMM_GROUP_M, m_tiles - first_m);
+  const int r = t - group * group_size;
+  mt = first_m + r % gm;
+  nt = r / gm;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
+  // barrier slots
+  const uint32_t full0 = smem_addr(bars);
+  const uint32_t empty0 = smem_addr(bars + GEMM_STAGES);
+  const uint32_t tfull0 = smem_addr(bars + 2 * GEMM_STAGES);
+  const uint32_t tempty0 = smem_addr(bars + 2 * GEMM_STAGES + 2);
+  const uint32_t mma_done = smem_addr(bars + 2 * GEMM_STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * GEMM_STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * GEMM_STAGES + 6);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const uint32_t smem_base = smem_addr(smem);
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < GEMM_STAGES; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), GEMM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = args.m_tiles * args.n_tiles;
+  const int k_blocks = args.K / GEMM_BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_parity = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        int mt, nt;
+        gemm_tile_coords(t, args.m_tiles, args.n_tiles, mt, nt);
+        const int m0 = mt * GEMM_BM, n0 = nt * GEMM_BN;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag)) goto producer_done;
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t sa = smem_base + stage * GEMM_STAGE_BYTES;
+          mbar_arrive_expect_tx(fb, GEMM_STAGE_BYTES);
+          tma_load_2d(sa, &tmA, fb, kb * GEMM_BK, m0);
+#pragma unroll
+          for (int j = 0; j < GEMM_BN / 64; ++j)
+            tma_load_2d(sa + GEMM_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);
+          issued |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    producer_done:
+      // never leave with tile copies still landing in shared memory
+      for (int i = 0; i < GEMM_STAGES; ++i)
+        if (issued & (1u << i)) {
+          volatile int dummy = 0;
+          mbar_wait(full0 + 8 * i, (last_parity >> i) & 1u, &dummy);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, 0, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * GEMM_BN;
+        bool ok = true;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + stage * GEMM_STAGE_BYTES;
+          const uint32_t sb = sa + GEMM_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(sb + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024);
+            mma_bf16_ss(d, adesc, bdesc, idesc, (kb | kk) != 0);
+          }
+          mma_commit(empty0 + 8 * stage);
+          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8 * acc);
+      }
+      mma_commit(mma_done);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      int mt, nt;
+      gemm_tile_coords(t, args.m_tiles, args.n_tiles, mt, nt);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!warp_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int row = mt * GEMM_BM + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + acc * GEMM_BN + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < GEMM_BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_load32(taddr + c * 32, r);
+        const int col = nt * GEMM_BN + c * 32;
+        if (row < args.M && col < args.N) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          gemm_epilogue<MODE>(args, row, col, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      volatile int dummy = 0;
+      mbar_wait(mma_done, 0, &dummy);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+}  // namespace bpt

@@ -204,3 +204,19 @@ SWEEP_BLOCKS = (64, 128, 256, 512, 1024, 2048)
 def sweep_shape(block: int, causal: bool) -> LayerShape:
     """Block-size sweep point: b 1, s 16384, h 2048, 16 heads of 128."""
     return LayerShape(1, 16384, 2048, 16, block, block, causal)
+
+
+def to_torch(a: np.ndarray, device="cuda"):
+    """A generated tensor as a torch tensor (bf16 for bit patterns, else fp32)."""
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+PARAM_NAMES = ("Wqkv", "bqkv", "Wo", "bo", "W1", "b1", "W2", "b2")
+
+
+def oracle_args(inp: dict) -> tuple:
+    """(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2) as exact fp64 arrays."""
+    return tuple(to_f64(inp[k]) for k in ("x",) + PARAM_NAMES)

@@ -1,0 +1,163 @@
+/*
+ * bpt.h - C ABI of the B200 (sm_100a) Blockwise Parallel Transformer layer forward.
+ *
+ * One call computes, for every query block Q_i of the sequence, exact
+ * multi-head attention over all key/value blocks with a running max and
+ * running sum (online-softmax rescaling), then the output projection, the
+ * first residual, the position-wise FFN max(0, y W1 + b1) W2 + b2 and the
+ * second residual:
+ *
+ *     [Q | K | V] = x Wqkv + bqkv
+ *     O_i         = concat_k softmax(Q_i,k K_k^T / sqrt(dh)) V_k      (per head k)
+ *     hid_i       = x_i + O_i Wo + bo
+ *     out_i       = hid_i + max(0, hid_i W1 + b1) W2 + b2
+ *
+ * Sources: "Blockwise Parallel Transformer for Large Context Models" (paper
+ * review of arXiv:2305.19370), section 3: core formulas (standard attention,
+ * standard FFN, Eq. 3 blockwise attention and its scaling operation, the
+ * blockwise FFN with residuals) and Algorithm 1 (input sequence x, query block
+ * count B_q, key/value block count B_kv). Head split and concatenation follow
+ * "PyTorch 2.3 multi-head self-attention from QKV to 8 heads", sections 2-4;
+ * the fused QKV projection follows "Transformer QKV matrix computation and 3
+ * parallel strategies", section 2.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are CUDA device pointers owned by the caller unless a
+ *   function says otherwise. The library keeps no pointer after a call returns
+ *   (work it queued on the stream still reads them until it completes).
+ * - Layouts are row-major. x and out are [b, s, h] (token-major). Weights are
+ *   [in, out] so that a projection reads x W: Wqkv [h, 3h] with columns
+ *   [W_Q | W_K | W_V] and head k of each third in columns k*dh .. k*dh+dh-1;
+ *   Wo [h, h]; W1 [h, 4h]; W2 [4h, h]. Biases are vectors of the output width.
+ * - bf16 entry points take bf16 x, weights and biases. The f32 entry points
+ *   take fp32 x, weights and biases; their matrix products round operands to
+ *   bf16 (fp32 accumulation) while the residual and bias additions use the
+ *   fp32 values.
+ * - out is fp32 [b, s, h]. It is written entirely and is also used as scratch
+ *   during the call (it must not overlap any input).
+ * - Shapes: b >= 0, s >= 0 (b*s == 0 is a no-op), h = heads * dh with
+ *   dh in {64, 128}, b*s <= 2^31 - 1. The FFN width is fixed at 4h.
+ * - Blocks: 1 <= q_block <= s, 1 <= kv_block <= s, s % q_block == 0,
+ *   s % kv_block == 0 (equal-length blocks). The result does not depend on the
+ *   block sizes (the blockwise computation is exact); q_block sets the rows of
+ *   each FFN wave, which is a whole number of query blocks.
+ * - causal != 0: key u is visible to query t iff u <= t in the same sequence.
+ * - Pointers must be 16-byte aligned (tensor-memory-access tiles).
+ * - Errors: argument errors return a negative bpt_status synchronously, with
+ *   nothing launched and nothing written. Otherwise the call is asynchronous on
+ *   `stream` (a cudaStream_t; NULL means the legacy default stream) and
+ *   returns BPT_OK once all kernels are queued. Device-side failures (a
+ *   bounded wait that gave up) are reported by bpt_device_status().
+ * - Reentrancy: calls on different streams may run concurrently; the only
+ *   process-wide state is the device error word, the launch counter and the
+ *   optional kernel timing log.
+ */
+#ifndef BPT_H_
+#define BPT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bpt_status {
+  BPT_OK = 0,
+  BPT_ERR_NULL = -1,        /* a required pointer is NULL */
+  BPT_ERR_SHAPE = -2,       /* b, s, h, heads out of range; h % heads; dh not 64 or 128 */
+  BPT_ERR_BLOCK = -3,       /* q_block / kv_block <= 0, > s, or not dividing s */
+  BPT_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned */
+  BPT_ERR_ALIAS = -5,       /* out overlaps an input, or workspace overlaps out or an input */
+  BPT_ERR_NOMEM = -6,       /* workspace allocation failed, or ws_bytes too small */
+  BPT_ERR_CUDA = -7,        /* a CUDA runtime / driver call failed */
+  BPT_ERR_TIMEOUT = -8,     /* a kernel gave up a bounded wait (device-side) */
+  BPT_ERR_UNSUPPORTED = -9, /* the current device is not sm_100 */
+  BPT_ERR_DTYPE = -10       /* unknown dtype code */
+} bpt_status;
+
+typedef enum bpt_dtype {
+  BPT_DTYPE_BF16 = 0,
+  BPT_DTYPE_F32 = 1
+} bpt_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bpt_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * The layer forward (Algorithm 1 of the BPT paper review, section 3).
+ * ------------------------------------------------------------------------ */
+
+/* bf16 inputs. Allocates its workspace stream-ordered (cudaMallocAsync on
+ * `stream`) and frees it stream-ordered after the last kernel; returns
+ * BPT_ERR_NOMEM if that allocation fails. */
+int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                      const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                      int heads, int q_block, int kv_block, int causal, float* out, void* stream);
+
+/* fp32 inputs (same arguments, fp32 tensors). */
+int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, const float* Wo, const float* bo,
+                          const float* W1, const float* b1, const float* W2, const float* b2, int b, int s, int h,
+                          int heads, int q_block, int kv_block, int causal, float* out, void* stream);
+
+/* Bytes of workspace a caller must pass to bpt_layer_forward_ws for these
+ * arguments (0 if they are invalid or b*s == 0). wave_rows <= 0 selects the
+ * library's default FFN wave (a whole number of query blocks, about 4096 rows);
+ * otherwise it is rounded down to a multiple of q_block (at least q_block). */
+size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
+                                 int wave_rows);
+
+/* The layer with a caller-owned workspace (device memory, 256-byte aligned,
+ * at least bpt_layer_workspace_bytes(...) bytes, not overlapping any argument;
+ * BPT_ERR_NOMEM if ws_bytes is too small). dtype is a bpt_dtype and gives the
+ * element type of x, the weights and the biases. Allocates nothing. */
+int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
+                         const void* bo, const void* W1, const void* b1, const void* W2, const void* b2, int b,
+                         int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
+                         void* workspace, size_t ws_bytes, float* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Single steps of Algorithm 1, for checking intermediate results.
+ * ------------------------------------------------------------------------ */
+
+/* Step 1: [Q | K | V] = x Wqkv + bqkv with bf16 x [b*s, h], Wqkv [h, 3h],
+ * bqkv [3h]; writes bf16 q, k, v, each [b*s, h] row-major. */
+int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,
+                       void* v, void* stream);
+
+/* Steps 2-10: O = concat_k softmax(Q_k K_k^T / sqrt(dh)) V_k over all key
+ * blocks with online-softmax rescaling; bf16 q, k, v [b, s, h] in, bf16 o
+ * [b, s, h] out. q_block / kv_block are validated as for the layer. */
+int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int q_block,
+                  int kv_block, int causal, void* o, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Status and measurement.
+ * ------------------------------------------------------------------------ */
+
+/* Synchronise the current device, return the device error word (BPT_OK or
+ * BPT_ERR_TIMEOUT) and reset it to BPT_OK. BPT_ERR_CUDA if the sync failed. */
+int bpt_device_status(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t bpt_launch_count(void);
+
+/* Kernel timing log: while enabled, every launch is bracketed by CUDA events
+ * recorded on its own stream. bpt_kernel_times synchronises and writes, for at
+ * most `max` kernel kinds, the name, launch count and summed milliseconds,
+ * then clears the log; it returns the number of kinds written. */
+typedef struct bpt_kernel_time {
+  char name[32];
+  int launches;
+  double total_ms;
+} bpt_kernel_time;
+
+int bpt_set_kernel_timing(int enable);
+int bpt_kernel_times(bpt_kernel_time* out, int max);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BPT_H_ */

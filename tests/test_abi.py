@@ -1,0 +1,146 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/bpt.h declares, and rejects bad arguments synchronously (argument
+checks run before any CUDA call, so these run on a CPU-only machine)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import blockwise_attn_ffn_bpt_b200 as bpt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bpt.h")
+
+OK, NULL, SHAPE, BLOCK, ALIGN, ALIAS, NOMEM, DTYPE = 0, -1, -2, -3, -4, -5, -6, -10
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bpt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    L = bpt.lib()
+    names = declared_functions()
+    assert "bpt_layer_forward" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in bpt.h but not exported"
+    assert set(bpt.EXPORTED) == set(names)
+
+
+def test_status_strings():
+    for code in (OK, NULL, SHAPE, BLOCK, ALIGN, ALIAS, NOMEM, -7, -8, -9, DTYPE):
+        assert bpt.status_string(code).startswith("BPT_")
+    assert bpt.status_string(12345) == "unknown bpt status"
+
+
+# fake, aligned, non-overlapping "device" addresses: the checks fail before any are used
+BASE = 1 << 40
+STEP = 1 << 36
+
+
+def fake_ptrs(n):
+    return [BASE + i * STEP for i in range(n)]
+
+
+def call_layer(b=1, s=256, h=256, heads=4, qb=64, kb=64, causal=0, ptrs=None, out=None):
+    p = ptrs or fake_ptrs(9)
+    o = out if out is not None else BASE + 20 * STEP
+    return bpt.lib().bpt_layer_forward(*p, b, s, h, heads, qb, kb, causal, o, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(h=256, heads=3), SHAPE),          # h % heads
+    (dict(h=256, heads=8), SHAPE),          # dh = 32
+    (dict(h=512, heads=2), SHAPE),          # dh = 256
+    (dict(b=-1), SHAPE),
+    (dict(s=-5), SHAPE),
+    (dict(qb=0), BLOCK),
+    (dict(qb=48), BLOCK),                   # 256 % 48
+    (dict(kb=512), BLOCK),                  # > s
+    (dict(kb=-64), BLOCK),
+])
+def test_layer_rejects_bad_shapes(kw, code):
+    assert call_layer(**kw) == code
+
+
+def test_empty_problem_is_a_noop():
+    assert call_layer(b=0) == OK
+    assert call_layer(s=0, qb=1, kb=1) == OK
+    # empty problems need no pointers at all
+    assert bpt.lib().bpt_layer_forward(*([None] * 9), 0, 128, 256, 4, 64, 64, 1, None, None) == OK
+
+
+def test_layer_rejects_null_and_misaligned_pointers():
+    p = fake_ptrs(9)
+    for i in range(9):
+        q = list(p)
+        q[i] = None
+        assert call_layer(ptrs=q) == NULL
+        q[i] = p[i] + 8
+        assert call_layer(ptrs=q) == ALIGN
+    assert bpt.lib().bpt_layer_forward(*p, 1, 256, 256, 4, 64, 64, 0, None, None) == NULL
+
+
+def test_layer_rejects_out_overlapping_an_input():
+    p = fake_ptrs(9)
+    assert call_layer(ptrs=p, out=p[0] + 256) == ALIAS      # inside x
+    assert call_layer(ptrs=p, out=p[5] - 1024) == ALIAS     # runs into W1
+
+
+def test_ws_entry_checks_dtype_and_workspace():
+    L = bpt.lib()
+    p = fake_ptrs(9)
+    out = BASE + 20 * STEP
+    ws = BASE + 30 * STEP
+    need = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)
+    args = [1, 256, 256, 4, 64, 64, 1, 0]
+    assert L.bpt_layer_forward_ws(7, *p, *args, ws, need, out, None) == DTYPE
+    assert L.bpt_layer_forward_ws(0, *p, *args, None, need, out, None) == NULL
+    assert L.bpt_layer_forward_ws(0, *p, *args, ws + 16, need, out, None) == ALIGN
+    assert L.bpt_layer_forward_ws(0, *p, *args, ws, need - 1, out, None) == NOMEM
+    assert L.bpt_layer_forward_ws(0, *p, *args, p[3], need, out, None) == ALIAS
+
+
+def test_workspace_bytes_follow_the_layout():
+    # bf16: K and V for the whole sequence, plus per-wave bf16 hid copy and the
+    # O / U scratch (wave rows x 5h bf16), each region rounded up to 1 KiB
+    def up(v):
+        return (v + 1023) // 1024 * 1024
+    b, s, h = 1, 32768, 4096
+    ws = bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048)
+    wr = 4096
+    assert ws == up(b * s * h * 2) * 2 + up(wr * h * 2) + up(wr * 4 * h * 2)
+    # element ratio against 2bsh stays within 1.5
+    assert ws / 2 / (2 * b * s * h) <= 1.5
+    # wave rows are whole query blocks; a whole-sequence wave covers whole sequences
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == \
+        up(2 * 2048 * 1024 * 2) * 2 + up(4096 * 1024 * 2) + up(4096 * 4096 * 2)
+    assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == \
+        up(16384 * 2048 * 2) * 2 + up(2048 * 2048 * 2) + up(2048 * 4 * 2048 * 2)
+    # fp32 inputs add bf16 copies of x and the weights
+    f = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
+    g = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)
+    assert f == g + up(256 * 256 * 2) + up(3 * 256 * 256 * 2) + up(256 * 256 * 2) + 2 * up(4 * 256 * 256 * 2)
+    assert bpt.workspace_bytes(0, 1, 256, 256, 3, 64, 64) == 0
+    assert bpt.workspace_bytes(0, 0, 256, 256, 4, 64, 64) == 0
+
+
+def test_stage_entry_points_validate():
+    L = bpt.lib()
+    p = fake_ptrs(6)
+    assert L.bpt_qkv_projection(p[0], p[1], p[2], 1, 128, 100, p[3], p[4], p[5], None) == SHAPE
+    assert L.bpt_qkv_projection(p[0], None, p[2], 1, 128, 128, p[3], p[4], p[5], None) == NULL
+    assert L.bpt_attention(p[0], p[1], p[2], 1, 128, 256, 2, 128, 64, 1, None, None) == NULL
+    assert L.bpt_attention(p[0], p[1], p[2], 1, 128, 256, 2, 96, 64, 1, p[3], None) == BLOCK
+    assert L.bpt_attention(p[0], p[1], p[2] + 4, 1, 128, 256, 2, 64, 64, 1, p[3], None) == ALIGN
+
+
+def test_kernel_timing_log_is_empty_without_launches():
+    bpt.set_kernel_timing(True)
+    assert bpt.kernel_times() == {}
+    bpt.set_kernel_timing(False)
+    assert bpt.launch_count() >= 0

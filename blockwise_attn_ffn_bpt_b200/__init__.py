@@ -22,7 +22,7 @@ BPT_DTYPE_F32 = 1
 
 EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
-    "bpt_layer_forward_ws", "bpt_qkv_projection", "bpt_attention", "bpt_device_status",
+    "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_qkv_projection", "bpt_attention", "bpt_device_status",
     "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
 )
 

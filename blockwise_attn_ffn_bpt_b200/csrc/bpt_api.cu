@@ -468,6 +468,32 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
   return r;
 }
 
+// Scratch of bpt_layer_forward_noalloc: one fixed array in device memory,
+// created with the library image on every device that loads it. In host code
+// the name g_static_ws denotes a host-side stand-in, never the device address:
+// the address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_ws[BPT_STATIC_WORKSPACE_BYTES];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {};
+
+// Device address of g_static_ws on the current device (looked up once per device).
+int static_workspace(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return BPT_ERR_CUDA;
+    }
+    g_static_ptr[dev] = p;
+  }
+  *ptr = g_static_ptr[dev];
+  return BPT_OK;
+}
+
 }  // namespace
 }  // namespace bpt
 
@@ -521,6 +547,22 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
   const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
   return layer_entry(dtype, p, b, s, h, heads, q_block, kv_block, causal, wave_rows, workspace, ws_bytes, true, out,
                      stream);
+}
+
+int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                              const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                              int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  BPT_TRY(validate_layer(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, kv_block, out));
+  if ((long long)b * s == 0) return BPT_OK;
+  const Layout L = layout_for(BPT_DTYPE_BF16, b, s, h, q_block, 0);
+  if (L.total > BPT_STATIC_WORKSPACE_BYTES) return BPT_ERR_NOMEM;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  void* ws = nullptr;
+  BPT_TRY(static_workspace(&ws));
+  return run_layer(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, causal, 0, reinterpret_cast<uint8_t*>(ws), out,
+                   reinterpret_cast<cudaStream_t>(stream), sms);
 }
 
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,

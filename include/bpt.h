@@ -117,6 +117,38 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
                          int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
                          void* workspace, size_t ws_bytes, float* out, void* stream);
 
+/* Allocation-free variant of bpt_layer_forward (bf16 inputs, same arguments
+ * and result). The paper has no counterpart: this entry point exists for
+ * callers that cannot call cudaMalloc (or any allocator) while they run, for
+ * example code executing inside an inference engine's enqueue/execute hook
+ * where allocating is forbidden, or a process whose device memory is reserved
+ * up front by another memory manager, and that also cannot lend the library a
+ * workspace buffer. Its scratch is one fixed array of
+ * BPT_STATIC_WORKSPACE_BYTES in the library's device memory: every GPU on
+ * which the library is loaded holds that array until the process exits.
+ *
+ * - Allocates nothing: no cudaMalloc / cudaMallocAsync / cudaFree, and no
+ *   allocating library routine. The caller still owns x, the weights, the
+ *   biases and out.
+ * - Size limit: returns BPT_ERR_NOMEM, with nothing launched, when the
+ *   workspace the layer needs (bpt_layer_workspace_bytes(BPT_DTYPE_BF16, b, s,
+ *   h, heads, q_block, kv_block, 0)) exceeds BPT_STATIC_WORKSPACE_BYTES; for
+ *   example b=2, s=2048, h=1024 needs 56 MiB and fits, s=8192, h=2048 does not.
+ * - The first call on each device looks up that device's address of the array
+ *   (one cudaGetSymbolAddress, with that device current). Make that first call
+ *   before any stream capture on the device.
+ * - Every call on a device uses the same array, and it keeps whatever the last
+ *   call left in it. No part of it needs to start at zero: each byte a call
+ *   reads was written earlier in the same call. Calls whose work overlaps on
+ *   the GPU (different streams, or different host threads, without ordering
+ *   between them) race on the array and corrupt each other's results; order
+ *   them on one stream or with events. */
+#define BPT_STATIC_WORKSPACE_BYTES ((size_t)64 << 20)
+
+int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                              const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                              int heads, int q_block, int kv_block, int causal, float* out, void* stream);
+
 /* ------------------------------------------------------------------------
  * Single steps of Algorithm 1, for checking intermediate results.
  * ------------------------------------------------------------------------ */

@@ -1,47 +1,58 @@
-// Fused blockwise attention for one query tile (128 rows of one head of one
-// sequence) over all of its key/value tiles, with online-softmax rescaling.
+// Fused blockwise attention: one CTA computes two query tiles (2 x 128 rows of
+// one head of one sequence) over all of their key/value tiles, with
+// online-softmax rescaling.
 //
-// Follows Eq. 3 and Algorithm 1 (steps 4-10) of the BPT paper review: scores of
-// the query block against each key/value block, normalisation statistics kept
-// per row (running max m and running sum l in fp32 registers), the block's
+// Follows Eq. 3 and Algorithm 1 (steps 4-10) of the BPT paper review: scores
+// of a query block against each key/value block, normalisation statistics per
+// row (running max m and running sum l, fp32 registers), the block's
 // exp-weights applied to V, and a final rescale by 1/l. The s x s score matrix
-// never leaves the SM: S lives in tensor memory, P in shared memory.
+// never leaves the SM: S and P live in tensor memory.
 //
-// Roles (192 threads): warp 0 loads Q once and K/V tiles into a two-stage
-// ring with TMA; one thread of warp 1 issues S = Q K^T into one of two TMEM
-// score buffers and O += P V into the TMEM output accumulator; warps 2-5 own
-// one query row each (TMEM lane), run the softmax, write P (bf16) to shared
-// memory in the operand layout of the next MMA, rescale O when the running
-// max grows, and write the normalised output row.
+// Roles (320 threads): warp 0 loads Q (both tiles, once) and the K/V tiles
+// into two-stage rings with TMA; one thread of warp 1 issues the MMAs; warps
+// 2-5 run the softmax of query tile 0 and warps 6-9 that of tile 1 (one row
+// per thread = one TMEM lane; warp w reaches lanes 32*(w%4) .. +31, so each
+// group of four consecutive warps covers all 128 lanes). While one warpgroup computes exponentials the
+// tensor core works on the other tile, in the order
+//     PV0(j), S0(j+1), PV1(j), S1(j+1), PV0(j+1), ...
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+dh),
+// O1 [384, 384+dh). The softmax writes P (bf16 pairs) over the first 64
+// columns of its S; the P V product reads it from there (A operand in TMEM),
+// and the next S MMA of that tile, issued after it, overwrites it (MMAs of one
+// thread execute in issue order).
 #pragma once
 
 #include "ptx.cuh"
 
 namespace bpt {
 
-constexpr int ATT_BM = 128;  // query rows per CTA
+constexpr int ATT_BM = 128;  // query rows per tile; two tiles per CTA
 constexpr int ATT_BN = 128;  // keys per key/value tile
-constexpr int ATT_THREADS = 192;
-constexpr int ATT_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+dh)
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_TMEM_COLS = 512;
 // Skip rescaling O until the running max has grown by more than this (log2
-// units); P then holds values up to 2^8, which bf16 and fp32 carry exactly in
-// range. The final division by l uses the same stale max, so the result is exact.
+// units); P then holds values up to 2^8, well inside bf16 and fp32 range. The
+// final division by l uses the same stale max, so the result is exact.
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;
+// Of each group of four element pairs of an interior (unmasked) tile, this
+// many take their 2^x from exp2_poly_x2 on the FMA pipe, the rest from the
+// MUFU unit, so that neither unit alone limits the softmax.
+#ifndef ATT_POLY_PAIRS_OF_4
+#define ATT_POLY_PAIRS_OF_4 0
+#endif
 
 template <int DH>
 struct AttnCfg {
-  static constexpr int Q_BYTES = ATT_BM * DH * 2;
-  static constexpr int KV_BYTES = ATT_BN * DH * 2;
-  static constexpr int P_BYTES = ATT_BM * ATT_BN * 2;
-  static constexpr int ATOM_BYTES = 128 * 128;  // [128 rows][64 bf16] swizzle-128B box
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int Q_BYTES = ATT_BM * DH * 2;   // one query tile
+  static constexpr int KV_BYTES = ATT_BN * DH * 2;  // one K or V tile
+  static constexpr int ATOM_BYTES = 128 * 128;      // [128 rows][64 bf16] 128B-swizzled box
+  static constexpr int OFF_Q = 0;                   // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES; // two stages
   static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
   static constexpr int USED = OFF_BAR + 256 + 1024;
-  // at least 116 KB so that one CTA holds an SM (the 512 TMEM columns are
-  // allocated whole)
+  // at least 116 KB so that one CTA holds an SM (all 512 TMEM columns are
+  // allocated)
   static constexpr int SMEM_BYTES = USED > 118784 ? USED : 118784;
 };
 
@@ -50,11 +61,22 @@ struct AttnArgs {
   int beta0;        // first sequence of this launch
   int t_start;      // query positions [t_start, t_start + t_len) of each sequence
   int t_len;
-  int n_qtiles;     // ceil(t_len / 128)
+  int n_pairs;      // ceil(t_len / 256): CTAs per (sequence, head)
   __nv_bfloat16* o; // output rows: (beta - beta0) * t_len + (t - t_start)
   long long ldo;
   float scale_log2; // log2(e) / sqrt(dh)
 };
+
+// D[tmem] (+)= A[tmem] * B[smem]: bf16 A read from tensor memory (K-major).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 template <int DH>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
@@ -69,10 +91,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const uint32_t k_empty0 = smem_addr(bars + 3);  // [2]
   const uint32_t v_full0 = smem_addr(bars + 5);   // [2]
   const uint32_t v_empty0 = smem_addr(bars + 7);  // [2]
-  const uint32_t s_full0 = smem_addr(bars + 9);   // [2]
-  const uint32_t s_free0 = smem_addr(bars + 11);  // [2]
-  const uint32_t p_full = smem_addr(bars + 13);
-  const uint32_t pv_done = smem_addr(bars + 14);
+  const uint32_t s_full0 = smem_addr(bars + 9);   // [2] per query tile
+  const uint32_t p_full0 = smem_addr(bars + 11);  // [2] per query tile
+  const uint32_t o_done0 = smem_addr(bars + 13);  // [2] per query tile
   const uint32_t mma_done = smem_addr(bars + 15);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
@@ -81,14 +102,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int lane = lane_id();
   const uint32_t sbase = smem_addr(smem);
 
-  // ------------------------------------------------------------ tile geometry
+  // ------------------------------------------------------------ geometry
   const int head = blockIdx.x;
-  const int qt = args.causal ? (args.n_qtiles - 1 - (int)blockIdx.y) : (int)blockIdx.y;  // heavy tiles first
+  const int pair = args.causal ? (args.n_pairs - 1 - (int)blockIdx.y) : (int)blockIdx.y;  // heavy pairs first
   const int beta = args.beta0 + blockIdx.z;
-  const int t0 = args.t_start + qt * ATT_BM;
-  const int rows_valid = min(ATT_BM, args.t_start + args.t_len - t0);
-  const int kv_end = args.causal ? min(args.s, t0 + rows_valid) : args.s;  // keys [0, kv_end)
-  const int n_kv = (kv_end + ATT_BN - 1) / ATT_BN;
+  const int t0 = args.t_start + pair * 2 * ATT_BM;  // first row of query tile 0
+  const int t_end = args.t_start + args.t_len;
+  int rows_valid[2], n_kv[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    rows_valid[q] = max(0, min(ATT_BM, t_end - (t0 + q * ATT_BM)));
+    const int kv_end = args.causal ? min(args.s, t0 + q * ATT_BM + rows_valid[q]) : args.s;
+    n_kv[q] = rows_valid[q] > 0 ? (kv_end + ATT_BN - 1) / ATT_BN : 0;
+  }
+  const int n_tiles = max(n_kv[0], n_kv[1]);
+  const bool has1 = rows_valid[1] > 0;
 
   if (warp == 0 && lane == 0) {
     mbar_init(q_full, 1);
@@ -98,10 +126,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(v_full0 + 8 * i, 1);
       mbar_init(v_empty0 + 8 * i, 1);
       mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_free0 + 8 * i, 4);
+      mbar_init(p_full0 + 8 * i, 4);
+      mbar_init(o_done0 + 8 * i, 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -117,17 +144,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tS0 = tmem_base, tO = tmem_base + 256;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
       uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      const int nq = has1 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
+      for (int q = 0; q < nq; ++q)
 #pragma unroll
-      for (int a = 0; a < DH / 64; ++a)
-        tma_load_3d(sbase + C::OFF_Q + a * C::ATOM_BYTES, &tmQ, q_full, head * DH + a * 64, t0, beta);
-      for (int j = 0; j < n_kv; ++j) {
+        for (int a = 0; a < DH / 64; ++a)
+          tma_load_3d(sbase + C::OFF_Q + q * C::Q_BYTES + a * C::ATOM_BYTES, &tmQ, q_full, head * DH + a * 64,
+                      t0 + q * ATT_BM, beta);
+      for (int j = 0; j < n_tiles; ++j) {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         if (!mbar_wait(k_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
@@ -159,151 +188,165 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_s = idesc_bf16_f32(ATT_BM, ATT_BN, 0, 0);  // Q K-major, K tile K-major
-      const uint32_t idesc_o = idesc_bf16_f32(ATT_BM, DH, 0, 1);      // P K-major, V tile MN-major
-      const uint32_t q_s = sbase + C::OFF_Q;
-      const uint32_t p_s = sbase + C::OFF_P;
+      const uint32_t idesc_o = idesc_bf16_f32(ATT_BM, DH, 0, 1);      // P K-major (TMEM), V MN-major
+      int k_waited = -1, v_waited = -1;
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      // S(n) = Q K_n^T into score buffer n % 2
-      auto issue_s = [&](int n) -> bool {
-        const int sb = n & 1;
-        if (n >= 2 && !mbar_wait(s_free0 + 8 * sb, ((n >> 1) - 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(k_full0 + 8 * sb, (n >> 1) & 1, abort_flag)) return false;
+      // the last query tile that uses key/value tile j releases its stage
+      auto last_user = [&](int j) { return (has1 && j < n_kv[1]) ? 1 : 0; };
+      auto issue_s = [&](int q, int j) -> bool {
+        const int st = j & 1;
+        if (k_waited < j) {
+          if (!mbar_wait(k_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+          k_waited = j;
+        }
         tc_fence_after();
-        const uint32_t k_s = sbase + C::OFF_K + sb * C::KV_BYTES;
+        const uint32_t q_s = sbase + C::OFF_Q + q * C::Q_BYTES;
+        const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tS0 + sb * ATT_BN, smem_desc_sw128(q_s + off, 16, 1024), smem_desc_sw128(k_s + off, 16, 1024),
-                      idesc_s, kk > 0);
+          mma_bf16_ss(tmem_base + q * 128, smem_desc_sw128(q_s + off, 16, 1024),
+                      smem_desc_sw128(k_s + off, 16, 1024), idesc_s, kk > 0);
         }
-        mma_commit(s_full0 + 8 * sb);
-        mma_commit(k_empty0 + 8 * sb);
+        mma_commit(s_full0 + 8 * q);
+        if (last_user(j) == q) mma_commit(k_empty0 + 8 * st);
         return true;
       };
-      if (ok && n_kv > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv && !issue_s(j + 1)) break;
+      auto issue_pv = [&](int q, int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(p_full, j & 1, abort_flag)) break;
-        if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(p_full0 + 8 * q, j & 1, abort_flag)) return false;
+        if (v_waited < j) {
+          if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+          v_waited = j;
+        }
         tc_fence_after();
         const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
+        const uint32_t p_t = tmem_base + q * 128;
+        const uint32_t o_t = tmem_base + 256 + q * 128;
 #pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; ++kk) {
-          const uint64_t pdesc = smem_desc_sw128(p_s + (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32, 16, 1024);
-          const uint64_t vdesc = smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024);
-          mma_bf16_ss(tO, pdesc, vdesc, idesc_o, (j | kk) != 0);
+        for (int kk = 0; kk < ATT_BN / 16; ++kk)
+          mma_bf16_ts(o_t, p_t + kk * 8, smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024), idesc_o,
+                      (j | kk) != 0);
+        if (last_user(j) == q) mma_commit(v_empty0 + 8 * st);
+        if (j == n_kv[q] - 1) mma_commit(o_done0 + 8 * q);
+        return true;
+      };
+      for (int q = 0; ok && q < 2; ++q)
+        if (n_kv[q] > 0) ok = issue_s(q, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        for (int q = 0; ok && q < 2; ++q) {
+          if (j < n_kv[q]) ok = issue_pv(q, j);
+          if (ok && j + 1 < n_kv[q]) ok = issue_s(q, j + 1);
         }
-        mma_commit(pv_done);
-        mma_commit(v_empty0 + 8 * st);
       }
       mma_commit(mma_done);
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int q = (warp - 2) >> 2;  // query tile of this group of four warps
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
-    const int t = t0 + r;
+    const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
+    const int tq0 = t0 + q * ATT_BM;    // first row of the tile
+    const int t = tq0 + r;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem_base + q * 128 + lane_base;
+    const uint32_t tO = tmem_base + 256 + q * 128 + lane_base;
     const float sl2 = args.scale_log2;
+    const int nk = n_kv[q];
+    const int lim = args.causal ? min(args.s - 1, t) : args.s - 1;  // last visible key of this row
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
-    const uint32_t p_row = sbase + C::OFF_P + r * 128;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!warp_wait(s_full0 + 8 * sb, (j >> 1) & 1, abort_flag)) { ok = false; break; }
+    for (int j = 0; j < nk; ++j) {
+      if (!warp_wait(s_full0 + 8 * q, j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float sv[ATT_BN];
-      {
-        uint32_t a[32], b[32];
-        tmem_load32x2(tS0 + sb * ATT_BN + lane_base, tS0 + sb * ATT_BN + 32 + lane_base, a, b);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(a[i]); sv[32 + i] = __uint_as_float(b[i]); }
-        tmem_load32x2(tS0 + sb * ATT_BN + 64 + lane_base, tS0 + sb * ATT_BN + 96 + lane_base, a, b);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sv[64 + i] = __uint_as_float(a[i]); sv[96 + i] = __uint_as_float(b[i]); }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free0 + 8 * sb);
-
-      // scale into log2 units, mask, row max
+      tmem_load64f<0>(tS, sv);
+      tmem_load64f<64>(tS + 64, sv);
+      // mask and row max of the raw scores (the scale is positive)
       const int key0 = j * ATT_BN;
-      const bool need_mask = (key0 + ATT_BN > args.s) || (args.causal && key0 + ATT_BN - 1 > t0);
-      float mx = -INFINITY;
+      const bool need_mask = (key0 + ATT_BN > args.s) || (args.causal && key0 + ATT_BN - 1 > tq0);
+      // eight independent running maxima: a single chain of 128 dependent
+      // max operations would serialise on their latency
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       if (need_mask) {
-        const int lim = args.causal ? min(args.s - 1, t) : args.s - 1;  // last visible key
 #pragma unroll
         for (int i = 0; i < ATT_BN; ++i) {
-          const float v = (key0 + i <= lim) ? sv[i] * sl2 : -INFINITY;
-          sv[i] = v;
-          mx = fmaxf(mx, v);
+          sv[i] = (key0 + i <= lim) ? sv[i] : -INFINITY;
+          mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < ATT_BN; ++i) {
-          sv[i] *= sl2;
-          mx = fmaxf(mx, sv[i]);
-        }
+        for (int i = 0; i < ATT_BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
       }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      mx *= sl2;
       float m_new = m, alpha = 1.0f;
       if (mx > m + ATT_RESCALE_THRESHOLD) {
         m_new = mx;
         alpha = ex2_approx(m - mx);  // 0 on the first tile (m = -inf)
       }
-      uint32_t pk[ATT_BN / 2];
-      float sum = 0.0f;
-#pragma unroll
-      for (int i = 0; i < ATT_BN; i += 2) {
-        const float p0 = ex2_approx(sv[i] - m_new);
-        const float p1 = ex2_approx(sv[i + 1] - m_new);
-        const uint32_t pp = pack_bf16x2(p0, p1);
-        pk[i / 2] = pp;
-        // l sums the bf16 weights the P V product uses, so that O = sum(P V) / l
-        // is an exact weighted mean (V == 1 gives exactly 1)
-        sum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
-      }
-      l = l * alpha + sum;
-      m = m_new;
-
-      // P buffer and O are free once the previous P V product has completed
-      if (j > 0) {
-        if (!warp_wait(pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+      // O may be rescaled now: the MMA that produced this S was committed after
+      // every earlier P V product of this tile, so those have completed
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t o[32];
-            tmem_load32(tO + c * 32 + lane_base, o);
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t o[32];
+          tmem_load32(tO + c * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_store32(tO + c * 32 + lane_base, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_store32(tO + c * 32, o);
         }
       }
-      // P row -> shared memory, K-major 128B-swizzled: two [128][64] atoms
+      // P = 2^(S*scale - m) in bf16, written over the first 64 columns of S.
+      // l sums the bf16 weights that the P V product uses, so that
+      // O = sum(P V) / l is an exact weighted mean (V == 1 gives exactly 1).
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_new, -m_new);
+      float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        const uint32_t addr = p_row + (c16 >> 3) * C::ATOM_BYTES + (((c16 & 7) ^ (r & 7)) << 4);
-        st_shared_v4(addr, pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+          const int i = 32 * half + i2;
+          const uint64_t x2 = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), sl2x2, negm2);
+          float p0, p1;
+          if (!need_mask && (i & 3) < ATT_POLY_PAIRS_OF_4) {
+            f2_unpack(exp2_poly_x2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          const uint32_t pp = pack_bf16x2(p0, p1);
+          pk[i2] = pp;
+          sum4[i & 3] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+        }
+        tmem_store32(tS + 32 * half, pk);
       }
-      fence_async_smem();
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      l = l * alpha + sum;
+      m = m_new;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full0 + 8 * q);
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok && n_kv > 0 && warp_wait(pv_done, (n_kv - 1) & 1, abort_flag)) {
+    if (ok && nk > 0 && warp_wait(o_done0 + 8 * q, 0, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      const bool row_ok = r < rows_valid;
+      const bool row_ok = r < rows_valid[q];
       __nv_bfloat16* orow =
           args.o + ((long long)(beta - args.beta0) * args.t_len + (t - args.t_start)) * args.ldo + head * DH;
 #pragma unroll 1
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t o[32];
-        tmem_load32(tO + c * 32 + lane_base, o);
+        tmem_load32(tO + c * 32, o);
         if (row_ok) {
           float v[32];
 #pragma unroll

@@ -5,12 +5,15 @@
 //   1. QKV projection over the whole sequence (step 1): K and V go to the
 //      workspace, Q is parked inside `out` (a bf16 Q row fits in the first half
 //      of its fp32 output row and is consumed before that row is written).
-//   2. For each wave of query blocks (a whole number of q_block rows, about
-//      4096 by default): blockwise attention of the wave's query tiles over all
-//      key/value tiles (steps 4-10), then Wo + bo + x (first residual, fp32 into
-//      `out`), W1 + b1 + ReLU (bf16 U) and W2 + b2 + hid (second residual) on
-//      the wave's rows (step 11). Scratch is bounded by the wave, not by s: the
-//      full-sequence 4h FFN intermediate and the s x s scores never exist.
+//   2. Blockwise attention of every query tile over all of its key/value tiles
+//      (steps 4-10) in one launch; each CTA writes its output O over the Q of
+//      its own rows and head inside `out`.
+//   3. For each wave of query blocks (a whole number of q_block rows, about
+//      4096 by default): Wo + bo + x (first residual, fp32 hid in the wave
+//      scratch), W1 + b1 + ReLU (bf16 U) and W2 + b2 + hid (second residual,
+//      into `out`) on the wave's rows (step 11). Scratch is bounded by the
+//      wave, not by s: the full-sequence 4h FFN intermediate and the s x s
+//      scores never exist.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -163,6 +166,37 @@ int check_device(int* sms) {
   return BPT_OK;
 }
 
+// ------------------------------------------------------------- workspace pool
+// The allocating entry points take their workspace from a library-owned,
+// stream-ordered memory pool per device that keeps freed memory for the next
+// call (release threshold: never), so a call does not map and unmap hundreds
+// of MB each time. The pool holds at most the largest workspace requested by
+// concurrent calls.
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[64] = {};
+
+int workspace_pool(cudaMemPool_t* pool) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return BPT_ERR_CUDA;
+    }
+    uint64_t keep = UINT64_MAX;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = p;
+  }
+  *pool = g_pool[dev];
+  return BPT_OK;
+}
+
 // ------------------------------------------------------------- argument checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -228,7 +262,7 @@ std::vector<Wave> plan_waves(int b, int s, int q_block, int wave_rows) {
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-  size_t k, v, hb, ou, xb, wqkv, wo, w1, w2, total;
+  size_t k, v, hid, hb, u, xb, wqkv, wo, w1, w2, total;
   int wave_rows;
 };
 
@@ -245,8 +279,9 @@ Layout layout_for(int dtype, int b, int s, int h, int q_block, int wave_rows) {
   };
   L.k = take(tok * h * 2);
   L.v = take(tok * h * 2);
+  L.hid = take((size_t)wr * h * 4);
   L.hb = take((size_t)wr * h * 2);
-  L.ou = take((size_t)wr * 4 * h * 2);
+  L.u = take((size_t)wr * 4 * h * 2);
   if (dtype == BPT_DTYPE_F32) {
     L.xb = take(tok * h * 2);
     L.wqkv = take((size_t)h * 3 * h * 2);
@@ -295,14 +330,14 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
   a.causal = causal ? 1 : 0;
   a.t_start = t_start;
   a.t_len = t_len;
-  a.n_qtiles = (t_len + ATT_BM - 1) / ATT_BM;
+  a.n_pairs = (t_len + 2 * ATT_BM - 1) / (2 * ATT_BM);
   a.ldo = ldo;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
   for (int z0 = 0; z0 < n_seq; z0 += 65535) {
     const int nz = std::min(65535, n_seq - z0);
     a.beta0 = beta0 + z0;
     a.o = o + (long long)z0 * t_len * ldo;
-    dim3 grid(heads, a.n_qtiles, nz);
+    dim3 grid(heads, a.n_pairs, nz);
     LaunchScope ls("attention", st);
     if (dh == 64)
       attention_fwd_tcgen05<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);
@@ -372,9 +407,12 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   const long long tok = (long long)b * s;
   __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(ws + L.k);
   __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(ws + L.v);
+  float* HID = reinterpret_cast<float*>(ws + L.hid);
   __nv_bfloat16* HB = reinterpret_cast<__nv_bfloat16*>(ws + L.hb);
-  __nv_bfloat16* OU = reinterpret_cast<__nv_bfloat16*>(ws + L.ou);
-  __nv_bfloat16* Q = reinterpret_cast<__nv_bfloat16*>(out);  // bf16 row r at out row r
+  __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + L.u);
+  // Q, then the attention output O, live in out: bf16 row r in the first half
+  // of out's fp32 row r
+  __nv_bfloat16* QO = reinterpret_cast<__nv_bfloat16*>(out);
   const long long ldq = 2LL * h;
 
   const void *xa = p.x, *wqkv = p.Wqkv, *wo = p.Wo, *w1 = p.W1, *w2 = p.W2;
@@ -397,7 +435,7 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     GemmArgs a{};
     a.bias = p.bqkv;
     a.bias_f32 = f32;
-    a.q = Q;
+    a.q = QO;
     a.ldq = ldq;
     a.k = K;
     a.v = V;
@@ -406,14 +444,19 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, "gemm_qkv"));
   }
 
-  // steps 4-11 per wave of query blocks
+  // steps 4-10 for every query block at once: each CTA overwrites the Q of its
+  // own rows and head with their attention output
+  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st));
+
+  // step 11 per wave of query blocks: out-projection, residuals and FFN
   for (const Wave& w : plan_waves(b, s, q_block, wave_rows)) {
     const long long rows = w.rows();
-    BPT_TRY(launch_attention(Q, ldq, K, V, b, s, h, heads, causal, w.beta0, w.n_seq, w.t_start, w.t_len, OU, h, st));
     GemmArgs a{};
     a.resid = p.x;
     a.resid_f32 = f32;
     a.ld_resid = h;
+    a.hid = HID;
+    a.ld_hid = h;
     a.out = out;
     a.ld_out = h;
     a.row0 = w.row0;
@@ -421,13 +464,13 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.bias = p.bo;
     a.dst = HB;
     a.ld_dst = h;
-    BPT_TRY(launch_gemm<EPI_OUTPROJ>(OU, rows, h, h, wo, h, a, sms, st, "gemm_outproj"));
+    BPT_TRY(launch_gemm<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, h, a, sms, st, "gemm_outproj"));
     a.bias = p.b1;
-    a.dst = OU;
+    a.dst = U;
     a.ld_dst = 4LL * h;
     BPT_TRY(launch_gemm<EPI_FFN_UP>(HB, rows, h, h, w1, 4LL * h, a, sms, st, "gemm_ffn_up"));
     a.bias = p.b2;
-    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(OU, rows, 4LL * h, 4LL * h, w2, h, a, sms, st, "gemm_ffn_down"));
+    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(U, rows, 4LL * h, 4LL * h, w2, h, a, sms, st, "gemm_ffn_down"));
   }
   return BPT_OK;
 }
@@ -456,8 +499,10 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   if (!caller_ws) {
+    cudaMemPool_t pool = nullptr;
+    BPT_TRY(workspace_pool(&pool));
     void* m = nullptr;
-    if (cudaMallocAsync(&m, L.total, st) != cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&m, L.total, pool, st) != cudaSuccess) {
       cudaGetLastError();
       return BPT_ERR_NOMEM;
     }

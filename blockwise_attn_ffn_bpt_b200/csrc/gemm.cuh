@@ -29,9 +29,9 @@ constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + 256;
 
 enum EpiMode {
   EPI_QKV = 0,       // + bqkv -> bf16 Q | K | V
-  EPI_OUTPROJ = 1,   // + bo + x (first residual) -> fp32 hid into out, bf16 copy for the FFN
+  EPI_OUTPROJ = 1,   // + bo + x (first residual) -> fp32 hid and its bf16 copy (wave scratch)
   EPI_FFN_UP = 2,    // + b1, ReLU -> bf16 U
-  EPI_FFN_DOWN = 3,  // + b2 + hid (second residual, read from out) -> fp32 out
+  EPI_FFN_DOWN = 3,  // + b2 + hid (second residual) -> fp32 out
 };
 
 struct GemmArgs {
@@ -50,7 +50,10 @@ struct GemmArgs {
   const void* resid;
   int resid_f32;
   long long ld_resid;
-  // fp32 out (OUTPROJ writes hid, FFN_DOWN reads hid and writes the result)
+  // fp32 hid of the wave's rows (OUTPROJ writes it, FFN_DOWN reads it)
+  float* hid;
+  long long ld_hid;
+  // fp32 layer output (FFN_DOWN)
   float* out;
   long long ld_out;
   long long row0;    // flat row of local row 0 (for x and out)
@@ -121,7 +124,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int co
     load32(a.resid, a.resid_f32, grow * a.ld_resid + col, x);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += bias[i] + x[i];
-    store32_f32(a.out + grow * a.ld_out + col, v);
+    store32_f32(a.hid + (long long)row * a.ld_hid + col, v);
     store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
   } else if constexpr (MODE == EPI_FFN_UP) {
 #pragma unroll
@@ -129,11 +132,10 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int co
     store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
   } else {
     float hid[32];
-    const long long grow = a.row0 + row;
-    float* o = a.out + grow * a.ld_out + col;
-    load32(o, 1, 0, hid);
+    load32(a.hid + (long long)row * a.ld_hid + col, 1, 0, hid);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += bias[i] + hid[i];
+    float* o = a.out + (a.row0 + row) * a.ld_out + col;
     store32_f32(o, v);
   }
 }

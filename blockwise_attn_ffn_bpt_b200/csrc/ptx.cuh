@@ -202,6 +202,59 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
+// 64 consecutive fp32 columns ([col, col + 64)) of this thread's lane into
+// v[0..63], with the completion wait in the same asm statement.
+#define BPT_F32x32(v, o)                                                                                          \
+  "=f"(v[o + 0]), "=f"(v[o + 1]), "=f"(v[o + 2]), "=f"(v[o + 3]), "=f"(v[o + 4]), "=f"(v[o + 5]), "=f"(v[o + 6]), \
+      "=f"(v[o + 7]), "=f"(v[o + 8]), "=f"(v[o + 9]), "=f"(v[o + 10]), "=f"(v[o + 11]), "=f"(v[o + 12]),          \
+      "=f"(v[o + 13]), "=f"(v[o + 14]), "=f"(v[o + 15]), "=f"(v[o + 16]), "=f"(v[o + 17]), "=f"(v[o + 18]),       \
+      "=f"(v[o + 19]), "=f"(v[o + 20]), "=f"(v[o + 21]), "=f"(v[o + 22]), "=f"(v[o + 23]), "=f"(v[o + 24]),       \
+      "=f"(v[o + 25]), "=f"(v[o + 26]), "=f"(v[o + 27]), "=f"(v[o + 28]), "=f"(v[o + 29]), "=f"(v[o + 30]),       \
+      "=f"(v[o + 31])
+
+template <int O>
+__device__ __forceinline__ void tmem_load64f(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : BPT_F32x32(v, O), BPT_F32x32(v, O + 32)
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+}
+
+// Store 64 columns of this thread's lane (two 32-column stores, one wait).
+__device__ __forceinline__ void tmem_store64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, "
+      "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%1], "
+      "{%34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, "
+      "%50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(taddr + 32), BPT_IN32(r), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]),
+      "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]),
+      "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]),
+      "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+
+// Store 16 columns of this thread's lane and wait until the store completed.
+__device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm100 format): start address, leading and
 // stride byte offsets (all >> 4), version 1, 128-byte swizzle.
@@ -230,6 +283,52 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---------------------------------------------------------------- packed fp32 pairs
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU unit.
+// Method: clamp x to >= -125, split x = n + f with n = round-to-nearest(x)
+// obtained by adding and subtracting 1.5 * 2^23 (so f is in [-1/2, 1/2]),
+// evaluate a degree-3 polynomial for 2^f whose coefficients were fitted for
+// this library by Lawson's iteratively reweighted least squares (minimax
+// relative error 8.3e-5 on [-1/2, 1/2]), then add n to the exponent field.
+// Inputs must be finite and <= 127; results below 2^-125 come out as ~2^-125.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t shift = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x2, shift);                              // n in the low mantissa bits
+  const uint64_t nf = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));  // n as a float
+  const uint64_t f = f2_fma(nf, f2_pack(-1.0f, -1.0f), x2);          // x - n
+  uint64_t q = f2_fma(f2_pack(0.055212993174791336f, 0.055212993174791336f), f,
+                      f2_pack(0.24271413683891296f, 0.24271413683891296f));
+  q = f2_fma(q, f, f2_pack(0.6932621598243713f, 0.6932621598243713f));
+  q = f2_fma(q, f, f2_pack(0.999919593334198f, 0.999919593334198f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -89,9 +89,11 @@ const char* bpt_status_string(int status);
  * The layer forward (Algorithm 1 of the BPT paper review, section 3).
  * ------------------------------------------------------------------------ */
 
-/* bf16 inputs. Allocates its workspace stream-ordered (cudaMallocAsync on
- * `stream`) and frees it stream-ordered after the last kernel; returns
- * BPT_ERR_NOMEM if that allocation fails. */
+/* bf16 inputs. Allocates its workspace stream-ordered on `stream` from a
+ * library-owned memory pool of the current device and frees it stream-ordered
+ * after the last kernel; the pool keeps freed memory for later calls (so
+ * repeated calls do not map device memory again). Returns BPT_ERR_NOMEM if the
+ * allocation fails. */
 int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
                       const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                       int heads, int q_block, int kv_block, int causal, float* out, void* stream);
@@ -133,7 +135,7 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
  * - Size limit: returns BPT_ERR_NOMEM, with nothing launched, when the
  *   workspace the layer needs (bpt_layer_workspace_bytes(BPT_DTYPE_BF16, b, s,
  *   h, heads, q_block, kv_block, 0)) exceeds BPT_STATIC_WORKSPACE_BYTES; for
- *   example b=2, s=2048, h=1024 needs 56 MiB and fits, s=8192, h=2048 does not.
+ *   example b=1, s=2048, h=1024 needs 36 MiB and fits, s=8192, h=2048 does not.
  * - The first call on each device looks up that device's address of the array
  *   (one cudaGetSymbolAddress, with that device current). Make that first call
  *   before any stream capture on the device.

@@ -106,21 +106,23 @@ def test_ws_entry_checks_dtype_and_workspace():
 
 
 def test_workspace_bytes_follow_the_layout():
-    # bf16: K and V for the whole sequence, plus per-wave bf16 hid copy and the
-    # O / U scratch (wave rows x 5h bf16), each region rounded up to 1 KiB
+    # bf16: K and V for the whole sequence, plus per wave the fp32 hid, its bf16
+    # copy and the bf16 FFN intermediate U (wave rows x 4h), each region rounded
+    # up to 1 KiB
     def up(v):
         return (v + 1023) // 1024 * 1024
+
+    def expect(b, s, h, wr):
+        return up(b * s * h * 2) * 2 + up(wr * h * 4) + up(wr * h * 2) + up(wr * 4 * h * 2)
+
     b, s, h = 1, 32768, 4096
     ws = bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048)
-    wr = 4096
-    assert ws == up(b * s * h * 2) * 2 + up(wr * h * 2) + up(wr * 4 * h * 2)
+    assert ws == expect(b, s, h, 4096)
     # element ratio against 2bsh stays within 1.5
     assert ws / 2 / (2 * b * s * h) <= 1.5
     # wave rows are whole query blocks; a whole-sequence wave covers whole sequences
-    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == \
-        up(2 * 2048 * 1024 * 2) * 2 + up(4096 * 1024 * 2) + up(4096 * 4096 * 2)
-    assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == \
-        up(16384 * 2048 * 2) * 2 + up(2048 * 2048 * 2) + up(2048 * 4 * 2048 * 2)
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == expect(2, 2048, 1024, 4096)
+    assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == expect(1, 16384, 2048, 2048)
     # fp32 inputs add bf16 copies of x and the weights
     f = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
     g = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)

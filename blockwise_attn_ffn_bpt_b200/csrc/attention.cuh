@@ -8,11 +8,15 @@
 // exp-weights applied to V, and a final rescale by 1/l. The s x s score matrix
 // never leaves the SM: S and P live in tensor memory.
 //
-// Roles (320 threads): warp 0 loads Q (both tiles, once) and the K/V tiles
-// into two-stage rings with TMA; one thread of warp 1 issues the MMAs; warps
-// 2-5 run the softmax of query tile 0 and warps 6-9 that of tile 1 (one row
-// per thread = one TMEM lane; warp w reaches lanes 32*(w%4) .. +31, so each
-// group of four consecutive warps covers all 128 lanes). While one warpgroup computes exponentials the
+// Roles (384 threads = three warpgroups): warp 0 loads Q (both tiles, once)
+// and the K/V tiles into two-stage rings with TMA; one thread of warp 1 issues
+// the MMAs; warps 2-3 idle; warpgroup 1 (warps 4-7) runs the softmax of query
+// tile 0 and warpgroup 2 (warps 8-11) that of tile 1, one row per thread =
+// one TMEM lane (warp w reaches lanes 32*(w%4) .. +31). Registers are split
+// per warpgroup: the kernel is built for 168 per thread (384 x 168 = 64512),
+// warpgroup 0 gives back down to ATT_REGS_CONTROL and the softmax warpgroups
+// grow to ATT_REGS_SOFTMAX (128 x 56 + 256 x 216 = 62464 <= 64512). The host
+// launches the kernel only if it was built with exactly ATT_REGS_LAUNCH. While one warpgroup computes exponentials the
 // tensor core works on the other tile, in the order
 //     PV0(j), S0(j+1), PV1(j), S1(j+1), PV0(j+1), ...
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+dh),
@@ -28,7 +32,12 @@ namespace bpt {
 
 constexpr int ATT_BM = 128;  // query rows per tile; two tiles per CTA
 constexpr int ATT_BN = 128;  // keys per key/value tile
-constexpr int ATT_THREADS = 320;
+constexpr int ATT_THREADS = 384;
+constexpr int ATT_REGS_LAUNCH = 168;   // registers per thread the kernel is built with
+constexpr int ATT_REGS_CONTROL = 56;   // warpgroup 0: TMA producer and MMA issuer
+constexpr int ATT_REGS_SOFTMAX = 216;  // warpgroups 1 and 2
+static_assert(ATT_THREADS * ATT_REGS_LAUNCH >= 128 * ATT_REGS_CONTROL + 256 * ATT_REGS_SOFTMAX,
+              "register split exceeds the block's launch allocation");
 constexpr int ATT_TMEM_COLS = 512;
 // Skip rescaling O until the running max has grown by more than this (log2
 // units); P then holds values up to 2^8, well inside bf16 and fp32 range. The
@@ -145,105 +154,110 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
-      uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
-      const int nq = has1 ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
-      for (int q = 0; q < nq; ++q)
+  if (warp < 4) {
+    // each role stays inside the branch that set its register budget
+    regs_decrease<ATT_REGS_CONTROL>();
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- TMA producer
+        uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
+        const int nq = has1 ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
+        for (int q = 0; q < nq; ++q)
 #pragma unroll
-        for (int a = 0; a < DH / 64; ++a)
-          tma_load_3d(sbase + C::OFF_Q + q * C::Q_BYTES + a * C::ATOM_BYTES, &tmQ, q_full, head * DH + a * 64,
-                      t0 + q * ATT_BM, beta);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(k_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(k_full0 + 8 * st, C::KV_BYTES);
+          for (int a = 0; a < DH / 64; ++a)
+            tma_load_3d(sbase + C::OFF_Q + q * C::Q_BYTES + a * C::ATOM_BYTES, &tmQ, q_full, head * DH + a * 64,
+                        t0 + q * ATT_BM, beta);
+        for (int j = 0; j < n_tiles; ++j) {
+          const int st = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (!mbar_wait(k_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(k_full0 + 8 * st, C::KV_BYTES);
 #pragma unroll
-        for (int a = 0; a < DH / 64; ++a)
-          tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmK, k_full0 + 8 * st,
-                      head * DH + a * 64, j * ATT_BN, beta);
-        k_issued |= 1u << st;
-        k_par = (k_par & ~(1u << st)) | (ph << st);
-        if (!mbar_wait(v_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(v_full0 + 8 * st, C::KV_BYTES);
+          for (int a = 0; a < DH / 64; ++a)
+            tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmK, k_full0 + 8 * st,
+                        head * DH + a * 64, j * ATT_BN, beta);
+          k_issued |= 1u << st;
+          k_par = (k_par & ~(1u << st)) | (ph << st);
+          if (!mbar_wait(v_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(v_full0 + 8 * st, C::KV_BYTES);
 #pragma unroll
-        for (int a = 0; a < DH / 64; ++a)
-          tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmV, v_full0 + 8 * st,
-                      head * DH + a * 64, j * ATT_BN, beta);
-        v_issued |= 1u << st;
-        v_par = (v_par & ~(1u << st)) | (ph << st);
-      }
-      // never leave with copies still landing in shared memory
-      volatile int dummy = 0;
-      mbar_wait(q_full, 0, &dummy);
-      for (int i = 0; i < 2; ++i) {
-        if (k_issued & (1u << i)) mbar_wait(k_full0 + 8 * i, (k_par >> i) & 1u, &dummy);
-        if (v_issued & (1u << i)) mbar_wait(v_full0 + 8 * i, (v_par >> i) & 1u, &dummy);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      const uint32_t idesc_s = idesc_bf16_f32(ATT_BM, ATT_BN, 0, 0);  // Q K-major, K tile K-major
-      const uint32_t idesc_o = idesc_bf16_f32(ATT_BM, DH, 0, 1);      // P K-major (TMEM), V MN-major
-      int k_waited = -1, v_waited = -1;
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      // the last query tile that uses key/value tile j releases its stage
-      auto last_user = [&](int j) { return (has1 && j < n_kv[1]) ? 1 : 0; };
-      auto issue_s = [&](int q, int j) -> bool {
-        const int st = j & 1;
-        if (k_waited < j) {
-          if (!mbar_wait(k_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
-          k_waited = j;
+          for (int a = 0; a < DH / 64; ++a)
+            tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmV, v_full0 + 8 * st,
+                        head * DH + a * 64, j * ATT_BN, beta);
+          v_issued |= 1u << st;
+          v_par = (v_par & ~(1u << st)) | (ph << st);
         }
-        tc_fence_after();
-        const uint32_t q_s = sbase + C::OFF_Q + q * C::Q_BYTES;
-        const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tmem_base + q * 128, smem_desc_sw128(q_s + off, 16, 1024),
-                      smem_desc_sw128(k_s + off, 16, 1024), idesc_s, kk > 0);
-        }
-        mma_commit(s_full0 + 8 * q);
-        if (last_user(j) == q) mma_commit(k_empty0 + 8 * st);
-        return true;
-      };
-      auto issue_pv = [&](int q, int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(p_full0 + 8 * q, j & 1, abort_flag)) return false;
-        if (v_waited < j) {
-          if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
-          v_waited = j;
-        }
-        tc_fence_after();
-        const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
-        const uint32_t p_t = tmem_base + q * 128;
-        const uint32_t o_t = tmem_base + 256 + q * 128;
-#pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; ++kk)
-          mma_bf16_ts(o_t, p_t + kk * 8, smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024), idesc_o,
-                      (j | kk) != 0);
-        if (last_user(j) == q) mma_commit(v_empty0 + 8 * st);
-        if (j == n_kv[q] - 1) mma_commit(o_done0 + 8 * q);
-        return true;
-      };
-      for (int q = 0; ok && q < 2; ++q)
-        if (n_kv[q] > 0) ok = issue_s(q, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        for (int q = 0; ok && q < 2; ++q) {
-          if (j < n_kv[q]) ok = issue_pv(q, j);
-          if (ok && j + 1 < n_kv[q]) ok = issue_s(q, j + 1);
+        // never leave with copies still landing in shared memory
+        volatile int dummy = 0;
+        mbar_wait(q_full, 0, &dummy);
+        for (int i = 0; i < 2; ++i) {
+          if (k_issued & (1u << i)) mbar_wait(k_full0 + 8 * i, (k_par >> i) & 1u, &dummy);
+          if (v_issued & (1u << i)) mbar_wait(v_full0 + 8 * i, (v_par >> i) & 1u, &dummy);
         }
       }
-      mma_commit(mma_done);
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- MMA issuer
+        const uint32_t idesc_s = idesc_bf16_f32(ATT_BM, ATT_BN, 0, 0);  // Q K-major, K tile K-major
+        const uint32_t idesc_o = idesc_bf16_f32(ATT_BM, DH, 0, 1);      // P K-major (TMEM), V MN-major
+        int k_waited = -1, v_waited = -1;
+        bool ok = mbar_wait(q_full, 0, abort_flag);
+        // the last query tile that uses key/value tile j releases its stage
+        auto last_user = [&](int j) { return (has1 && j < n_kv[1]) ? 1 : 0; };
+        auto issue_s = [&](int q, int j) -> bool {
+          const int st = j & 1;
+          if (k_waited < j) {
+            if (!mbar_wait(k_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+            k_waited = j;
+          }
+          tc_fence_after();
+          const uint32_t q_s = sbase + C::OFF_Q + q * C::Q_BYTES;
+          const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+            mma_bf16_ss(tmem_base + q * 128, smem_desc_sw128(q_s + off, 16, 1024),
+                        smem_desc_sw128(k_s + off, 16, 1024), idesc_s, kk > 0);
+          }
+          mma_commit(s_full0 + 8 * q);
+          if (last_user(j) == q) mma_commit(k_empty0 + 8 * st);
+          return true;
+        };
+        auto issue_pv = [&](int q, int j) -> bool {
+          const int st = j & 1;
+          if (!mbar_wait(p_full0 + 8 * q, j & 1, abort_flag)) return false;
+          if (v_waited < j) {
+            if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+            v_waited = j;
+          }
+          tc_fence_after();
+          const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
+          const uint32_t p_t = tmem_base + q * 128;
+          const uint32_t o_t = tmem_base + 256 + q * 128;
+#pragma unroll
+          for (int kk = 0; kk < ATT_BN / 16; ++kk)
+            mma_bf16_ts(o_t, p_t + kk * 8, smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024), idesc_o,
+                        (j | kk) != 0);
+          if (last_user(j) == q) mma_commit(v_empty0 + 8 * st);
+          if (j == n_kv[q] - 1) mma_commit(o_done0 + 8 * q);
+          return true;
+        };
+        for (int q = 0; ok && q < 2; ++q)
+          if (n_kv[q] > 0) ok = issue_s(q, 0);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          for (int q = 0; ok && q < 2; ++q) {
+            if (j < n_kv[q]) ok = issue_pv(q, j);
+            if (ok && j + 1 < n_kv[q]) ok = issue_s(q, j + 1);
+          }
+        }
+        mma_commit(mma_done);
+      }
     }
   } else {
+    regs_increase<ATT_REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax
-    const int q = (warp - 2) >> 2;  // query tile of this group of four warps
+    const int q = (warp - 4) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const int tq0 = t0 + q * ATT_BM;    // first row of the tile

@@ -158,6 +158,14 @@ int check_device(int* sms) {
                    cudaFuncSetAttribute(attention_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         AttnCfg<128>::SMEM_BYTES) == cudaSuccess;
       if (!attrs) return BPT_ERR_CUDA;
+      // the attention kernel splits its registers between warpgroups assuming
+      // it was built with exactly ATT_REGS_LAUNCH per thread; any other build
+      // is never launched (its register requests could not be met)
+      cudaFuncAttributes fa64{}, fa128{};
+      if (cudaFuncGetAttributes(&fa64, attention_fwd_tcgen05<64>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa128, attention_fwd_tcgen05<128>) != cudaSuccess)
+        return BPT_ERR_CUDA;
+      if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH) d.ok = false;
     }
     d.checked = true;
   }

@@ -255,6 +255,17 @@ __device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
+// ---------------------------------------------------------------- register split
+// Per-warpgroup register budgets (all 128 threads of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm100 format): start address, leading and
 // stride byte offsets (all >> 4), version 1, 128-byte swizzle.

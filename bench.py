@@ -106,6 +106,11 @@ def rank_seed(rank: int) -> int:
     return rank
 
 
+def whole_job_throughput(tokens_per_rank: int, steps: int, world: int, ms_max: float) -> float:
+    """Tokens/s of the whole job: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * steps * world / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
@@ -347,7 +352,7 @@ def our_arm(args, shape, name):
     tokens = shape.b * shape.s
     flops = layer_flops(shape)
     total_flops = sum(flops.values())
-    value = tokens * args.steps * world / (ms_max / 1e3)
+    value = whole_job_throughput(tokens, args.steps, world, ms_max)
     tflops = total_flops * args.steps * world / (ms_max / 1e3) / 1e12
     peaks, peak_src = measured_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])

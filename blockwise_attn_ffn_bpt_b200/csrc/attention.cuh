@@ -39,6 +39,7 @@ constexpr int ATT_REGS_SOFTMAX = 216;  // warpgroups 1 and 2
 static_assert(ATT_THREADS * ATT_REGS_LAUNCH >= 128 * ATT_REGS_CONTROL + 256 * ATT_REGS_SOFTMAX,
               "register split exceeds the block's launch allocation");
 constexpr int ATT_TMEM_COLS = 512;
+constexpr int ATT_HEAD_GROUP = 4;  // heads scheduled together (see the grid order below)
 // Skip rescaling O until the running max has grown by more than this (log2
 // units); P then holds values up to 2^8, well inside bf16 and fp32 range. The
 // final division by l uses the same stale max, so the result is exact.
@@ -112,8 +113,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const uint32_t sbase = smem_addr(smem);
 
   // ------------------------------------------------------------ geometry
-  const int head = blockIdx.x;
-  const int pair = args.causal ? (args.n_pairs - 1 - (int)blockIdx.y) : (int)blockIdx.y;  // heavy pairs first
+  // grid: x enumerates (head, query-tile pair) in groups of ATT_HEAD_GROUP
+  // heads; inside a group the pairs go heaviest first (causal), cycling over
+  // the group's heads. CTAs resident together then touch a few heads, whose
+  // K/V stay in L2, and the end of the grid holds the lightest pairs.
+  // z = sequence.
+  const int per_group = ATT_HEAD_GROUP * args.n_pairs;
+  const int group = (int)blockIdx.x / per_group;
+  const int within = (int)blockIdx.x - group * per_group;
+  const int heads_in_group = min(ATT_HEAD_GROUP, args.heads - group * ATT_HEAD_GROUP);
+  const int pair_rank = within / heads_in_group;
+  const int head = group * ATT_HEAD_GROUP + (within - pair_rank * heads_in_group);
+  const int pair = args.causal ? (args.n_pairs - 1 - pair_rank) : pair_rank;
   const int beta = args.beta0 + blockIdx.z;
   const int t0 = args.t_start + pair * 2 * ATT_BM;  // first row of query tile 0
   const int t_end = args.t_start + args.t_len;

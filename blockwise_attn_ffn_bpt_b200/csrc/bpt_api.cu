@@ -345,7 +345,7 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
     const int nz = std::min(65535, n_seq - z0);
     a.beta0 = beta0 + z0;
     a.o = o + (long long)z0 * t_len * ldo;
-    dim3 grid(heads, a.n_pairs, nz);
+    dim3 grid((unsigned)a.n_pairs * (unsigned)heads, 1, nz);
     LaunchScope ls("attention", st);
     if (dh == 64)
       attention_fwd_tcgen05<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);

@@ -19,6 +19,7 @@ import argparse
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import tempfile
@@ -52,6 +53,28 @@ def layer_flops(shape: bi.LayerShape) -> dict:
         "gemm_ffn_up": 2.0 * tok * h * 4 * h,
         "gemm_ffn_down": 2.0 * tok * 4 * h * h,
     }
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when there is none for this workload or the kernel's
+    source changed since the counters were taken."""
+    if kernel != "attention":
+        return None
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attention_s16384_h2048_causal.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(rf"traffic_per_launch_{re.escape(workload)}_bytes: (\d+)", text)
+    m_h = re.search(r"kernel_source_sha256_16: ([0-9a-f]+)", text)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for f in ("attention.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "blockwise_attn_ffn_bpt_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return int(m_t.group(1)) if h.hexdigest()[:16] == m_h.group(1) else None
 
 
 def measured_peaks() -> tuple[dict, str]:
@@ -365,7 +388,8 @@ def our_arm(args, shape, name):
         kflops = flops.get(kname, 0.0) * args.steps
         achieved = kflops / (kms / 1e3) / 1e12 if kms > 0 else 0.0
         roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "launches": nl, "avg_launch_ms": kms / nl,
+                "frac": achieved / peak, "traffic": profiled_traffic(name, kname), "launches": nl,
+                "avg_launch_ms": kms / nl,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"}
     kernel_table = {k: {"launches": n, "ms": t, "share": t / sum(v[1] for v in ktimes.values())}
                     for k, (n, t) in ktimes.items()}

@@ -21,9 +21,10 @@
 //     PV0(j), S0(j+1), PV1(j), S1(j+1), PV0(j+1), ...
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+dh),
 // O1 [384, 384+dh). The softmax writes P (bf16 pairs) over the first 64
-// columns of its S; the P V product reads it from there (A operand in TMEM),
-// and the next S MMA of that tile, issued after it, overwrites it (MMAs of one
-// thread execute in issue order).
+// columns of its S, in two halves of 64 keys; the P V product reads it from
+// there (A operand in TMEM) and starts on the first half while the second is
+// being written; the next S MMA of that tile, issued after it, overwrites it
+// (MMAs of one thread execute in issue order).
 #pragma once
 
 #include "ptx.cuh"
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const uint32_t mma_done = smem_addr(bars + 15);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+  const uint32_t p_half0 = smem_addr(bars + 18);  // [2] per query tile: first 64 keys of P written
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(s_full0 + 8 * i, 1);
       mbar_init(p_full0 + 8 * i, 4);
       mbar_init(o_done0 + 8 * i, 1);
+      mbar_init(p_half0 + 8 * i, 4);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -235,21 +238,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (last_user(j) == q) mma_commit(k_empty0 + 8 * st);
           return true;
         };
+        // P V in two halves of 64 keys: the first starts as soon as the softmax
+        // has written the first half of P
         auto issue_pv = [&](int q, int j) -> bool {
           const int st = j & 1;
-          if (!mbar_wait(p_full0 + 8 * q, j & 1, abort_flag)) return false;
           if (v_waited < j) {
             if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
             v_waited = j;
           }
-          tc_fence_after();
           const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
           const uint32_t p_t = tmem_base + q * 128;
           const uint32_t o_t = tmem_base + 256 + q * 128;
 #pragma unroll
-          for (int kk = 0; kk < ATT_BN / 16; ++kk)
-            mma_bf16_ts(o_t, p_t + kk * 8, smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024), idesc_o,
-                        (j | kk) != 0);
+          for (int half = 0; half < 2; ++half) {
+            if (!mbar_wait((half ? p_full0 : p_half0) + 8 * q, j & 1, abort_flag)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int k4 = 0; k4 < ATT_BN / 32; ++k4) {
+              const int kk = half * (ATT_BN / 32) + k4;
+              mma_bf16_ts(o_t, p_t + kk * 8, smem_desc_sw128(v_s + kk * 16 * 128, C::ATOM_BYTES, 1024), idesc_o,
+                          (j | kk) != 0);
+            }
+          }
           if (last_user(j) == q) mma_commit(v_empty0 + 8 * st);
           if (j == n_kv[q] - 1) mma_commit(o_done0 + 8 * q);
           return true;
@@ -290,23 +300,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // mask and row max of the raw scores (the scale is positive)
       const int key0 = j * ATT_BN;
       const bool need_mask = (key0 + ATT_BN > args.s) || (args.causal && key0 + ATT_BN - 1 > tq0);
-      // eight independent running maxima: a single chain of 128 dependent
-      // max operations would serialise on their latency
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+      // four independent chains of three-input max operations (a single
+      // dependent chain would serialise on latency)
       if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < ATT_BN; ++i) {
-          sv[i] = (key0 + i <= lim) ? sv[i] : -INFINITY;
-          mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < ATT_BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+        for (int i = 0; i < ATT_BN; ++i) sv[i] = (key0 + i <= lim) ? sv[i] : -INFINITY;
       }
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < ATT_BN; i += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx4[k] = max3f(mx4[k], sv[i + 2 * k], sv[i + 2 * k + 1]);
+      }
+      float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
       mx *= sl2;
       float m_new = m, alpha = 1.0f;
       if (mx > m + ATT_RESCALE_THRESHOLD) {
@@ -349,16 +355,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           }
           const uint32_t pp = pack_bf16x2(p0, p1);
           pk[i2] = pp;
-          sum4[i & 3] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+          add_bf16x2_to(pp, sum4[i & 3], sum4[(i + 2) & 3]);
         }
         tmem_store32(tS + 32 * half, pk);
+        // hand this half of P to the MMA issuer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive((half ? p_full0 : p_half0) + 8 * q);
       }
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
       m = m_new;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full0 + 8 * q);
     }
 
     // ------------------------------------------------------------ epilogue

@@ -342,6 +342,21 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
                  __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// acc + (low bf16 of pp) and acc + (high bf16 of pp), each exact conversion
+// followed by one fp32 rounding (mixed-precision add)
+__device__ __forceinline__ void add_bf16x2_to(uint32_t pp, float& acc_lo, float& acc_hi) {
+  unsigned short lo, hi;
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(pp));
+  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc_lo) : "h"(lo));
+  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc_hi) : "h"(hi));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -9,7 +9,7 @@
 // never leaves the SM: S and P live in tensor memory.
 //
 // Roles (384 threads = three warpgroups): warp 0 loads Q (both tiles, once)
-// and the K/V tiles into two-stage rings with TMA; one thread of warp 1 issues
+// and the K/V tiles into a ring of shared-memory slots with TMA; one thread of warp 1 issues
 // the MMAs; warps 2-3 idle; warpgroup 1 (warps 4-7) runs the softmax of query
 // tile 0 and warpgroup 2 (warps 8-11) that of tile 1, one row per thread =
 // one TMEM lane (warp w reaches lanes 32*(w%4) .. +31). Registers are split
@@ -57,14 +57,17 @@ struct AttnCfg {
   static constexpr int Q_BYTES = ATT_BM * DH * 2;   // one query tile
   static constexpr int KV_BYTES = ATT_BN * DH * 2;  // one K or V tile
   static constexpr int ATOM_BYTES = 128 * 128;      // [128 rows][64 bf16] 128B-swizzled box
+  // K and V tiles share one ring of slots (K_j, V_j, K_j+1, ...), as deep as
+  // shared memory allows, so that several tiles are in flight from L2
+  static constexpr int RING = DH == 128 ? 5 : 8;
   static constexpr int OFF_Q = 0;                   // two query tiles
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES; // two stages
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
-  static constexpr int USED = OFF_BAR + 256 + 1024;
+  static constexpr int OFF_RING = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + RING * KV_BYTES;
+  static constexpr int USED = OFF_BAR + 512 + 1024;
   // at least 116 KB so that one CTA holds an SM (all 512 TMEM columns are
   // allocated)
   static constexpr int SMEM_BYTES = USED > 118784 ? USED : 118784;
+  static_assert(USED <= 232448, "shared memory budget");
 };
 
 struct AttnArgs {
@@ -98,17 +101,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   const uint32_t q_full = smem_addr(bars + 0);
-  const uint32_t k_full0 = smem_addr(bars + 1);   // [2]
-  const uint32_t k_empty0 = smem_addr(bars + 3);  // [2]
-  const uint32_t v_full0 = smem_addr(bars + 5);   // [2]
-  const uint32_t v_empty0 = smem_addr(bars + 7);  // [2]
-  const uint32_t s_full0 = smem_addr(bars + 9);   // [2] per query tile
-  const uint32_t p_full0 = smem_addr(bars + 11);  // [2] per query tile
-  const uint32_t o_done0 = smem_addr(bars + 13);  // [2] per query tile
-  const uint32_t mma_done = smem_addr(bars + 15);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
-  const uint32_t p_half0 = smem_addr(bars + 18);  // [2] per query tile: first 64 keys of P written
+  const uint32_t s_full0 = smem_addr(bars + 1);   // [2] per query tile
+  const uint32_t p_full0 = smem_addr(bars + 3);   // [2] per query tile
+  const uint32_t o_done0 = smem_addr(bars + 5);   // [2] per query tile
+  const uint32_t p_half0 = smem_addr(bars + 7);   // [2] per query tile: first 64 keys of P written
+  const uint32_t mma_done = smem_addr(bars + 9);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  const uint32_t ring_full0 = smem_addr(bars + 12);             // [RING]
+  const uint32_t ring_empty0 = smem_addr(bars + 12 + C::RING);  // [RING]
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -143,14 +144,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 0 && lane == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(k_full0 + 8 * i, 1);
-      mbar_init(k_empty0 + 8 * i, 1);
-      mbar_init(v_full0 + 8 * i, 1);
-      mbar_init(v_empty0 + 8 * i, 1);
       mbar_init(s_full0 + 8 * i, 1);
       mbar_init(p_full0 + 8 * i, 4);
       mbar_init(o_done0 + 8 * i, 1);
       mbar_init(p_half0 + 8 * i, 4);
+    }
+    for (int i = 0; i < C::RING; ++i) {
+      mbar_init(ring_full0 + 8 * i, 1);
+      mbar_init(ring_empty0 + 8 * i, 1);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -174,7 +175,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (warp == 0) {
       if (lane == 0) {
         // ---------------------------------------------------------- TMA producer
-        uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
+        // load n of the ring: K_j for n = 2j, V_j for n = 2j + 1
+        uint32_t issued = 0, par = 0;
         const int nq = has1 ? 2 : 1;
         mbar_arrive_expect_tx(q_full, nq * C::Q_BYTES);
         for (int q = 0; q < nq; ++q)
@@ -182,33 +184,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           for (int a = 0; a < DH / 64; ++a)
             tma_load_3d(sbase + C::OFF_Q + q * C::Q_BYTES + a * C::ATOM_BYTES, &tmQ, q_full, head * DH + a * 64,
                         t0 + q * ATT_BM, beta);
-        for (int j = 0; j < n_tiles; ++j) {
-          const int st = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (!mbar_wait(k_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
-          mbar_arrive_expect_tx(k_full0 + 8 * st, C::KV_BYTES);
+        for (int n = 0; n < 2 * n_tiles; ++n) {
+          const int slot = n % C::RING;
+          const uint32_t ph = (uint32_t)(n / C::RING) & 1u;
+          if (!mbar_wait(ring_empty0 + 8 * slot, ph ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(ring_full0 + 8 * slot, C::KV_BYTES);
+          const CUtensorMap* map = (n & 1) ? &tmV : &tmK;
 #pragma unroll
           for (int a = 0; a < DH / 64; ++a)
-            tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmK, k_full0 + 8 * st,
-                        head * DH + a * 64, j * ATT_BN, beta);
-          k_issued |= 1u << st;
-          k_par = (k_par & ~(1u << st)) | (ph << st);
-          if (!mbar_wait(v_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
-          mbar_arrive_expect_tx(v_full0 + 8 * st, C::KV_BYTES);
-#pragma unroll
-          for (int a = 0; a < DH / 64; ++a)
-            tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + a * C::ATOM_BYTES, &tmV, v_full0 + 8 * st,
-                        head * DH + a * 64, j * ATT_BN, beta);
-          v_issued |= 1u << st;
-          v_par = (v_par & ~(1u << st)) | (ph << st);
+            tma_load_3d(sbase + C::OFF_RING + slot * C::KV_BYTES + a * C::ATOM_BYTES, map, ring_full0 + 8 * slot,
+                        head * DH + a * 64, (n >> 1) * ATT_BN, beta);
+          issued |= 1u << slot;
+          par = (par & ~(1u << slot)) | (ph << slot);
         }
         // never leave with copies still landing in shared memory
         volatile int dummy = 0;
         mbar_wait(q_full, 0, &dummy);
-        for (int i = 0; i < 2; ++i) {
-          if (k_issued & (1u << i)) mbar_wait(k_full0 + 8 * i, (k_par >> i) & 1u, &dummy);
-          if (v_issued & (1u << i)) mbar_wait(v_full0 + 8 * i, (v_par >> i) & 1u, &dummy);
-        }
+        for (int i = 0; i < C::RING; ++i)
+          if (issued & (1u << i)) mbar_wait(ring_full0 + 8 * i, (par >> i) & 1u, &dummy);
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -217,17 +210,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t idesc_o = idesc_bf16_f32(ATT_BM, DH, 0, 1);      // P K-major (TMEM), V MN-major
         int k_waited = -1, v_waited = -1;
         bool ok = mbar_wait(q_full, 0, abort_flag);
-        // the last query tile that uses key/value tile j releases its stage
+        // the last query tile that uses key/value tile j releases its slots
         auto last_user = [&](int j) { return (has1 && j < n_kv[1]) ? 1 : 0; };
+        auto slot_of = [&](int n) { return n % C::RING; };
+        auto parity_of = [&](int n) { return (uint32_t)(n / C::RING) & 1u; };
         auto issue_s = [&](int q, int j) -> bool {
-          const int st = j & 1;
+          const int sl = slot_of(2 * j);
           if (k_waited < j) {
-            if (!mbar_wait(k_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+            if (!mbar_wait(ring_full0 + 8 * sl, parity_of(2 * j), abort_flag)) return false;
             k_waited = j;
           }
           tc_fence_after();
           const uint32_t q_s = sbase + C::OFF_Q + q * C::Q_BYTES;
-          const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
+          const uint32_t k_s = sbase + C::OFF_RING + sl * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < DH / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
@@ -235,18 +230,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         smem_desc_sw128(k_s + off, 16, 1024), idesc_s, kk > 0);
           }
           mma_commit(s_full0 + 8 * q);
-          if (last_user(j) == q) mma_commit(k_empty0 + 8 * st);
+          if (last_user(j) == q) mma_commit(ring_empty0 + 8 * sl);
           return true;
         };
         // P V in two halves of 64 keys: the first starts as soon as the softmax
         // has written the first half of P
         auto issue_pv = [&](int q, int j) -> bool {
-          const int st = j & 1;
+          const int sl = slot_of(2 * j + 1);
           if (v_waited < j) {
-            if (!mbar_wait(v_full0 + 8 * st, (j >> 1) & 1, abort_flag)) return false;
+            if (!mbar_wait(ring_full0 + 8 * sl, parity_of(2 * j + 1), abort_flag)) return false;
             v_waited = j;
           }
-          const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
+          const uint32_t v_s = sbase + C::OFF_RING + sl * C::KV_BYTES;
           const uint32_t p_t = tmem_base + q * 128;
           const uint32_t o_t = tmem_base + 256 + q * 128;
 #pragma unroll
@@ -260,7 +255,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                           (j | kk) != 0);
             }
           }
-          if (last_user(j) == q) mma_commit(v_empty0 + 8 * st);
+          if (last_user(j) == q) mma_commit(ring_empty0 + 8 * sl);
           if (j == n_kv[q] - 1) mma_commit(o_done0 + 8 * q);
           return true;
         };
@@ -295,8 +290,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       if (!warp_wait(s_full0 + 8 * q, j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float sv[ATT_BN];
-      tmem_load64f<0>(tS, sv);
-      tmem_load64f<64>(tS + 64, sv);
+      tmem_load128f(tS, sv);
       // mask and row max of the raw scores (the scale is positive)
       const int key0 = j * ATT_BN;
       const bool need_mask = (key0 + ATT_BN > args.s) || (args.causal && key0 + ATT_BN - 1 > tq0);

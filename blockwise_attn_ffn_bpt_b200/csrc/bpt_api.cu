@@ -8,11 +8,12 @@
 //   2. Blockwise attention of every query tile over all of its key/value tiles
 //      (steps 4-10) in one launch; each CTA writes its output O over the Q of
 //      its own rows and head inside `out`.
-//   3. For each wave of query blocks (a whole number of q_block rows, about
-//      4096 by default): Wo + bo + x (first residual, fp32 hid in the wave
-//      scratch), W1 + b1 + ReLU (bf16 U) and W2 + b2 + hid (second residual,
-//      into `out`) on the wave's rows (step 11). Scratch is bounded by the
-//      wave, not by s: the full-sequence 4h FFN intermediate and the s x s
+//   3. For each wave of query blocks (a whole number of q_block rows, sized
+//      by a tile-round model of the GEMMs): Wo + bo + x (first residual, fp32
+//      hid in the wave scratch), W1 + b1 + ReLU (bf16 U) and W2 + b2 + hid
+//      (second residual, into `out`) on the wave's rows (step 11). Scratch is
+//      bounded by the wave, not by s, and reuses the K/V region, dead once
+//      attention has run: the full-sequence 4h FFN intermediate and the s x s
 //      scores never exist.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -240,11 +241,59 @@ struct Wave {
   long long rows() const { return (long long)n_seq * t_len; }
 };
 
-constexpr int kDefaultWaveRows = 4096;
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-int wave_rows_for(int b, int s, int q_block, int wave_rows) {
-  long long wr = wave_rows > 0 ? wave_rows : kDefaultWaveRows;
-  wr = std::max<long long>(q_block, (wr / q_block) * q_block);
+// Bytes of the K and V copies of the whole sequence (bf16, 1 KB aligned).
+size_t kv_bytes(int b, int s, int h) { return 2 * align_up((size_t)b * s * h * 2, 1024); }
+
+// Bytes of one wave's scratch: fp32 hid, its bf16 copy and the bf16 FFN
+// intermediate U (4h wide), each 1 KB aligned.
+size_t wave_scratch_bytes(long long wr, int h) {
+  return align_up((size_t)wr * h * 4, 1024) + align_up((size_t)wr * h * 2, 1024) +
+         align_up((size_t)wr * 4 * h * 2, 1024);
+}
+
+// Modelled duration of the three FFN-side GEMMs of one wave of `rows` rows,
+// in units of one 128 x 256 x 64 tile step: a persistent launch takes
+// ceil(tiles / SMs) rounds of K/64 steps each, plus a fixed fill/drain cost.
+constexpr int kModelSms = 148;
+constexpr long long kLaunchSteps = 24;
+long long gemm_steps(long long rows, long long n, long long k) {
+  const long long tiles = ((rows + GEMM_BM - 1) / GEMM_BM) * ((n + GEMM_BN - 1) / GEMM_BN);
+  return (tiles + kModelSms - 1) / kModelSms * (k / GEMM_BK) + kLaunchSteps;
+}
+long long wave_steps(long long rows, int h) {
+  if (rows <= 0) return 0;
+  return gemm_steps(rows, h, h) + gemm_steps(rows, 4LL * h, h) + gemm_steps(rows, h, 4LL * h);
+}
+
+// Default wave: the whole number of query blocks (or, when a sequence fits,
+// of whole sequences) whose modelled GEMM time over the layer is within 1% of
+// the best, taking the smallest such wave. The scratch of a wave aliases the
+// K/V copies (dead once attention has run), and is held to 1.5x their size,
+// or to the scratch of a ~4096-row wave where that is larger (small problems).
+int default_wave_rows(int b, int s, int h, int q_block) {
+  const size_t per_row = 14 * (size_t)h;  // 4h + 2h + 8h bytes per row
+  const long long floor_rows = s >= 4096 ? std::max<long long>(q_block, 4096 / q_block * q_block)
+                                         : (long long)std::min(b, 4096 / s) * s;
+  const size_t budget = std::max(kv_bytes(b, s, h) / 2 * 3, wave_scratch_bytes(floor_rows, h));
+  const long long max_rows = std::max<long long>(q_block, (long long)(budget / per_row));
+  std::vector<std::pair<long long, long long>> cand;  // (modelled steps, wave rows)
+  for (long long wr = q_block; wr < s && wr <= max_rows; wr += q_block)
+    cand.push_back({b * ((s / wr) * wave_steps(wr, h) + wave_steps(s % wr, h)), wr});
+  for (long long g = 1; g <= b && (g * s <= max_rows || cand.empty()); ++g)
+    cand.push_back({(b / g) * wave_steps(g * s, h) + wave_steps((b % g) * s, h), g * s});
+  long long best = cand[0].first;
+  for (const auto& c : cand) best = std::min(best, c.first);
+  long long pick = 0;
+  for (const auto& c : cand)
+    if (c.first * 100 <= best * 101 && (pick == 0 || c.second < pick)) pick = c.second;
+  return (int)std::min<long long>(pick, 0x7fffffffLL);
+}
+
+int wave_rows_for(int b, int s, int h, int q_block, int wave_rows) {
+  if (wave_rows <= 0) return default_wave_rows(b, s, h, q_block);
+  long long wr = std::max<long long>(q_block, ((long long)wave_rows / q_block) * q_block);
   if (wr >= s) {
     const long long g = std::max<long long>(1, std::min<long long>(b, wr / s));
     return (int)std::min<long long>(g * s, 0x7fffffffLL);
@@ -252,9 +301,9 @@ int wave_rows_for(int b, int s, int q_block, int wave_rows) {
   return (int)wr;
 }
 
-std::vector<Wave> plan_waves(int b, int s, int q_block, int wave_rows) {
+std::vector<Wave> plan_waves(int b, int s, int h, int q_block, int wave_rows) {
   std::vector<Wave> w;
-  const int wr = wave_rows_for(b, s, q_block, wave_rows);
+  const int wr = wave_rows_for(b, s, h, q_block, wave_rows);
   if (wr >= s) {
     const int g = wr / s;
     for (int beta = 0; beta < b; beta += g) w.push_back(Wave{(long long)beta * s, beta, std::min(g, b - beta), 0, s});
@@ -267,8 +316,9 @@ std::vector<Wave> plan_waves(int b, int s, int q_block, int wave_rows) {
 }
 
 // ------------------------------------------------------------- workspace layout
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
+// Region 0 holds K and V during the projection and attention, then the wave
+// scratch (hid, hb, U) of the FFN side; the f32 entry's bf16 copies of x and
+// the weights follow it.
 struct Layout {
   size_t k, v, hid, hb, u, xb, wqkv, wo, w1, w2, total;
   int wave_rows;
@@ -277,19 +327,19 @@ struct Layout {
 Layout layout_for(int dtype, int b, int s, int h, int q_block, int wave_rows) {
   Layout L{};
   const size_t tok = (size_t)b * s;
-  const int wr = wave_rows_for(b, s, q_block, wave_rows);
+  const int wr = wave_rows_for(b, s, h, q_block, wave_rows);
   L.wave_rows = wr;
-  size_t off = 0;
+  L.k = 0;
+  L.v = align_up(tok * h * 2, 1024);
+  L.hid = 0;
+  L.hb = align_up((size_t)wr * h * 4, 1024);
+  L.u = L.hb + align_up((size_t)wr * h * 2, 1024);
+  size_t off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h));
   auto take = [&](size_t bytes) {
     size_t at = off;
     off = align_up(off + bytes, 1024);
     return at;
   };
-  L.k = take(tok * h * 2);
-  L.v = take(tok * h * 2);
-  L.hid = take((size_t)wr * h * 4);
-  L.hb = take((size_t)wr * h * 2);
-  L.u = take((size_t)wr * 4 * h * 2);
   if (dtype == BPT_DTYPE_F32) {
     L.xb = take(tok * h * 2);
     L.wqkv = take((size_t)h * 3 * h * 2);
@@ -457,7 +507,7 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st));
 
   // step 11 per wave of query blocks: out-projection, residuals and FFN
-  for (const Wave& w : plan_waves(b, s, q_block, wave_rows)) {
+  for (const Wave& w : plan_waves(b, s, h, q_block, wave_rows)) {
     const long long rows = w.rows();
     GemmArgs a{};
     a.resid = p.x;

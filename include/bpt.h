@@ -41,7 +41,8 @@
  * - Blocks: 1 <= q_block <= s, 1 <= kv_block <= s, s % q_block == 0,
  *   s % kv_block == 0 (equal-length blocks). The result does not depend on the
  *   block sizes (the blockwise computation is exact); q_block sets the rows of
- *   each FFN wave, which is a whole number of query blocks.
+ *   each FFN wave, which is a whole number of query blocks (or of whole
+ *   sequences).
  * - causal != 0: key u is visible to query t iff u <= t in the same sequence.
  * - Pointers must be 16-byte aligned (tensor-memory-access tiles).
  * - Errors: argument errors return a negative bpt_status synchronously, with
@@ -104,9 +105,18 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
                           int heads, int q_block, int kv_block, int causal, float* out, void* stream);
 
 /* Bytes of workspace a caller must pass to bpt_layer_forward_ws for these
- * arguments (0 if they are invalid or b*s == 0). wave_rows <= 0 selects the
- * library's default FFN wave (a whole number of query blocks, about 4096 rows);
- * otherwise it is rounded down to a multiple of q_block (at least q_block). */
+ * arguments (0 if they are invalid or b*s == 0): one region that holds the bf16
+ * K and V of the whole input (2 * b*s*h * 2 bytes) until attention is done and
+ * then the FFN scratch of one wave (14 * h bytes per wave row: fp32 residual
+ * stream, its bf16 copy and the 4h-wide bf16 intermediate), so its size is the
+ * larger of the two; the fp32 entry adds bf16 copies of x and the weights.
+ * wave_rows <= 0 selects the library's default FFN wave: the whole number of
+ * query blocks (or of whole sequences) that the library's model of its GEMM
+ * tile rounds finds fastest, with scratch of at most 1.5x the K/V bytes (or of
+ * about 4096 rows, where that is more); 8192 rows at b=1, s=32768, h=4096,
+ * q_block=1024, where the scratch fits inside the K/V region. Otherwise
+ * wave_rows is rounded down to a multiple of q_block (at least q_block), and a
+ * value of s or more groups whole sequences. */
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows);
 
@@ -135,7 +145,7 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
  * - Size limit: returns BPT_ERR_NOMEM, with nothing launched, when the
  *   workspace the layer needs (bpt_layer_workspace_bytes(BPT_DTYPE_BF16, b, s,
  *   h, heads, q_block, kv_block, 0)) exceeds BPT_STATIC_WORKSPACE_BYTES; for
- *   example b=1, s=2048, h=1024 needs 36 MiB and fits, s=8192, h=2048 does not.
+ *   example b=1, s=2048, h=1024 needs 28 MiB and fits, s=8192, h=2048 does not.
  * - The first call on each device looks up that device's address of the array
  *   (one cudaGetSymbolAddress, with that device current). Make that first call
  *   before any stream capture on the device.

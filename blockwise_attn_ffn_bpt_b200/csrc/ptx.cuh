@@ -338,32 +338,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
-// 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU unit.
-// Method: clamp x to >= -125, split x = n + f with n = round-to-nearest(x)
-// obtained by adding and subtracting 1.5 * 2^23 (so f is in [-1/2, 1/2]),
-// evaluate a degree-3 polynomial for 2^f whose coefficients were fitted for
-// this library by Lawson's iteratively reweighted least squares (minimax
-// relative error 8.3e-5 on [-1/2, 1/2]), then add n to the exponent field.
-// Inputs must be finite and <= 127; results below 2^-125 come out as ~2^-125.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t shift = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t t = f2_add(x2, shift);                              // n in the low mantissa bits
-  const uint64_t nf = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));  // n as a float
-  const uint64_t f = f2_fma(nf, f2_pack(-1.0f, -1.0f), x2);          // x - n
-  uint64_t q = f2_fma(f2_pack(0.055212993174791336f, 0.055212993174791336f), f,
-                      f2_pack(0.24271413683891296f, 0.24271413683891296f));
-  q = f2_fma(q, f, f2_pack(0.6932621598243713f, 0.6932621598243713f));
-  q = f2_fma(q, f, f2_pack(0.999919593334198f, 0.999919593334198f));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t, t0, t1);
-  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
-}
-
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -22,8 +22,9 @@ BPT_DTYPE_F32 = 1
 
 EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
-    "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_qkv_projection", "bpt_attention", "bpt_device_status",
-    "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
+    "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
+    "bpt_qkv_projection", "bpt_attention", "bpt_device_status", "bpt_launch_count", "bpt_set_kernel_timing",
+    "bpt_kernel_times",
 )
 
 
@@ -59,6 +60,10 @@ def lib() -> ctypes.CDLL:
     L.bpt_layer_workspace_bytes.argtypes = [i] * 8
     L.bpt_layer_forward_ws.restype = i
     L.bpt_layer_forward_ws.argtypes = [i] + [vp] * 9 + [i] * 8 + [vp, sz, vp, vp]
+    L.bpt_layer_workspace_bytes_ffn.restype = sz
+    L.bpt_layer_workspace_bytes_ffn.argtypes = [i] * 9
+    L.bpt_layer_forward_ffn.restype = i
+    L.bpt_layer_forward_ffn.argtypes = [i] + [vp] * 9 + [i] * 9 + [vp, sz, vp, vp]
     L.bpt_qkv_projection.restype = i
     L.bpt_qkv_projection.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
     L.bpt_attention.restype = i
@@ -101,16 +106,25 @@ PARAM_NAMES = ("Wqkv", "bqkv", "Wo", "bo", "W1", "b1", "W2", "b2")
 
 
 def workspace_bytes(dtype: int, b: int, s: int, h: int, heads: int, q_block: int, kv_block: int,
-                    wave_rows: int = 0) -> int:
-    return int(lib().bpt_layer_workspace_bytes(dtype, b, s, h, heads, q_block, kv_block, wave_rows))
+                    wave_rows: int = 0, ffn: Optional[int] = None) -> int:
+    """Workspace bytes of one call (0 for invalid arguments); ffn defaults to 4h."""
+    if ffn is None:
+        return int(lib().bpt_layer_workspace_bytes(dtype, b, s, h, heads, q_block, kv_block, wave_rows))
+    return int(lib().bpt_layer_workspace_bytes_ffn(dtype, b, s, h, heads, ffn, q_block, kv_block, wave_rows))
+
+
+def _param_shapes(h: int, ffn: int) -> dict:
+    return {"Wqkv": (h, 3 * h), "bqkv": (3 * h,), "Wo": (h, h), "bo": (h,), "W1": (h, ffn), "b1": (ffn,),
+            "W2": (ffn, h), "b2": (h,)}
 
 
 def layer_forward(x: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int, causal: bool,
                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   wave_rows: int = 0, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """One BPT layer forward; x [b, s, h] (bf16 or fp32) on the GPU, params a
-    dict of Wqkv [h,3h], bqkv, Wo [h,h], bo, W1 [h,4h], b1, W2 [4h,h], b2 of
-    x's dtype. Returns out, fp32 [b, s, h].
+    dict of Wqkv [h,3h], bqkv, Wo [h,h], bo, W1 [h,f], b1, W2 [f,h], b2 of
+    x's dtype, with FFN width f = W1's second dimension (4h in the pages; any
+    multiple of 64). Returns out, fp32 [b, s, h].
 
     With workspace=None the library allocates its workspace stream-ordered;
     otherwise `workspace` (a uint8 CUDA tensor of at least workspace_bytes(...))
@@ -126,11 +140,18 @@ def layer_forward(x: torch.Tensor, params: dict, heads: int, q_block: int, kv_bl
         dtype = BPT_DTYPE_F32
     else:
         raise TypeError(f"unsupported dtype {x.dtype}")
-    for k in PARAM_NAMES:
+    ffn = int(params["W1"].shape[-1])
+    for k, shape in _param_shapes(h, ffn).items():
         if params[k].dtype != x.dtype:
             raise TypeError(f"{k} must have dtype {x.dtype}")
+        if tuple(params[k].shape) != shape:
+            raise ValueError(f"{k} has shape {tuple(params[k].shape)}, expected {shape}")
     st = _stream(stream)
-    if workspace is None and wave_rows == 0:
+    if ffn != 4 * h:
+        ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+        r = lib().bpt_layer_forward_ffn(dtype, _ptr(x), *ps, b, s, h, heads, ffn, q_block, kv_block,
+                                        int(bool(causal)), wave_rows, ws_ptr, ws_n, _ptr(out), st)
+    elif workspace is None and wave_rows == 0:
         fn = lib().bpt_layer_forward if dtype == BPT_DTYPE_BF16 else lib().bpt_layer_forward_f32
         r = fn(_ptr(x), *ps, b, s, h, heads, q_block, kv_block, int(bool(causal)), _ptr(out), st)
     else:

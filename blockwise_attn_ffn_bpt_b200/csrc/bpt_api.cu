@@ -247,10 +247,10 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t kv_bytes(int b, int s, int h) { return 2 * align_up((size_t)b * s * h * 2, 1024); }
 
 // Bytes of one wave's scratch: fp32 hid, its bf16 copy and the bf16 FFN
-// intermediate U (4h wide), each 1 KB aligned.
-size_t wave_scratch_bytes(long long wr, int h) {
+// intermediate U (ffn wide), each 1 KB aligned.
+size_t wave_scratch_bytes(long long wr, int h, int ffn) {
   return align_up((size_t)wr * h * 4, 1024) + align_up((size_t)wr * h * 2, 1024) +
-         align_up((size_t)wr * 4 * h * 2, 1024);
+         align_up((size_t)wr * ffn * 2, 1024);
 }
 
 // Modelled duration of the three FFN-side GEMMs of one wave of `rows` rows,
@@ -262,9 +262,9 @@ long long gemm_steps(long long rows, long long n, long long k) {
   const long long tiles = ((rows + GEMM_BM - 1) / GEMM_BM) * ((n + GEMM_BN - 1) / GEMM_BN);
   return (tiles + kModelSms - 1) / kModelSms * (k / GEMM_BK) + kLaunchSteps;
 }
-long long wave_steps(long long rows, int h) {
+long long wave_steps(long long rows, int h, int ffn) {
   if (rows <= 0) return 0;
-  return gemm_steps(rows, h, h) + gemm_steps(rows, 4LL * h, h) + gemm_steps(rows, h, 4LL * h);
+  return gemm_steps(rows, h, h) + gemm_steps(rows, ffn, h) + gemm_steps(rows, h, ffn);
 }
 
 // Default wave: the whole number of query blocks (or, when a sequence fits,
@@ -272,17 +272,17 @@ long long wave_steps(long long rows, int h) {
 // the best, taking the smallest such wave. The scratch of a wave aliases the
 // K/V copies (dead once attention has run), and is held to 1.5x their size,
 // or to the scratch of a ~4096-row wave where that is larger (small problems).
-int default_wave_rows(int b, int s, int h, int q_block) {
-  const size_t per_row = 14 * (size_t)h;  // 4h + 2h + 8h bytes per row
+int default_wave_rows(int b, int s, int h, int ffn, int q_block) {
+  const size_t per_row = 6 * (size_t)h + 2 * (size_t)ffn;  // 4h + 2h + 2 ffn bytes per row
   const long long floor_rows = s >= 4096 ? std::max<long long>(q_block, 4096 / q_block * q_block)
                                          : (long long)std::min(b, 4096 / s) * s;
-  const size_t budget = std::max(kv_bytes(b, s, h) / 2 * 3, wave_scratch_bytes(floor_rows, h));
+  const size_t budget = std::max(kv_bytes(b, s, h) / 2 * 3, wave_scratch_bytes(floor_rows, h, ffn));
   const long long max_rows = std::max<long long>(q_block, (long long)(budget / per_row));
   std::vector<std::pair<long long, long long>> cand;  // (modelled steps, wave rows)
   for (long long wr = q_block; wr < s && wr <= max_rows; wr += q_block)
-    cand.push_back({b * ((s / wr) * wave_steps(wr, h) + wave_steps(s % wr, h)), wr});
+    cand.push_back({b * ((s / wr) * wave_steps(wr, h, ffn) + wave_steps(s % wr, h, ffn)), wr});
   for (long long g = 1; g <= b && (g * s <= max_rows || cand.empty()); ++g)
-    cand.push_back({(b / g) * wave_steps(g * s, h) + wave_steps((b % g) * s, h), g * s});
+    cand.push_back({(b / g) * wave_steps(g * s, h, ffn) + wave_steps((b % g) * s, h, ffn), g * s});
   long long best = cand[0].first;
   for (const auto& c : cand) best = std::min(best, c.first);
   long long pick = 0;
@@ -291,8 +291,8 @@ int default_wave_rows(int b, int s, int h, int q_block) {
   return (int)std::min<long long>(pick, 0x7fffffffLL);
 }
 
-int wave_rows_for(int b, int s, int h, int q_block, int wave_rows) {
-  if (wave_rows <= 0) return default_wave_rows(b, s, h, q_block);
+int wave_rows_for(int b, int s, int h, int ffn, int q_block, int wave_rows) {
+  if (wave_rows <= 0) return default_wave_rows(b, s, h, ffn, q_block);
   long long wr = std::max<long long>(q_block, ((long long)wave_rows / q_block) * q_block);
   if (wr >= s) {
     const long long g = std::max<long long>(1, std::min<long long>(b, wr / s));
@@ -301,9 +301,9 @@ int wave_rows_for(int b, int s, int h, int q_block, int wave_rows) {
   return (int)wr;
 }
 
-std::vector<Wave> plan_waves(int b, int s, int h, int q_block, int wave_rows) {
+std::vector<Wave> plan_waves(int b, int s, int h, int ffn, int q_block, int wave_rows) {
   std::vector<Wave> w;
-  const int wr = wave_rows_for(b, s, h, q_block, wave_rows);
+  const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
   if (wr >= s) {
     const int g = wr / s;
     for (int beta = 0; beta < b; beta += g) w.push_back(Wave{(long long)beta * s, beta, std::min(g, b - beta), 0, s});
@@ -324,17 +324,17 @@ struct Layout {
   int wave_rows;
 };
 
-Layout layout_for(int dtype, int b, int s, int h, int q_block, int wave_rows) {
+Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave_rows) {
   Layout L{};
   const size_t tok = (size_t)b * s;
-  const int wr = wave_rows_for(b, s, h, q_block, wave_rows);
+  const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
   L.wave_rows = wr;
   L.k = 0;
   L.v = align_up(tok * h * 2, 1024);
   L.hid = 0;
   L.hb = align_up((size_t)wr * h * 4, 1024);
   L.u = L.hb + align_up((size_t)wr * h * 2, 1024);
-  size_t off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h));
+  size_t off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h, ffn));
   auto take = [&](size_t bytes) {
     size_t at = off;
     off = align_up(off + bytes, 1024);
@@ -344,8 +344,8 @@ Layout layout_for(int dtype, int b, int s, int h, int q_block, int wave_rows) {
     L.xb = take(tok * h * 2);
     L.wqkv = take((size_t)h * 3 * h * 2);
     L.wo = take((size_t)h * h * 2);
-    L.w1 = take((size_t)h * 4 * h * 2);
-    L.w2 = take((size_t)4 * h * h * 2);
+    L.w1 = take((size_t)h * ffn * 2);
+    L.w2 = take((size_t)ffn * h * 2);
   }
   L.total = off;
   return L;
@@ -437,10 +437,14 @@ struct LayerPtrs {
   const void *x, *Wqkv, *bqkv, *Wo, *bo, *W1, *b1, *W2, *b2;
 };
 
-int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int kv_block,
-                   const float* out) {
+// FFN width: a positive multiple of 64 (one K step of the GEMMs, one TMA box)
+int check_ffn(int ffn) { return (ffn <= 0 || ffn % 64) ? BPT_ERR_SHAPE : BPT_OK; }
+
+int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block,
+                   int kv_block, const float* out) {
   if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return BPT_ERR_DTYPE;
   BPT_TRY(check_shape(b, s, h, heads));
+  BPT_TRY(check_ffn(ffn));
   BPT_TRY(check_blocks(s, q_block, kv_block));
   if ((long long)b * s == 0) return BPT_OK;
   const void* ptrs[10] = {p.x, p.Wqkv, p.bqkv, p.Wo, p.bo, p.W1, p.b1, p.W2, p.b2, out};
@@ -452,16 +456,16 @@ int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads
   const size_t tok = (size_t)b * s;
   const Range ro = rng(out, tok * h * 4);
   const Range in[9] = {rng(p.x, tok * h * es),      rng(p.Wqkv, (size_t)h * 3 * h * es), rng(p.bqkv, 3 * (size_t)h * es),
-                       rng(p.Wo, (size_t)h * h * es), rng(p.bo, (size_t)h * es),          rng(p.W1, (size_t)h * 4 * h * es),
-                       rng(p.b1, 4 * (size_t)h * es), rng(p.W2, (size_t)4 * h * h * es),    rng(p.b2, (size_t)h * es)};
+                       rng(p.Wo, (size_t)h * h * es), rng(p.bo, (size_t)h * es),          rng(p.W1, (size_t)h * ffn * es),
+                       rng(p.b1, (size_t)ffn * es), rng(p.W2, (size_t)ffn * h * es),       rng(p.b2, (size_t)h * es)};
   for (const Range& r : in)
     if (overlap(ro, r)) return BPT_ERR_ALIAS;
   return BPT_OK;
 }
 
-int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int causal,
+int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
               int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms) {
-  const Layout L = layout_for(dtype, b, s, h, q_block, wave_rows);
+  const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
   const long long tok = (long long)b * s;
   __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(ws + L.k);
   __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(ws + L.v);
@@ -479,8 +483,8 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     BPT_TRY(launch_convert((const float*)p.x, ws + L.xb, tok * h, sms, st));
     BPT_TRY(launch_convert((const float*)p.Wqkv, ws + L.wqkv, 3LL * h * h, sms, st));
     BPT_TRY(launch_convert((const float*)p.Wo, ws + L.wo, 1LL * h * h, sms, st));
-    BPT_TRY(launch_convert((const float*)p.W1, ws + L.w1, 4LL * h * h, sms, st));
-    BPT_TRY(launch_convert((const float*)p.W2, ws + L.w2, 4LL * h * h, sms, st));
+    BPT_TRY(launch_convert((const float*)p.W1, ws + L.w1, (long long)h * ffn, sms, st));
+    BPT_TRY(launch_convert((const float*)p.W2, ws + L.w2, (long long)ffn * h, sms, st));
     xa = ws + L.xb;
     wqkv = ws + L.wqkv;
     wo = ws + L.wo;
@@ -507,7 +511,7 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st));
 
   // step 11 per wave of query blocks: out-projection, residuals and FFN
-  for (const Wave& w : plan_waves(b, s, h, q_block, wave_rows)) {
+  for (const Wave& w : plan_waves(b, s, h, ffn, q_block, wave_rows)) {
     const long long rows = w.rows();
     GemmArgs a{};
     a.resid = p.x;
@@ -525,19 +529,20 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     BPT_TRY(launch_gemm<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, h, a, sms, st, "gemm_outproj"));
     a.bias = p.b1;
     a.dst = U;
-    a.ld_dst = 4LL * h;
-    BPT_TRY(launch_gemm<EPI_FFN_UP>(HB, rows, h, h, w1, 4LL * h, a, sms, st, "gemm_ffn_up"));
+    a.ld_dst = ffn;
+    BPT_TRY(launch_gemm<EPI_FFN_UP>(HB, rows, h, h, w1, ffn, a, sms, st, "gemm_ffn_up"));
     a.bias = p.b2;
-    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(U, rows, 4LL * h, 4LL * h, w2, h, a, sms, st, "gemm_ffn_down"));
+    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, h, a, sms, st, "gemm_ffn_down"));
   }
   return BPT_OK;
 }
 
-int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
-                int wave_rows, void* workspace, size_t ws_bytes, bool caller_ws, float* out, void* stream) {
-  BPT_TRY(validate_layer(dtype, p, b, s, h, heads, q_block, kv_block, out));
+int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int kv_block,
+                int causal, int wave_rows, void* workspace, size_t ws_bytes, bool caller_ws, float* out,
+                void* stream) {
+  BPT_TRY(validate_layer(dtype, p, b, s, h, heads, ffn, q_block, kv_block, out));
   if ((long long)b * s == 0) return BPT_OK;
-  const Layout L = layout_for(dtype, b, s, h, q_block, wave_rows);
+  const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
   if (caller_ws) {
     if (!workspace) return BPT_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BPT_ERR_ALIGN;
@@ -547,7 +552,7 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
     const Range rw = rng(workspace, L.total);
     const Range others[10] = {rng(out, tok * h * 4),      rng(p.x, tok * h * es),        rng(p.Wqkv, (size_t)3 * h * h * es),
                               rng(p.bqkv, (size_t)3 * h * es), rng(p.Wo, (size_t)h * h * es), rng(p.bo, (size_t)h * es),
-                              rng(p.W1, (size_t)4 * h * h * es), rng(p.b1, (size_t)4 * h * es), rng(p.W2, (size_t)4 * h * h * es),
+                              rng(p.W1, (size_t)h * ffn * es), rng(p.b1, (size_t)ffn * es), rng(p.W2, (size_t)ffn * h * es),
                               rng(p.b2, (size_t)h * es)};
     for (const Range& r : others)
       if (overlap(rw, r)) return BPT_ERR_ALIAS;
@@ -566,7 +571,7 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
     }
     ws = reinterpret_cast<uint8_t*>(m);
   }
-  const int r = run_layer(dtype, p, b, s, h, heads, q_block, causal, wave_rows, ws, out, st, sms);
+  const int r = run_layer(dtype, p, b, s, h, heads, ffn, q_block, causal, wave_rows, ws, out, st, sms);
   if (!caller_ws) cudaFreeAsync(ws, st);
   return r;
 }
@@ -625,22 +630,33 @@ int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const v
                       const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                       int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
   const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
-  return layer_entry(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, kv_block, causal, 0, nullptr, 0, false, out, stream);
+  if (check_shape(b, s, h, heads) != BPT_OK) return BPT_ERR_SHAPE;
+  return layer_entry(BPT_DTYPE_BF16, p, b, s, h, heads, 4 * h, q_block, kv_block, causal, 0, nullptr, 0, false, out,
+                     stream);
 }
 
 int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, const float* Wo, const float* bo,
                           const float* W1, const float* b1, const float* W2, const float* b2, int b, int s, int h,
                           int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
   const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
-  return layer_entry(BPT_DTYPE_F32, p, b, s, h, heads, q_block, kv_block, causal, 0, nullptr, 0, false, out, stream);
+  if (check_shape(b, s, h, heads) != BPT_OK) return BPT_ERR_SHAPE;
+  return layer_entry(BPT_DTYPE_F32, p, b, s, h, heads, 4 * h, q_block, kv_block, causal, 0, nullptr, 0, false, out,
+                     stream);
+}
+
+size_t bpt_layer_workspace_bytes_ffn(int dtype, int b, int s, int h, int heads, int ffn, int q_block, int kv_block,
+                                     int wave_rows) {
+  if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return 0;
+  if (check_shape(b, s, h, heads) != BPT_OK || check_blocks(s, q_block, kv_block) != BPT_OK) return 0;
+  if (check_ffn(ffn) != BPT_OK) return 0;
+  if ((long long)b * s == 0) return 0;
+  return layout_for(dtype, b, s, h, ffn, q_block, wave_rows).total;
 }
 
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows) {
-  if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return 0;
-  if (check_shape(b, s, h, heads) != BPT_OK || check_blocks(s, q_block, kv_block) != BPT_OK) return 0;
-  if ((long long)b * s == 0) return 0;
-  return layout_for(dtype, b, s, h, q_block, wave_rows).total;
+  if (check_shape(b, s, h, heads) != BPT_OK) return 0;
+  return bpt_layer_workspace_bytes_ffn(dtype, b, s, h, heads, 4 * h, q_block, kv_block, wave_rows);
 }
 
 int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
@@ -648,24 +664,36 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
                          int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
                          void* workspace, size_t ws_bytes, float* out, void* stream) {
   const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
-  return layer_entry(dtype, p, b, s, h, heads, q_block, kv_block, causal, wave_rows, workspace, ws_bytes, true, out,
-                     stream);
+  if (check_shape(b, s, h, heads) != BPT_OK) return BPT_ERR_SHAPE;
+  return layer_entry(dtype, p, b, s, h, heads, 4 * h, q_block, kv_block, causal, wave_rows, workspace, ws_bytes, true,
+                     out, stream);
+}
+
+int bpt_layer_forward_ffn(int dtype, const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
+                          const void* bo, const void* W1, const void* b1, const void* W2, const void* b2, int b,
+                          int s, int h, int heads, int ffn, int q_block, int kv_block, int causal, int wave_rows,
+                          void* workspace, size_t ws_bytes, float* out, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  const bool caller_ws = workspace != nullptr || ws_bytes != 0;
+  return layer_entry(dtype, p, b, s, h, heads, ffn, q_block, kv_block, causal, wave_rows, workspace, ws_bytes,
+                     caller_ws, out, stream);
 }
 
 int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
                               const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                               int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
   const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
-  BPT_TRY(validate_layer(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, kv_block, out));
+  BPT_TRY(check_shape(b, s, h, heads));
+  BPT_TRY(validate_layer(BPT_DTYPE_BF16, p, b, s, h, heads, 4 * h, q_block, kv_block, out));
   if ((long long)b * s == 0) return BPT_OK;
-  const Layout L = layout_for(BPT_DTYPE_BF16, b, s, h, q_block, 0);
+  const Layout L = layout_for(BPT_DTYPE_BF16, b, s, h, 4 * h, q_block, 0);
   if (L.total > BPT_STATIC_WORKSPACE_BYTES) return BPT_ERR_NOMEM;
   int sms = 0;
   BPT_TRY(check_device(&sms));
   void* ws = nullptr;
   BPT_TRY(static_workspace(&ws));
-  return run_layer(BPT_DTYPE_BF16, p, b, s, h, heads, q_block, causal, 0, reinterpret_cast<uint8_t*>(ws), out,
-                   reinterpret_cast<cudaStream_t>(stream), sms);
+  return run_layer(BPT_DTYPE_BF16, p, b, s, h, heads, 4 * h, q_block, causal, 0, reinterpret_cast<uint8_t*>(ws),
+                   out, reinterpret_cast<cudaStream_t>(stream), sms);
 }
 
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,

@@ -132,6 +132,7 @@ class LayerShape:
     kv_block: int
     causal: bool
     dtype: str = "bf16"  # "bf16" or "f32": the precision the inputs are rounded to
+    ffn: int = 0  # FFN width; 0 means the pages' 4h
 
     @property
     def dh(self) -> int:
@@ -139,7 +140,7 @@ class LayerShape:
 
     @property
     def f(self) -> int:
-        return 4 * self.h
+        return self.ffn if self.ffn else 4 * self.h
 
 
 def tensor_shapes(shape: LayerShape) -> dict:

@@ -120,6 +120,21 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows);
 
+/* The layer with an FFN of any width ffn (the pages fix ffn = 4h; every
+ * other entry point uses 4h): W1 is [h, ffn], b1 [ffn], W2 [ffn, h], in the
+ * element type dtype. ffn must be a positive multiple of 64 (BPT_ERR_SHAPE
+ * otherwise). workspace == NULL with ws_bytes == 0 takes the workspace from
+ * the library's stream-ordered pool, as bpt_layer_forward does; otherwise it
+ * is caller-owned with the rules of bpt_layer_forward_ws and must hold
+ * bpt_layer_workspace_bytes_ffn(...) bytes. All other arguments, the result
+ * and the error behaviour are those of bpt_layer_forward_ws. */
+size_t bpt_layer_workspace_bytes_ffn(int dtype, int b, int s, int h, int heads, int ffn, int q_block, int kv_block,
+                                     int wave_rows);
+int bpt_layer_forward_ffn(int dtype, const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
+                          const void* bo, const void* W1, const void* b1, const void* W2, const void* b2, int b,
+                          int s, int h, int heads, int ffn, int q_block, int kv_block, int causal, int wave_rows,
+                          void* workspace, size_t ws_bytes, float* out, void* stream);
+
 /* The layer with a caller-owned workspace (device memory, 256-byte aligned,
  * at least bpt_layer_workspace_bytes(...) bytes, not overlapping any argument;
  * BPT_ERR_NOMEM if ws_bytes is too small). dtype is a bpt_dtype and gives the

@@ -33,7 +33,8 @@ notes of the repository):
 * "Attention(Q_i, K, V)" in the residual formula includes the output
   projection Wo, bo, and the residual adds the layer input block x_i (the
   figure caption: the input block is what gets projected to a query).
-* No LayerNorm and no dropout (deterministic forward); FFN width 4h.
+* No LayerNorm and no dropout (deterministic forward); FFN width 4h in the
+  pages, taken here from the shapes of W1 [h, f] and W2 [f, h], so any f.
 * Causal mask: key u is allowed for query t iff u <= t within the same
   sequence; a masked score has weight exactly 0.
 * Weights are [in, out] (x @ W); Wqkv's columns are [W_Q | W_K | W_V], and

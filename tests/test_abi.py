@@ -137,6 +137,38 @@ def test_workspace_bytes_follow_the_layout():
     assert bpt.workspace_bytes(0, 0, 256, 256, 4, 64, 64) == 0
 
 
+def test_ffn_width_entry_validates_and_sizes_its_workspace():
+    L = bpt.lib()
+    p = fake_ptrs(9)
+    out = BASE + 20 * STEP
+
+    def up(v):
+        return (v + 1023) // 1024 * 1024
+
+    # the FFN width must be a positive multiple of 64; refused before any CUDA call
+    for bad in (0, -64, 32, 100):
+        assert L.bpt_layer_forward_ffn(0, *p, 1, 256, 256, 4, bad, 64, 64, 1, 0, None, 0, out, None) == SHAPE
+        assert bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, ffn=bad) == 0
+    # 4h through the general entry is the default layout
+    for wr in (0, 128, 1000):
+        assert bpt.workspace_bytes(0, 2, 512, 256, 4, 64, 64, wr, ffn=1024) == \
+            bpt.workspace_bytes(0, 2, 512, 256, 4, 64, 64, wr)
+    # one region: K and V, or the wave scratch with an ffn-wide U
+    assert bpt.workspace_bytes(0, 1, 2048, 1024, 16, 128, 128, 512, ffn=192) == \
+        max(2 * up(2048 * 1024 * 2), up(512 * 1024 * 4) + up(512 * 1024 * 2) + up(512 * 192 * 2))
+    assert bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 256, ffn=4096) == \
+        max(2 * up(256 * 256 * 2), up(256 * 256 * 4) + up(256 * 256 * 2) + up(256 * 4096 * 2))
+    # fp32 inputs add bf16 copies of W1 [h, f] and W2 [f, h]
+    f32 = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64, 256, ffn=640)
+    b16 = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 256, ffn=640)
+    assert f32 == b16 + up(256 * 256 * 2) + up(3 * 256 * 256 * 2) + up(256 * 256 * 2) + 2 * up(256 * 640 * 2)
+    # a too-small caller workspace and a misaligned one are refused
+    need = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 0, ffn=512)
+    ws = BASE + 30 * STEP
+    assert L.bpt_layer_forward_ffn(0, *p, 1, 256, 256, 4, 512, 64, 64, 1, 0, ws, need - 1, out, None) == NOMEM
+    assert L.bpt_layer_forward_ffn(0, *p, 1, 256, 256, 4, 512, 64, 64, 1, 0, ws + 16, need, out, None) == ALIGN
+
+
 def test_stage_entry_points_validate():
     L = bpt.lib()
     p = fake_ptrs(6)

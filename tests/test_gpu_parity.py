@@ -55,7 +55,8 @@ def run_layer(shape, inp, wave_rows=0, workspace=False):
     params = device_params(inp)
     if workspace:
         nbytes = bpt.workspace_bytes(bpt.BPT_DTYPE_F32 if shape.dtype == "f32" else bpt.BPT_DTYPE_BF16,
-                                     shape.b, shape.s, shape.h, shape.heads, shape.q_block, shape.kv_block, wave_rows)
+                                     shape.b, shape.s, shape.h, shape.heads, shape.q_block, shape.kv_block, wave_rows,
+                                     ffn=shape.f)
         ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
         out = bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
                                 workspace=ws, wave_rows=wave_rows)
@@ -169,6 +170,25 @@ def test_layer_small_matches_oracle(shape):
     ref = oracle_full(shape, inp)
     got = run_layer(shape, inp)
     assert_parity(got, ref, str(shape))
+
+
+# FFN widths other than the pages' 4h (bpt_layer_forward_ffn): f = h, a width
+# that leaves a partial 256-column tile and three 64-deep K steps, f = 8h, and
+# the fp32 entry with f = 5h/3
+FFN_SHAPES = [
+    bi.LayerShape(1, 256, 256, 4, 64, 64, True, "bf16", ffn=256),
+    bi.LayerShape(2, 200, 256, 2, 40, 100, False, "bf16", ffn=192),
+    bi.LayerShape(1, 320, 256, 4, 64, 160, True, "bf16", ffn=2048),
+    bi.LayerShape(1, 256, 384, 3, 128, 64, True, "f32", ffn=640),
+]
+
+
+@pytest.mark.parametrize("shape", FFN_SHAPES, ids=lambda s: f"f{s.f}h{s.h}{s.dtype}")
+@pytest.mark.parametrize("workspace", [False, True])
+def test_layer_any_ffn_width_matches_oracle(shape, workspace):
+    inp = bi.make_inputs(shape, seed=5)
+    got = run_layer(shape, inp, workspace=workspace)
+    assert_parity(got, oracle_full(shape, inp), f"ffn {shape.f}: {shape}")
 
 
 @pytest.mark.parametrize("wave_rows", [64, 128, 384, 100000])

@@ -71,3 +71,18 @@ def test_make_inputs_shapes_and_scales():
     assert abs(bi.to_f64(inp["b1"]).std() - 0.02) < 0.004
     f32 = bi.make_inputs(bi.LayerShape(1, 8, 64, 1, 8, 8, False, "f32"))
     assert f32["x"].dtype == np.float32
+
+
+def test_ffn_width_sets_the_ffn_shapes_and_keeps_the_streams():
+    base = bi.LayerShape(1, 8, 64, 1, 8, 8, True)
+    wide = bi.LayerShape(1, 8, 64, 1, 8, 8, True, ffn=192)
+    assert base.f == 256 and wide.f == 192
+    shp = bi.tensor_shapes(wide)
+    assert shp["W1"] == (64, 192) and shp["b1"] == (192,) and shp["W2"] == (192, 64)
+    assert bi.tensor_std("W2", wide) == 1.0 / math.sqrt(192)
+    assert bi.tensor_std("W1", wide) == 1.0 / math.sqrt(64)
+    a, b = bi.make_inputs(base, seed=3), bi.make_inputs(wide, seed=3)
+    # same counter streams: tensors of equal shape are identical, W1 is a prefix
+    for k in ("x", "Wqkv", "bqkv", "Wo", "bo", "b2"):
+        assert np.array_equal(a[k], b[k])
+    assert np.array_equal(a["W1"].reshape(-1)[: 64 * 192], b["W1"].reshape(-1))

@@ -25,10 +25,11 @@ import oracle
 # helpers
 # ---------------------------------------------------------------------------
 
-def rand_layer(b, s, h, heads, seed=0, scale_q=1.0):
-    """Random fp64 layer parameters (plain numpy RNG; exactness tests need no bf16)."""
+def rand_layer(b, s, h, heads, seed=0, scale_q=1.0, f=None):
+    """Random fp64 layer parameters (plain numpy RNG; exactness tests need no bf16);
+    FFN width f (4h unless given)."""
     rng = np.random.default_rng(seed)
-    f = 4 * h
+    f = 4 * h if f is None else f
     p = dict(
         x=rng.standard_normal((b, s, h)),
         Wqkv=rng.standard_normal((h, 3 * h)) / math.sqrt(h),
@@ -99,6 +100,17 @@ def test_layer_equals_brute_force(b, s, h, heads, causal):
     p = rand_layer(b, s, h, heads, seed=s * 10 + h)
     ref = brute_force_layer(p, heads, causal)
     got = oracle.layer_forward(*args(p), heads=heads, causal=causal, threads=1)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("f", [1, 3, 8, 20])
+@pytest.mark.parametrize("causal", [False, True])
+def test_layer_equals_brute_force_any_ffn_width(f, causal):
+    # the oracle takes the FFN width from W1/W2, so widths other than 4h follow
+    # the same definition
+    p = rand_layer(2, 3, 4, 2, seed=f, f=f)
+    ref = brute_force_layer(p, 2, causal)
+    got = oracle.layer_forward(*args(p), heads=2, causal=causal, threads=1)
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
 
 

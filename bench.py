@@ -331,26 +331,23 @@ def our_arm(args, shape, name):
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, dist, device)
 
-    # ---- end to end through the public API from pinned host memory
+    # ---- end to end through the C ABI's host-memory entry (bpt_layer_forward_host):
+    # every step copies its input from pinned host memory and its result back;
+    # the library overlaps step i's copies with the compute of steps i -/+ 1
     x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     x_host.copy_(x)
     out_host = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
-    x_dev = torch.empty_like(x)
-    for _ in range(max(1, args.warmup // 2)):
-        bpt.layer_forward_from_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
-                                    out_host=out_host, x_dev=x_dev, out_dev=out, stream=stream)
+    torch.cuda.synchronize(device)
+    bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+                           out_host=out_host, n_inputs=max(1, args.warmup // 2), stream=stream)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(dist, device)
     torch.cuda.synchronize(device)
+    e2e_steps = max(1, args.steps)
     e0.record(stream)
-    e2e_steps = max(1, min(args.steps, 5))
-    for _ in range(e2e_steps):
-        with torch.cuda.stream(stream):
-            x_dev.copy_(x_host, non_blocking=True)
-            bpt.layer_forward(x_dev, params, shape.heads, shape.q_block, shape.kv_block, shape.causal, out=out,
-                              stream=stream)
-            out_host.copy_(out, non_blocking=True)
+    bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+                           out_host=out_host, n_inputs=e2e_steps, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier(dist, device)
@@ -405,7 +402,8 @@ def our_arm(args, shape, name):
         "cpu_baseline": cpu,
         "e2e": {"value": tokens * e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
-                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+                "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+                "steps": e2e_steps, "api": "bpt_layer_forward_host (pinned host buffers)"},
         "gpu_launches": int(launches),
         "kernels": kernel_table,
         "clocks": clocks.summary(),

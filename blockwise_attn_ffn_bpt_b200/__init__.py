@@ -23,6 +23,7 @@ BPT_DTYPE_F32 = 1
 EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
     "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
+    "bpt_layer_forward_host",
     "bpt_qkv_projection", "bpt_attention", "bpt_device_status", "bpt_launch_count", "bpt_set_kernel_timing",
     "bpt_kernel_times",
 )
@@ -64,6 +65,9 @@ def lib() -> ctypes.CDLL:
     L.bpt_layer_workspace_bytes_ffn.argtypes = [i] * 9
     L.bpt_layer_forward_ffn.restype = i
     L.bpt_layer_forward_ffn.argtypes = [i] + [vp] * 9 + [i] * 9 + [vp, sz, vp, vp]
+    ll = ctypes.c_longlong
+    L.bpt_layer_forward_host.restype = i
+    L.bpt_layer_forward_host.argtypes = [i, vp, ll] + [vp] * 8 + [i] * 7 + [vp, ll, i, vp]
     L.bpt_qkv_projection.restype = i
     L.bpt_qkv_projection.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
     L.bpt_attention.restype = i
@@ -164,28 +168,55 @@ def layer_forward(x: torch.Tensor, params: dict, heads: int, q_block: int, kv_bl
     return out
 
 
+def layer_forward_host(x_host: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int, causal: bool,
+                       out_host: Optional[torch.Tensor] = None, n_inputs: Optional[int] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """End to end from host memory through bpt_layer_forward_host.
+
+    x_host is a host tensor [n, b, s, h] of n inputs, or [b, s, h] used
+    n_inputs times (default 1); bf16 or fp32, pinned for the copies to overlap
+    the compute. Weights are on the GPU. Returns out_host (fp32, [n, b, s, h]
+    or [b, s, h] holding the last result), after every result has arrived.
+    """
+    if x_host.is_cuda:
+        raise ValueError("x_host must be in host memory")
+    if x_host.dim() == 4:
+        n, b, s, h = x_host.shape
+        x_stride = b * s * h * x_host.element_size()
+        shape = (n, b, s, h)
+    else:
+        b, s, h = x_host.shape
+        n = 1 if n_inputs is None else int(n_inputs)
+        x_stride = 0
+        shape = (b, s, h)
+    if out_host is None:
+        out_host = torch.empty(shape, dtype=torch.float32, pin_memory=True)
+    if tuple(out_host.shape) != shape or out_host.dtype != torch.float32 or out_host.is_cuda:
+        raise ValueError(f"out_host must be a host fp32 tensor of shape {shape}")
+    out_stride = b * s * h * 4 if x_host.dim() == 4 else 0
+    if x_host.dtype == torch.bfloat16:
+        dtype = BPT_DTYPE_BF16
+    elif x_host.dtype == torch.float32:
+        dtype = BPT_DTYPE_F32
+    else:
+        raise TypeError(f"unsupported dtype {x_host.dtype}")
+    for k, shp in _param_shapes(h, 4 * h).items():
+        if params[k].dtype != x_host.dtype or tuple(params[k].shape) != shp or not params[k].is_cuda:
+            raise ValueError(f"{k} must be a CUDA {x_host.dtype} tensor of shape {shp}")
+    ps = [_ptr(params[k]) for k in PARAM_NAMES]
+    dev = params["Wqkv"].device
+    st = (stream if stream is not None else torch.cuda.current_stream(dev)).cuda_stream
+    r = lib().bpt_layer_forward_host(dtype, _ptr(x_host), x_stride, *ps, b, s, h, heads, q_block, kv_block,
+                                     int(bool(causal)), _ptr(out_host), out_stride, n, st)
+    _check(r, "bpt_layer_forward_host")
+    return out_host
+
+
 def layer_forward_from_host(x_host: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int,
                             causal: bool, out_host: Optional[torch.Tensor] = None,
-                            x_dev: Optional[torch.Tensor] = None, out_dev: Optional[torch.Tensor] = None,
                             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """End-to-end call from host memory: copy x (pinned host) to the device,
-    run the layer (weights already resident on the device), copy out back to
-    (pinned) host memory. Returns out_host after the stream has finished."""
-    b, s, h = x_host.shape
-    dev = params["Wqkv"].device
-    st = stream if stream is not None else torch.cuda.current_stream(dev)
-    if x_dev is None:
-        x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device=dev)
-    if out_dev is None:
-        out_dev = torch.empty((b, s, h), dtype=torch.float32, device=dev)
-    if out_host is None:
-        out_host = torch.empty((b, s, h), dtype=torch.float32, pin_memory=True)
-    with torch.cuda.stream(st):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer_forward(x_dev, params, heads, q_block, kv_block, causal, out=out_dev, stream=st)
-        out_host.copy_(out_dev, non_blocking=True)
-    st.synchronize()
-    return out_host
+    """One input [b, s, h] from host memory to a host fp32 result (see layer_forward_host)."""
+    return layer_forward_host(x_host, params, heads, q_block, kv_block, causal, out_host=out_host, stream=stream)
 
 
 def qkv_projection(x: torch.Tensor, Wqkv: torch.Tensor, bqkv: torch.Tensor,

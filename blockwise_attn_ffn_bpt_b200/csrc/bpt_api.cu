@@ -602,6 +602,110 @@ int static_workspace(void** ptr) {
   return BPT_OK;
 }
 
+// n independent inputs from host memory: input i is copied in while input
+// i - 1 computes, and its result is copied out while input i + 1 computes.
+// Two device buffers each for x and out plus one workspace come from the
+// library's pool; two non-blocking copy streams are ordered against the
+// compute stream with events; every copy is one cudaMemcpyAsync.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ready = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+  bool create() {
+    if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
+    cudaEvent_t* all[7] = {&ready, &h2d_done[0], &h2d_done[1], &comp_done[0], &comp_done[1], &d2h_done[0],
+                           &d2h_done[1]};
+    for (cudaEvent_t* e : all)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  void destroy() {
+    if (h2d) cudaStreamSynchronize(h2d), cudaStreamDestroy(h2d);
+    if (d2h) cudaStreamSynchronize(d2h), cudaStreamDestroy(d2h);
+    cudaEvent_t all[7] = {ready, h2d_done[0], h2d_done[1], comp_done[0], comp_done[1], d2h_done[0], d2h_done[1]};
+    for (cudaEvent_t e : all)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtrs& w, int b, int s, int h,
+               int heads, int q_block, int kv_block, int causal, float* out_host, long long out_stride, int n,
+               void* stream) {
+  if (dtype != BPT_DTYPE_BF16 && dtype != BPT_DTYPE_F32) return BPT_ERR_DTYPE;
+  BPT_TRY(check_shape(b, s, h, heads));
+  BPT_TRY(check_blocks(s, q_block, kv_block));
+  if (n < 0) return BPT_ERR_SHAPE;
+  const size_t es = dtype == BPT_DTYPE_F32 ? 4 : 2;
+  const size_t tok = (size_t)b * s;
+  const size_t xb = tok * h * es, ob = tok * h * 4;
+  if (n == 0 || tok == 0) return BPT_OK;
+  const void* dev_ptrs[8] = {w.Wqkv, w.bqkv, w.Wo, w.bo, w.W1, w.b1, w.W2, w.b2};
+  if (!x_host || !out_host) return BPT_ERR_NULL;
+  for (const void* q : dev_ptrs)
+    if (!q) return BPT_ERR_NULL;
+  for (const void* q : dev_ptrs)
+    if (!aligned16(q)) return BPT_ERR_ALIGN;
+  if (x_stride < 0 || out_stride < 0 || (x_stride && (size_t)x_stride < xb) || (out_stride && (size_t)out_stride < ob))
+    return BPT_ERR_SHAPE;
+  // host ranges: every input against every output (both are arithmetic progressions)
+  const Range xr = rng(x_host, (size_t)x_stride * (n - 1) + xb), orr = rng(out_host, (size_t)out_stride * (n - 1) + ob);
+  if (overlap(xr, orr)) return BPT_ERR_ALIAS;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  const Layout L = layout_for(dtype, b, s, h, 4 * h, q_block, 0);
+  const size_t xa = align_up(xb, 1024), oa = align_up(ob, 1024);
+  const size_t total = 2 * xa + 2 * oa + L.total;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaMemPool_t pool = nullptr;
+  BPT_TRY(workspace_pool(&pool));
+  void* mem = nullptr;
+  if (cudaMallocFromPoolAsync(&mem, total, pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return BPT_ERR_NOMEM;
+  }
+  uint8_t* base = reinterpret_cast<uint8_t*>(mem);
+  uint8_t* xdev[2] = {base, base + xa};
+  float* odev[2] = {reinterpret_cast<float*>(base + 2 * xa), reinterpret_cast<float*>(base + 2 * xa + oa)};
+  uint8_t* ws = base + 2 * xa + 2 * oa;
+  HostPipe pp;
+  int r = pp.create() ? BPT_OK : BPT_ERR_CUDA;
+  if (r == BPT_OK) {
+    bool cu = cudaEventRecord(pp.ready, st) == cudaSuccess && cudaStreamWaitEvent(pp.h2d, pp.ready, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(pp.d2h, pp.ready, 0) == cudaSuccess;
+    for (int i = 0; cu && r == BPT_OK && i < n; ++i) {
+      const int k = i & 1;
+      const uint8_t* xi = reinterpret_cast<const uint8_t*>(x_host) + (size_t)x_stride * i;
+      uint8_t* oi = reinterpret_cast<uint8_t*>(out_host) + (size_t)out_stride * i;
+      // x buffer k is free once input i - 2 has been computed
+      if (i >= 2) cu = cu && cudaStreamWaitEvent(pp.h2d, pp.comp_done[k], 0) == cudaSuccess;
+      cu = cu && cudaMemcpyAsync(xdev[k], xi, xb, cudaMemcpyHostToDevice, pp.h2d) == cudaSuccess &&
+           cudaEventRecord(pp.h2d_done[k], pp.h2d) == cudaSuccess;
+      // out buffer k is free once result i - 2 has been copied out
+      cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k], 0) == cudaSuccess;
+      if (i >= 2) cu = cu && cudaStreamWaitEvent(st, pp.d2h_done[k], 0) == cudaSuccess;
+      if (!cu) break;
+      LayerPtrs p = w;
+      p.x = xdev[k];
+      r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms);
+      if (r != BPT_OK) break;
+      cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess &&
+           cudaStreamWaitEvent(pp.d2h, pp.comp_done[k], 0) == cudaSuccess &&
+           cudaMemcpyAsync(oi, odev[k], ob, cudaMemcpyDeviceToHost, pp.d2h) == cudaSuccess &&
+           cudaEventRecord(pp.d2h_done[k], pp.d2h) == cudaSuccess;
+    }
+    if (!cu && r == BPT_OK) r = BPT_ERR_CUDA;
+  }
+  // the buffers go back to the pool only after every copy has finished
+  if (pp.h2d && pp.d2h) {
+    if (cudaStreamSynchronize(pp.h2d) != cudaSuccess || cudaStreamSynchronize(pp.d2h) != cudaSuccess)
+      if (r == BPT_OK) r = BPT_ERR_CUDA;
+  }
+  cudaFreeAsync(mem, st);
+  if (cudaStreamSynchronize(st) != cudaSuccess && r == BPT_OK) r = BPT_ERR_CUDA;
+  pp.destroy();
+  return r;
+}
+
 }  // namespace
 }  // namespace bpt
 
@@ -694,6 +798,15 @@ int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv,
   BPT_TRY(static_workspace(&ws));
   return run_layer(BPT_DTYPE_BF16, p, b, s, h, heads, 4 * h, q_block, causal, 0, reinterpret_cast<uint8_t*>(ws),
                    out, reinterpret_cast<cudaStream_t>(stream), sms);
+}
+
+int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, const void* Wqkv, const void* bqkv,
+                           const void* Wo, const void* bo, const void* W1, const void* b1, const void* W2,
+                           const void* b2, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
+                           float* out_host, long long out_stride, int n_inputs, void* stream) {
+  const LayerPtrs w{nullptr, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  return host_entry(dtype, x_host, x_stride, w, b, s, h, heads, q_block, kv_block, causal, out_host, out_stride,
+                    n_inputs, stream);
 }
 
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,

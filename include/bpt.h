@@ -144,6 +144,25 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
                          int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
                          void* workspace, size_t ws_bytes, float* out, void* stream);
 
+/* End to end from host memory: for i in [0, n_inputs), out_host + i *
+ * out_stride receives the layer applied to x_host + i * x_stride (strides in
+ * bytes; 0 reuses the same input, or writes every result to the same place).
+ * x is [b, s, h] of dtype (bf16 or fp32) in host memory; out is fp32 [b, s, h]
+ * in host memory; the weights and biases are device pointers as for
+ * bpt_layer_forward. Host buffers should be pinned (page-locked) for the
+ * copies to overlap the compute; pageable memory works, slower. Input i is
+ * copied in while input i - 1 computes and its result copied out while input
+ * i + 1 computes (two device buffers each for x and out and one workspace,
+ * from the library's pool; two internal copy streams ordered by events
+ * against `stream`, which runs the layer). Returns after every result has
+ * reached host memory. Errors as bpt_layer_forward; BPT_ERR_SHAPE also for
+ * n_inputs < 0 or a nonzero stride smaller than one input (output); and
+ * BPT_ERR_ALIAS if the input and output host ranges overlap. */
+int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, const void* Wqkv, const void* bqkv,
+                           const void* Wo, const void* bo, const void* W1, const void* b1, const void* W2,
+                           const void* b2, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
+                           float* out_host, long long out_stride, int n_inputs, void* stream);
+
 /* Allocation-free variant of bpt_layer_forward (bf16 inputs, same arguments
  * and result). The paper has no counterpart: this entry point exists for
  * callers that cannot call cudaMalloc (or any allocator) while they run, for

@@ -169,6 +169,27 @@ def test_ffn_width_entry_validates_and_sizes_its_workspace():
     assert L.bpt_layer_forward_ffn(0, *p, 1, 256, 256, 4, 512, 64, 64, 1, 0, ws + 16, need, out, None) == ALIGN
 
 
+def test_host_entry_validates_before_touching_memory():
+    L = bpt.lib()
+    w = fake_ptrs(8)  # device weights (never dereferenced: every case fails validation first)
+    xh, oh = BASE + 40 * STEP, BASE + 50 * STEP
+    shp = [1, 256, 256, 4, 64, 64, 1]
+    xb, ob = 256 * 256 * 2, 256 * 256 * 4
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, oh, ob, 0, None) == OK  # nothing to do
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, oh, ob, -1, None) == SHAPE
+    assert L.bpt_layer_forward_host(0, None, xb, *w, *shp, oh, ob, 2, None) == NULL
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, None, ob, 2, None) == NULL
+    assert L.bpt_layer_forward_host(0, xh, xb, *w[:7], None, *shp, oh, ob, 2, None) == NULL
+    assert L.bpt_layer_forward_host(0, xh, xb, *w[:7], w[7] + 8, *shp, oh, ob, 2, None) == ALIGN
+    assert L.bpt_layer_forward_host(0, xh, xb - 2, *w, *shp, oh, ob, 2, None) == SHAPE  # stride below one input
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, oh, ob - 4, 2, None) == SHAPE
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, xh + xb, ob, 2, None) == ALIAS  # out inside the inputs
+    assert L.bpt_layer_forward_host(0, xh, 0, *w, *shp, xh, 0, 3, None) == ALIAS
+    assert L.bpt_layer_forward_host(5, xh, xb, *w, *shp, oh, ob, 2, None) == DTYPE
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, 1, 256, 256, 3, 64, 64, 1, oh, ob, 2, None) == SHAPE
+    assert L.bpt_layer_forward_host(0, xh, xb, *w, 1, 256, 256, 4, 48, 64, 1, oh, ob, 2, None) == BLOCK
+
+
 def test_stage_entry_points_validate():
     L = bpt.lib()
     p = fake_ptrs(6)

@@ -191,6 +191,31 @@ def test_layer_any_ffn_width_matches_oracle(shape, workspace):
     assert_parity(got, oracle_full(shape, inp), f"ffn {shape.f}: {shape}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_host_entry_equals_the_device_path(dtype):
+    # three different inputs through bpt_layer_forward_host (pinned host
+    # memory, copies overlapped with compute) give, bit for bit, what the
+    # device entry gives for each; stride 0 repeats one input
+    shape = bi.LayerShape(1, 320, 256, 4, 64, 64, True, dtype)
+    inps = [bi.make_inputs(shape, seed=s) for s in (11, 12, 13)]
+    params = device_params(inps[0])
+    xs = [bi.to_torch(i["x"], device="cpu") for i in inps]
+    x_host = torch.stack(xs).pin_memory()
+    got = bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal)
+    assert bpt.device_status() == 0
+    for k in range(3):
+        ref = bpt.layer_forward(xs[k].cuda(), params, shape.heads, shape.q_block, shape.kv_block, shape.causal)
+        torch.cuda.synchronize()
+        assert torch.equal(got[k], ref.cpu()), f"input {k}"
+    one = bpt.layer_forward_host(xs[1].pin_memory(), params, shape.heads, shape.q_block, shape.kv_block,
+                                 shape.causal, n_inputs=4)
+    assert torch.equal(one, got[1])
+    # and for bf16 the result is the oracle's layer (the fp32 entry's own
+    # accuracy is checked by the fp32 workload and FFN-width tests)
+    if dtype == "bf16":
+        assert_parity(got[0].numpy(), oracle_full(shape, inps[0]), "host entry bf16")
+
+
 @pytest.mark.parametrize("wave_rows", [64, 128, 384, 100000])
 def test_layer_result_does_not_depend_on_the_wave(wave_rows):
     shape = bi.LayerShape(2, 768, 256, 2, 64, 128, True)

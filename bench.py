@@ -418,6 +418,96 @@ def our_arm(args, shape, name):
     return 0
 
 
+def max_context_arm(args):
+    """The longest single sequence one 7B-class BPT layer forward (h 4096, 32
+    heads, causal, q_block 1024, kv_block 2048) fits on this GPU, measured by
+    running it: the budget is the free device memory minus the weights and a
+    margin, the need per length is x (bf16) + out (fp32) + the library's exact
+    workspace. Inputs are seeded synthetic tensors drawn on the device; the
+    first rows are checked against the oracle (a causal row depends only on
+    its prefix)."""
+    import torch
+    import blockwise_attn_ffn_bpt_b200 as bpt
+    import oracle
+
+    h, heads, qb, kvb = 4096, 32, 1024, 2048
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    g = torch.Generator(device=device).manual_seed(0)
+    std = {"Wqkv": 1 / math.sqrt(h), "Wo": 1 / math.sqrt(h), "W1": 1 / math.sqrt(h), "W2": 1 / math.sqrt(4 * h)}
+    shapes = {"Wqkv": (h, 3 * h), "bqkv": (3 * h,), "Wo": (h, h), "bo": (h,), "W1": (h, 4 * h), "b1": (4 * h,),
+              "W2": (4 * h, h), "b2": (h,)}
+    params = {k: (torch.randn(shp, generator=g, device=device) * std.get(k, 0.02)).to(torch.bfloat16)
+              for k, shp in shapes.items()}
+    # load the kernels and the library's pool on a short prefix first
+    warm = torch.randn((1, 8192, h), generator=g, device=device).to(torch.bfloat16)
+    bpt.layer_forward(warm, params, heads, qb, kvb, True)
+    del warm
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    free, total = torch.cuda.mem_get_info(device)
+    margin = 3 << 30  # input generation chunks, the library's own allocations, fragmentation
+
+    def need(s):
+        return s * h * 2 + s * h * 4 + bpt.workspace_bytes(0, 1, s, h, heads, qb, kvb)
+
+    lo, hi = 1, (free - margin) // (10 * h * kvb) + 2
+    while need(hi * kvb) <= free - margin:
+        hi *= 2
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if need(mid * kvb) <= free - margin else (lo, mid)
+    s = lo * kvb
+    x = torch.empty((1, s, h), dtype=torch.bfloat16, device=device)
+    chunk = 1 << 16
+    for r0 in range(0, s, chunk):
+        r1 = min(s, r0 + chunk)
+        x[0, r0:r1] = torch.randn((r1 - r0, h), generator=g, device=device).to(torch.bfloat16)
+    out = torch.empty((1, s, h), dtype=torch.float32, device=device)
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    free_before, _ = torch.cuda.mem_get_info(device)
+    stream = torch.cuda.current_stream(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0 if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                      int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[0])) as clocks:
+        ev0.record(stream)
+        bpt.layer_forward(x, params, heads, qb, kvb, True, out=out, stream=stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+    ms = ev0.elapsed_time(ev1)
+    free_after, _ = torch.cuda.mem_get_info(device)
+    status = bpt.device_status()
+    # oracle check of the first rows, and finiteness of rows spread over the sequence
+    R = 256
+    p64 = {k: v.float().cpu().numpy().astype(np.float64) for k, v in params.items()}
+    x0 = x[0, :R].float().cpu().numpy().astype(np.float64)[None]
+    ref = oracle.layer_rows(x0, *(p64[k] for k in bi.PARAM_NAMES), heads=heads, causal=True, rows=np.arange(R))
+    got = out[0, :R].cpu().numpy().astype(np.float64)
+    d = got - ref
+    spread = torch.linspace(0, s - 1, 64, device=device).long()
+    finite = bool(torch.isfinite(out[0, spread]).all().item())
+    shape = bi.LayerShape(1, s, h, heads, qb, kvb, True)
+    flops = sum(layer_flops(shape).values())
+    ws = bpt.workspace_bytes(0, 1, s, h, heads, qb, kvb)
+    line = {
+        "metric": "longest single sequence of one 7B-class BPT layer forward on one GPU",
+        "value": s, "unit": "tokens", "n_gpus": 1, "dtype": "bf16", "data": "synthetic (seeded on the device)",
+        "config": {"workload": "max_context_h4096", "d_model": h, "heads": heads, "q_block": qb, "kv_block": kvb,
+                   "causal": True, "ffn_hidden": 4 * h},
+        "ms": ms, "tokens_per_s": s / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12,
+        "memory": {"device_total_bytes": total, "free_before_bytes": free_before, "free_after_bytes": free_after,
+                   "x_bytes": s * h * 2, "out_bytes": s * h * 4, "workspace_bytes": ws,
+                   "workspace_vs_2bsh_elements": ws / (2 * s * h * 2)},
+        "parity_first_rows": {"rows": R, "max_abs": float(np.abs(d).max()),
+                              "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(ref))},
+        "finite_at_64_spread_rows": finite, "device_status": status,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line))
+    return 0 if (status == 0 and finite) else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -428,7 +518,11 @@ def main(argv=None):
                     help="one of: " + ", ".join(list(bi.WORKLOADS) + ["sweep_<block>_<causal|noncausal>"]))
     ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-context", action="store_true",
+                    help="instead: the longest sequence one 7B-class layer forward fits on the GPU, run once")
     args = ap.parse_args(argv)
+    if args.max_context:
+        return max_context_arm(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     name = args.workload

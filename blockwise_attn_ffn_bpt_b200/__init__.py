@@ -23,7 +23,7 @@ BPT_DTYPE_F32 = 1
 EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
     "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
-    "bpt_layer_forward_host",
+    "bpt_layer_forward_host", "bpt_convert_f32_to_bf16",
     "bpt_qkv_projection", "bpt_attention", "bpt_device_status", "bpt_launch_count", "bpt_set_kernel_timing",
     "bpt_kernel_times",
 )
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
     L.bpt_layer_forward_ffn.restype = i
     L.bpt_layer_forward_ffn.argtypes = [i] + [vp] * 9 + [i] * 9 + [vp, sz, vp, vp]
     ll = ctypes.c_longlong
+    L.bpt_convert_f32_to_bf16.restype = i
+    L.bpt_convert_f32_to_bf16.argtypes = [vp, vp, ll, vp]
     L.bpt_layer_forward_host.restype = i
     L.bpt_layer_forward_host.argtypes = [i, vp, ll] + [vp] * 8 + [i] * 7 + [vp, ll, i, vp]
     L.bpt_qkv_projection.restype = i
@@ -217,6 +219,34 @@ def layer_forward_from_host(x_host: torch.Tensor, params: dict, heads: int, q_bl
                             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """One input [b, s, h] from host memory to a host fp32 result (see layer_forward_host)."""
     return layer_forward_host(x_host, params, heads, q_block, kv_block, causal, out_host=out_host, stream=stream)
+
+
+def convert_f32_to_bf16(src: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """src (fp32, CUDA) rounded to bf16 by the library's kernel."""
+    if src.dtype != torch.float32 or not src.is_cuda:
+        raise TypeError("src must be a CUDA fp32 tensor")
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    if out.dtype != torch.bfloat16 or out.numel() != src.numel():
+        raise ValueError("out must be a bf16 tensor with as many elements as src")
+    _check(lib().bpt_convert_f32_to_bf16(_ptr(src), _ptr(out), src.numel(), _stream(stream)),
+           "bpt_convert_f32_to_bf16")
+    return out
+
+
+def stack_forward(x: torch.Tensor, layers: list, heads: int, q_block: int, kv_block: int, causal: bool,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """A stack of BPT layers: x (bf16 [b, s, h], CUDA) through each parameter
+    dict of `layers` in turn; between layers the fp32 output is rounded to
+    bf16 on the device. Returns the last layer's fp32 output."""
+    out = None
+    cur = x
+    for i, params in enumerate(layers):
+        out = layer_forward(cur, params, heads, q_block, kv_block, causal, stream=stream)
+        if i + 1 < len(layers):
+            cur = convert_f32_to_bf16(out, stream=stream).view(x.shape)
+    return out
 
 
 def qkv_projection(x: torch.Tensor, Wqkv: torch.Tensor, bqkv: torch.Tensor,

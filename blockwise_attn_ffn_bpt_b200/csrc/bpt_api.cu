@@ -809,6 +809,17 @@ int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, co
                     n_inputs, stream);
 }
 
+int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stream) {
+  if (n < 0) return BPT_ERR_SHAPE;
+  if (n == 0) return BPT_OK;
+  if (!src || !dst) return BPT_ERR_NULL;
+  if (!aligned16(src) || !aligned16(dst)) return BPT_ERR_ALIGN;
+  if (overlap(rng(src, (size_t)n * 4), rng(dst, (size_t)n * 2))) return BPT_ERR_ALIAS;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  return launch_convert(src, dst, n, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,
                        void* v, void* stream) {
   if (b < 0 || s < 0 || h <= 0 || h % 64 || (long long)b * s > 0x7fffffffLL) return BPT_ERR_SHAPE;

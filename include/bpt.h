@@ -163,6 +163,13 @@ int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, co
                            const void* b2, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
                            float* out_host, long long out_stride, int n_inputs, void* stream);
 
+/* dst[i] = src[i] rounded to bf16 (nearest, ties to even), i < n; device
+ * pointers, 16-byte aligned, not overlapping; asynchronous on `stream`.
+ * Chains layers: one layer's fp32 out becomes the next layer's bf16 x (a
+ * stack of BPT layers, as the pages' models are). Errors: BPT_ERR_SHAPE for
+ * n < 0, BPT_ERR_NULL, BPT_ERR_ALIGN, BPT_ERR_ALIAS; nothing launched then. */
+int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stream);
+
 /* Allocation-free variant of bpt_layer_forward (bf16 inputs, same arguments
  * and result). The paper has no counterpart: this entry point exists for
  * callers that cannot call cudaMalloc (or any allocator) while they run, for

@@ -190,6 +190,18 @@ def test_host_entry_validates_before_touching_memory():
     assert L.bpt_layer_forward_host(0, xh, xb, *w, 1, 256, 256, 4, 48, 64, 1, oh, ob, 2, None) == BLOCK
 
 
+def test_convert_entry_validates():
+    L = bpt.lib()
+    a, b = BASE, BASE + STEP
+    assert L.bpt_convert_f32_to_bf16(a, b, 0, None) == OK
+    assert L.bpt_convert_f32_to_bf16(a, b, -1, None) == SHAPE
+    assert L.bpt_convert_f32_to_bf16(None, b, 8, None) == NULL
+    assert L.bpt_convert_f32_to_bf16(a, None, 8, None) == NULL
+    assert L.bpt_convert_f32_to_bf16(a + 4, b, 8, None) == ALIGN
+    assert L.bpt_convert_f32_to_bf16(a, b + 8, 8, None) == ALIGN
+    assert L.bpt_convert_f32_to_bf16(a, a + 16, 8, None) == ALIAS
+
+
 def test_stage_entry_points_validate():
     L = bpt.lib()
     p = fake_ptrs(6)

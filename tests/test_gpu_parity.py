@@ -216,6 +216,45 @@ def test_host_entry_equals_the_device_path(dtype):
         assert_parity(got[0].numpy(), oracle_full(shape, inps[0]), "host entry bf16")
 
 
+def test_convert_rounds_to_nearest_even_like_torch():
+    g = torch.Generator(device="cuda").manual_seed(7)
+    src = torch.randn(1 << 20 | 3, generator=g, device="cuda") * 100.0
+    src[:4] = torch.tensor([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -0.0, 3.0e38], device="cuda")  # ties, sign, range
+    got = bpt.convert_f32_to_bf16(src)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), src.to(torch.bfloat16).view(torch.int16))
+
+
+def test_two_layer_stack_matches_the_oracle_applied_twice():
+    # layer 2 reads layer 1's fp32 output rounded to bf16
+    s1 = bi.LayerShape(1, 256, 256, 4, 64, 128, True)
+    p1, p2 = bi.make_inputs(s1, seed=21), bi.make_inputs(s1, seed=22)
+    d1, d2 = device_params(p1), device_params(p2)
+    x = bi.to_torch(p1["x"])
+    got = bpt.stack_forward(x, [d1, d2], s1.heads, s1.q_block, s1.kv_block, s1.causal)
+    # the stack is the composition of the library's calls, bit for bit
+    y1 = bpt.layer_forward(x, d1, s1.heads, s1.q_block, s1.kv_block, s1.causal)
+    x2 = bpt.convert_f32_to_bf16(y1).view(x.shape)
+    y2 = bpt.layer_forward(x2, d2, s1.heads, s1.q_block, s1.kv_block, s1.causal)
+    torch.cuda.synchronize()
+    assert bpt.device_status() == 0
+    assert torch.equal(got, y2)
+    # layer 2 on that bf16 input is the oracle's layer (the usual bound)
+    x2_64 = x2.float().cpu().numpy().astype(np.float64)
+    ref2 = oracle.layer_forward(x2_64, *bi.oracle_args(p2)[1:], heads=s1.heads, causal=s1.causal)
+    assert_parity(got.cpu().numpy(), ref2, "stack, layer 2 on the GPU's bf16 intermediate")
+    # against the oracle applied twice (its own intermediate rounded to bf16):
+    # where the two layer-1 results straddle a bf16 rounding boundary the
+    # intermediates differ by one bf16 ulp (up to 2^-8 |x|, ~0.03 at |x| ~ 8),
+    # so elementwise max-abs is not a stable measure here; rel-L2 is
+    r1 = oracle.layer_forward(*bi.oracle_args(p1), heads=s1.heads, causal=s1.causal)
+    r2 = oracle.layer_forward(bi.to_f64(bi.f32_to_bf16_bits(r1.astype(np.float32))), *bi.oracle_args(p2)[1:],
+                              heads=s1.heads, causal=s1.causal)
+    mx, rl2 = errors(got.cpu().numpy(), r2)
+    log_errors("two-layer stack vs oracle twice", mx, rl2)
+    assert rl2 <= REL_L2, f"rel-L2 {rl2:.3e}"
+
+
 @pytest.mark.parametrize("wave_rows", [64, 128, 384, 100000])
 def test_layer_result_does_not_depend_on_the_wave(wave_rows):
     shape = bi.LayerShape(2, 768, 256, 2, 64, 128, True)

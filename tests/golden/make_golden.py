@@ -11,7 +11,6 @@ Run from the repository root:  python tests/golden/make_golden.py
 import os
 import sys
 
-import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 sys.path.insert(0, ROOT)

@@ -2,7 +2,6 @@
 include/bpt.h declares, and rejects bad arguments synchronously (argument
 checks run before any CUDA call, so these run on a CPU-only machine)."""
 
-import ctypes
 import os
 import re
 

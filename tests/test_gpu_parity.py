@@ -9,7 +9,6 @@ checked for equality.
 """
 
 import json
-import math
 import os
 
 import numpy as np

@@ -605,26 +605,42 @@ int static_workspace(void** ptr) {
 // n independent inputs from host memory: input i is copied in while input
 // i - 1 computes, and its result is copied out while input i + 1 computes.
 // Two device buffers each for x and out plus one workspace come from the
-// library's pool; two non-blocking copy streams are ordered against the
-// compute stream with events; every copy is one cudaMemcpyAsync.
+// library's pool; non-blocking copy streams are ordered against the compute
+// stream with events; every copy is one cudaMemcpyAsync. Each result goes
+// out in two halves on two streams, so that two copy engines share it.
 struct HostPipe {
-  cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t ready = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+  static constexpr int kOut = 2;  // device-to-host streams
+  cudaStream_t h2d = nullptr, d2h[kOut] = {};
+  cudaEvent_t ready = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2][kOut] = {};
   bool create() {
     if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
-    if (cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
-    cudaEvent_t* all[7] = {&ready, &h2d_done[0], &h2d_done[1], &comp_done[0], &comp_done[1], &d2h_done[0],
-                           &d2h_done[1]};
+    for (cudaStream_t& s : d2h)
+      if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
+    cudaEvent_t* all[5] = {&ready, &h2d_done[0], &h2d_done[1], &comp_done[0], &comp_done[1]};
     for (cudaEvent_t* e : all)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    for (auto& row : d2h_done)
+      for (cudaEvent_t& e : row)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
     return true;
   }
+  bool sync_copies() {
+    bool ok = !h2d || cudaStreamSynchronize(h2d) == cudaSuccess;
+    for (cudaStream_t s : d2h)
+      if (s) ok = cudaStreamSynchronize(s) == cudaSuccess && ok;
+    return ok;
+  }
   void destroy() {
-    if (h2d) cudaStreamSynchronize(h2d), cudaStreamDestroy(h2d);
-    if (d2h) cudaStreamSynchronize(d2h), cudaStreamDestroy(d2h);
-    cudaEvent_t all[7] = {ready, h2d_done[0], h2d_done[1], comp_done[0], comp_done[1], d2h_done[0], d2h_done[1]};
+    sync_copies();
+    if (h2d) cudaStreamDestroy(h2d);
+    for (cudaStream_t s : d2h)
+      if (s) cudaStreamDestroy(s);
+    cudaEvent_t all[5] = {ready, h2d_done[0], h2d_done[1], comp_done[0], comp_done[1]};
     for (cudaEvent_t e : all)
       if (e) cudaEventDestroy(e);
+    for (auto& row : d2h_done)
+      for (cudaEvent_t e : row)
+        if (e) cudaEventDestroy(e);
   }
 };
 
@@ -670,8 +686,8 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
   HostPipe pp;
   int r = pp.create() ? BPT_OK : BPT_ERR_CUDA;
   if (r == BPT_OK) {
-    bool cu = cudaEventRecord(pp.ready, st) == cudaSuccess && cudaStreamWaitEvent(pp.h2d, pp.ready, 0) == cudaSuccess &&
-              cudaStreamWaitEvent(pp.d2h, pp.ready, 0) == cudaSuccess;
+    bool cu = cudaEventRecord(pp.ready, st) == cudaSuccess && cudaStreamWaitEvent(pp.h2d, pp.ready, 0) == cudaSuccess;
+    for (int c = 0; c < HostPipe::kOut; ++c) cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.ready, 0) == cudaSuccess;
     for (int i = 0; cu && r == BPT_OK && i < n; ++i) {
       const int k = i & 1;
       const uint8_t* xi = reinterpret_cast<const uint8_t*>(x_host) + (size_t)x_stride * i;
@@ -682,24 +698,28 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
            cudaEventRecord(pp.h2d_done[k], pp.h2d) == cudaSuccess;
       // out buffer k is free once result i - 2 has been copied out
       cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k], 0) == cudaSuccess;
-      if (i >= 2) cu = cu && cudaStreamWaitEvent(st, pp.d2h_done[k], 0) == cudaSuccess;
+      for (int c = 0; i >= 2 && c < HostPipe::kOut; ++c)
+        cu = cu && cudaStreamWaitEvent(st, pp.d2h_done[k][c], 0) == cudaSuccess;
       if (!cu) break;
       LayerPtrs p = w;
       p.x = xdev[k];
       r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms);
       if (r != BPT_OK) break;
-      cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess &&
-           cudaStreamWaitEvent(pp.d2h, pp.comp_done[k], 0) == cudaSuccess &&
-           cudaMemcpyAsync(oi, odev[k], ob, cudaMemcpyDeviceToHost, pp.d2h) == cudaSuccess &&
-           cudaEventRecord(pp.d2h_done[k], pp.d2h) == cudaSuccess;
+      cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess;
+      // the two halves split at a row boundary
+      const size_t half = (tok / 2) * h * 4;
+      for (int c = 0; c < HostPipe::kOut; ++c) {
+        const size_t lo = c == 0 ? 0 : half, bytes = c == 0 ? half : ob - half;
+        cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.comp_done[k], 0) == cudaSuccess &&
+             (bytes == 0 || cudaMemcpyAsync(oi + lo, reinterpret_cast<uint8_t*>(odev[k]) + lo, bytes,
+                                            cudaMemcpyDeviceToHost, pp.d2h[c]) == cudaSuccess) &&
+             cudaEventRecord(pp.d2h_done[k][c], pp.d2h[c]) == cudaSuccess;
+      }
     }
     if (!cu && r == BPT_OK) r = BPT_ERR_CUDA;
   }
   // the buffers go back to the pool only after every copy has finished
-  if (pp.h2d && pp.d2h) {
-    if (cudaStreamSynchronize(pp.h2d) != cudaSuccess || cudaStreamSynchronize(pp.d2h) != cudaSuccess)
-      if (r == BPT_OK) r = BPT_ERR_CUDA;
-  }
+  if (!pp.sync_copies() && r == BPT_OK) r = BPT_ERR_CUDA;
   cudaFreeAsync(mem, st);
   if (cudaStreamSynchronize(st) != cudaSuccess && r == BPT_OK) r = BPT_ERR_CUDA;
   pp.destroy();

@@ -606,41 +606,50 @@ int static_workspace(void** ptr) {
 // i - 1 computes, and its result is copied out while input i + 1 computes.
 // Two device buffers each for x and out plus one workspace come from the
 // library's pool; non-blocking copy streams are ordered against the compute
-// stream with events; every copy is one cudaMemcpyAsync. Each result goes
-// out in two halves on two streams, so that two copy engines share it.
+// stream with events; every copy is one cudaMemcpyAsync. Each input comes
+// in, and each result goes out, in two halves on two streams, so that two
+// copy engines share every transfer.
 struct HostPipe {
-  static constexpr int kOut = 2;  // device-to-host streams
-  cudaStream_t h2d = nullptr, d2h[kOut] = {};
-  cudaEvent_t ready = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2][kOut] = {};
+  static constexpr int kCopy = 2;  // streams per direction
+  cudaStream_t h2d[kCopy] = {}, d2h[kCopy] = {};
+  cudaEvent_t ready = nullptr, comp_done[2] = {}, h2d_done[2][kCopy] = {}, d2h_done[2][kCopy] = {};
   bool create() {
-    if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
-    for (cudaStream_t& s : d2h)
-      if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
-    cudaEvent_t* all[5] = {&ready, &h2d_done[0], &h2d_done[1], &comp_done[0], &comp_done[1]};
+    for (int c = 0; c < kCopy; ++c)
+      if (cudaStreamCreateWithFlags(&h2d[c], cudaStreamNonBlocking) != cudaSuccess ||
+          cudaStreamCreateWithFlags(&d2h[c], cudaStreamNonBlocking) != cudaSuccess)
+        return false;
+    cudaEvent_t* all[3] = {&ready, &comp_done[0], &comp_done[1]};
     for (cudaEvent_t* e : all)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
-    for (auto& row : d2h_done)
-      for (cudaEvent_t& e : row)
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    for (int k = 0; k < 2; ++k)
+      for (int c = 0; c < kCopy; ++c)
+        if (cudaEventCreateWithFlags(&h2d_done[k][c], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&d2h_done[k][c], cudaEventDisableTiming) != cudaSuccess)
+          return false;
     return true;
   }
   bool sync_copies() {
-    bool ok = !h2d || cudaStreamSynchronize(h2d) == cudaSuccess;
-    for (cudaStream_t s : d2h)
-      if (s) ok = cudaStreamSynchronize(s) == cudaSuccess && ok;
+    bool ok = true;
+    for (int c = 0; c < kCopy; ++c) {
+      if (h2d[c]) ok = cudaStreamSynchronize(h2d[c]) == cudaSuccess && ok;
+      if (d2h[c]) ok = cudaStreamSynchronize(d2h[c]) == cudaSuccess && ok;
+    }
     return ok;
   }
   void destroy() {
     sync_copies();
-    if (h2d) cudaStreamDestroy(h2d);
-    for (cudaStream_t s : d2h)
-      if (s) cudaStreamDestroy(s);
-    cudaEvent_t all[5] = {ready, h2d_done[0], h2d_done[1], comp_done[0], comp_done[1]};
+    for (int c = 0; c < kCopy; ++c) {
+      if (h2d[c]) cudaStreamDestroy(h2d[c]);
+      if (d2h[c]) cudaStreamDestroy(d2h[c]);
+    }
+    cudaEvent_t all[3] = {ready, comp_done[0], comp_done[1]};
     for (cudaEvent_t e : all)
       if (e) cudaEventDestroy(e);
-    for (auto& row : d2h_done)
-      for (cudaEvent_t e : row)
-        if (e) cudaEventDestroy(e);
+    for (int k = 0; k < 2; ++k)
+      for (int c = 0; c < kCopy; ++c) {
+        if (h2d_done[k][c]) cudaEventDestroy(h2d_done[k][c]);
+        if (d2h_done[k][c]) cudaEventDestroy(d2h_done[k][c]);
+      }
   }
 };
 
@@ -686,19 +695,27 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
   HostPipe pp;
   int r = pp.create() ? BPT_OK : BPT_ERR_CUDA;
   if (r == BPT_OK) {
-    bool cu = cudaEventRecord(pp.ready, st) == cudaSuccess && cudaStreamWaitEvent(pp.h2d, pp.ready, 0) == cudaSuccess;
-    for (int c = 0; c < HostPipe::kOut; ++c) cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.ready, 0) == cudaSuccess;
+    bool cu = cudaEventRecord(pp.ready, st) == cudaSuccess;
+    for (int c = 0; c < HostPipe::kCopy; ++c)
+      cu = cu && cudaStreamWaitEvent(pp.h2d[c], pp.ready, 0) == cudaSuccess &&
+           cudaStreamWaitEvent(pp.d2h[c], pp.ready, 0) == cudaSuccess;
+    // transfers split at a row boundary: [0, half) and [half, end)
+    const size_t x_half = (tok / 2) * h * es, o_half = (tok / 2) * h * 4;
     for (int i = 0; cu && r == BPT_OK && i < n; ++i) {
       const int k = i & 1;
       const uint8_t* xi = reinterpret_cast<const uint8_t*>(x_host) + (size_t)x_stride * i;
       uint8_t* oi = reinterpret_cast<uint8_t*>(out_host) + (size_t)out_stride * i;
       // x buffer k is free once input i - 2 has been computed
-      if (i >= 2) cu = cu && cudaStreamWaitEvent(pp.h2d, pp.comp_done[k], 0) == cudaSuccess;
-      cu = cu && cudaMemcpyAsync(xdev[k], xi, xb, cudaMemcpyHostToDevice, pp.h2d) == cudaSuccess &&
-           cudaEventRecord(pp.h2d_done[k], pp.h2d) == cudaSuccess;
+      for (int c = 0; c < HostPipe::kCopy; ++c) {
+        const size_t lo = c == 0 ? 0 : x_half, bytes = c == 0 ? x_half : xb - x_half;
+        if (i >= 2) cu = cu && cudaStreamWaitEvent(pp.h2d[c], pp.comp_done[k], 0) == cudaSuccess;
+        cu = cu && (bytes == 0 || cudaMemcpyAsync(xdev[k] + lo, xi + lo, bytes, cudaMemcpyHostToDevice,
+                                                  pp.h2d[c]) == cudaSuccess) &&
+             cudaEventRecord(pp.h2d_done[k][c], pp.h2d[c]) == cudaSuccess;
+        cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k][c], 0) == cudaSuccess;
+      }
       // out buffer k is free once result i - 2 has been copied out
-      cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k], 0) == cudaSuccess;
-      for (int c = 0; i >= 2 && c < HostPipe::kOut; ++c)
+      for (int c = 0; i >= 2 && c < HostPipe::kCopy; ++c)
         cu = cu && cudaStreamWaitEvent(st, pp.d2h_done[k][c], 0) == cudaSuccess;
       if (!cu) break;
       LayerPtrs p = w;
@@ -706,10 +723,8 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
       r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms);
       if (r != BPT_OK) break;
       cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess;
-      // the two halves split at a row boundary
-      const size_t half = (tok / 2) * h * 4;
-      for (int c = 0; c < HostPipe::kOut; ++c) {
-        const size_t lo = c == 0 ? 0 : half, bytes = c == 0 ? half : ob - half;
+      for (int c = 0; c < HostPipe::kCopy; ++c) {
+        const size_t lo = c == 0 ? 0 : o_half, bytes = c == 0 ? o_half : ob - o_half;
         cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.comp_done[k], 0) == cudaSuccess &&
              (bytes == 0 || cudaMemcpyAsync(oi + lo, reinterpret_cast<uint8_t*>(odev[k]) + lo, bytes,
                                             cudaMemcpyDeviceToHost, pp.d2h[c]) == cudaSuccess) &&

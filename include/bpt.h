@@ -153,9 +153,9 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
  * copies to overlap the compute; pageable memory works, slower. Input i is
  * copied in while input i - 1 computes and its result copied out while input
  * i + 1 computes (two device buffers each for x and out and one workspace,
- * from the library's pool; three internal copy streams, one for the inputs
- * and two that each copy half of every result, ordered by events against
- * `stream`, which runs the layer). Returns after every result has
+ * from the library's pool; four internal copy streams, two each way, that
+ * move every input and every result in two halves, ordered by events
+ * against `stream`, which runs the layer). Returns after every result has
  * reached host memory. Errors as bpt_layer_forward; BPT_ERR_SHAPE also for
  * n_inputs < 0 or a nonzero stride smaller than one input (output); and
  * BPT_ERR_ALIAS if the input and output host ranges overlap. */

@@ -341,24 +341,30 @@ Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave
     return at;
   };
   if (dtype == BPT_DTYPE_F32) {
-    L.xb = take(tok * h * 2);
-    L.wqkv = take((size_t)h * 3 * h * 2);
-    L.wo = take((size_t)h * h * 2);
-    L.w1 = take((size_t)h * ffn * 2);
-    L.w2 = take((size_t)ffn * h * 2);
+    // split bf16 parts: x as rows [x_hi | x_lo]; Wqkv as [hi; lo; hi] and
+    // Wo, W1, W2 as [hi; lo], stacked along K
+    L.xb = take(tok * 2 * h * 2);
+    L.wqkv = take((size_t)3 * h * 3 * h * 2);
+    L.wo = take((size_t)2 * h * h * 2);
+    L.w1 = take((size_t)2 * h * ffn * 2);
+    L.w2 = take((size_t)2 * ffn * h * 2);
   }
   L.total = off;
   return L;
 }
 
 // ------------------------------------------------------------- launches
+// A [M, a_cols] (row stride lda) times B [K, N]; with a_split != 0 the K
+// blocks of B pair with A's blocks as a_block() maps them (split products).
 template <int MODE>
-int launch_gemm(const void* A, long long M, long long K, long long lda, const void* B, long long N,
-                GemmArgs args, int sms, cudaStream_t st, const char* name) {
+int launch_gemm_split(const void* A, long long M, long long a_cols, long long lda, const void* B, long long K,
+                      long long N, int a_split, int a_kb, GemmArgs args, int sms, cudaStream_t st, const char* name) {
   if (M <= 0) return BPT_OK;
   CUtensorMap ta, tb;
-  if (!map_rows(&ta, A, M, K, lda, GEMM_BM)) return BPT_ERR_CUDA;
+  if (!map_rows(&ta, A, M, a_cols, lda, GEMM_BM)) return BPT_ERR_CUDA;
   if (!map_rows(&tb, B, K, N, N, 64)) return BPT_ERR_CUDA;
+  args.a_split = a_split;
+  args.a_kb = a_kb;
   args.M = (int)M;
   args.N = (int)N;
   args.K = (int)K;
@@ -371,6 +377,12 @@ int launch_gemm(const void* A, long long M, long long K, long long lda, const vo
     gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
   }
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+template <int MODE>
+int launch_gemm(const void* A, long long M, long long K, long long lda, const void* B, long long N,
+                GemmArgs args, int sms, cudaStream_t st, const char* name) {
+  return launch_gemm_split<MODE>(A, M, K, lda, B, K, N, 0, 0, args, sms, st, name);
 }
 
 // Attention of the query rows [t_start, t_start + t_len) of sequences
@@ -427,6 +439,53 @@ int launch_convert(const float* src, void* dst, long long n, int sms, cudaStream
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
+// The two bf16 parts of fp32 values: hi = bf16(v), lo = bf16(v - hi), so that
+// hi + lo carries v to about 16 significant bits. hi is also written to hi2
+// when it is given.
+__global__ void split_bf16_kernel(const float* __restrict__ src, long long n, __nv_bfloat16* hi,
+                                  __nv_bfloat16* lo, __nv_bfloat16* hi2) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = src[i];
+    const __nv_bfloat16 a = __float2bfloat16_rn(v);
+    const __nv_bfloat16 b = __float2bfloat16_rn(v - __bfloat162float(a));
+    hi[i] = a;
+    lo[i] = b;
+    if (hi2) hi2[i] = a;
+  }
+}
+
+// Rows of x as [x_hi | x_lo]: dst row r = hi parts of src row r, then lo parts.
+__global__ void split_rows_bf16_kernel(const float* __restrict__ src, long long rows, int cols,
+                                       __nv_bfloat16* dst) {
+  const long long n = rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols, c = i - r * cols;
+    const float v = src[i];
+    const __nv_bfloat16 a = __float2bfloat16_rn(v);
+    dst[r * 2 * cols + c] = a;
+    dst[r * 2 * cols + cols + c] = __float2bfloat16_rn(v - __bfloat162float(a));
+  }
+}
+
+int launch_split(const float* src, long long n, void* hi, void* lo, void* hi2, int sms, cudaStream_t st) {
+  if (n <= 0) return BPT_OK;
+  const long long blocks = std::min<long long>((n + 255) / 256, (long long)sms * 8);
+  LaunchScope ls("split_bf16", st);
+  split_bf16_kernel<<<(int)blocks, 256, 0, st>>>(src, n, reinterpret_cast<__nv_bfloat16*>(hi),
+                                                 reinterpret_cast<__nv_bfloat16*>(lo),
+                                                 reinterpret_cast<__nv_bfloat16*>(hi2));
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+int launch_split_rows(const float* src, long long rows, int cols, void* dst, int sms, cudaStream_t st) {
+  const long long n = rows * cols;
+  if (n <= 0) return BPT_OK;
+  const long long blocks = std::min<long long>((n + 255) / 256, (long long)sms * 8);
+  LaunchScope ls("split_bf16", st);
+  split_rows_bf16_kernel<<<(int)blocks, 256, 0, st>>>(src, rows, cols, reinterpret_cast<__nv_bfloat16*>(dst));
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
 #define BPT_TRY(expr)            \
   do {                           \
     int _r = (expr);             \
@@ -480,11 +539,18 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   const void *xa = p.x, *wqkv = p.Wqkv, *wo = p.Wo, *w1 = p.W1, *w2 = p.W2;
   const int f32 = dtype == BPT_DTYPE_F32 ? 1 : 0;
   if (f32) {
-    BPT_TRY(launch_convert((const float*)p.x, ws + L.xb, tok * h, sms, st));
-    BPT_TRY(launch_convert((const float*)p.Wqkv, ws + L.wqkv, 3LL * h * h, sms, st));
-    BPT_TRY(launch_convert((const float*)p.Wo, ws + L.wo, 1LL * h * h, sms, st));
-    BPT_TRY(launch_convert((const float*)p.W1, ws + L.w1, (long long)h * ffn, sms, st));
-    BPT_TRY(launch_convert((const float*)p.W2, ws + L.w2, (long long)ffn * h, sms, st));
+    // fp32 inputs: split bf16 products, so that neither x nor the weights
+    // lose more than about 16 significant bits (x W = x_hi W_hi + x_hi W_lo +
+    // x_lo W_hi for the projection; a W_hi + a W_lo for the other GEMMs,
+    // whose A is a bf16 activation of the path)
+    const long long q3 = 3LL * h * h;
+    BPT_TRY(launch_split_rows((const float*)p.x, tok, h, ws + L.xb, sms, st));
+    BPT_TRY(launch_split((const float*)p.Wqkv, q3, ws + L.wqkv, ws + L.wqkv + q3 * 2, ws + L.wqkv + q3 * 4, sms, st));
+    BPT_TRY(launch_split((const float*)p.Wo, 1LL * h * h, ws + L.wo, ws + L.wo + 2LL * h * h, nullptr, sms, st));
+    BPT_TRY(launch_split((const float*)p.W1, (long long)h * ffn, ws + L.w1, ws + L.w1 + 2LL * h * ffn, nullptr, sms,
+                         st));
+    BPT_TRY(launch_split((const float*)p.W2, (long long)ffn * h, ws + L.w2, ws + L.w2 + 2LL * ffn * h, nullptr, sms,
+                         st));
     xa = ws + L.xb;
     wqkv = ws + L.wqkv;
     wo = ws + L.wo;
@@ -503,7 +569,11 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.v = V;
     a.ldkv = h;
     a.h = h;
-    BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, "gemm_qkv"));
+    if (f32)
+      BPT_TRY(launch_gemm_split<EPI_QKV>(xa, tok, 2LL * h, 2LL * h, wqkv, 3LL * h, 3LL * h, 2, h / GEMM_BK, a, sms,
+                                         st, "gemm_qkv"));
+    else
+      BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, "gemm_qkv"));
   }
 
   // steps 4-10 for every query block at once: each CTA overwrites the Q of its
@@ -526,13 +596,17 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.bias = p.bo;
     a.dst = HB;
     a.ld_dst = h;
-    BPT_TRY(launch_gemm<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, h, a, sms, st, "gemm_outproj"));
+    const int sp = f32 ? 1 : 0, kf = f32 ? 2 : 1;  // fp32 inputs: A against [W_hi; W_lo]
+    BPT_TRY(launch_gemm_split<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, (long long)kf * h, h, sp,
+                                           h / GEMM_BK, a, sms, st, "gemm_outproj"));
     a.bias = p.b1;
     a.dst = U;
     a.ld_dst = ffn;
-    BPT_TRY(launch_gemm<EPI_FFN_UP>(HB, rows, h, h, w1, ffn, a, sms, st, "gemm_ffn_up"));
+    BPT_TRY(launch_gemm_split<EPI_FFN_UP>(HB, rows, h, h, w1, (long long)kf * h, ffn, sp, h / GEMM_BK, a, sms, st,
+                                          "gemm_ffn_up"));
     a.bias = p.b2;
-    BPT_TRY(launch_gemm<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, h, a, sms, st, "gemm_ffn_down"));
+    BPT_TRY(launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
+                                            st, "gemm_ffn_down"));
   }
   return BPT_OK;
 }

@@ -60,7 +60,20 @@ struct GemmArgs {
   // bf16 destination of OUTPROJ (hid copy) and FFN_UP (U)
   __nv_bfloat16* dst;
   long long ld_dst;
+  // Split products (fp32 inputs): B stacks bf16 parts of the weights along K
+  // and A is read again for each part. a_split 0: A's K block = kb; 1: kb
+  // modulo a_kb (A against [W_hi; W_lo]); 2: kb modulo a_kb for the first
+  // 2 a_kb blocks, then kb - a_kb (A = [x_hi | x_lo] against [W_hi; W_lo; W_hi]).
+  int a_split;
+  int a_kb;  // K blocks of one copy of A
 };
+
+// K block of A that pairs with K block kb of B
+__device__ __forceinline__ int a_block(const GemmArgs& a, int kb) {
+  if (a.a_split == 0) return kb;
+  if (a.a_split == 1 || kb < 2 * a.a_kb) return kb % a.a_kb;
+  return kb - a.a_kb;
+}
 
 __device__ __forceinline__ float load_vec_elem(const void* p, int f32, long long i) {
   return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
@@ -212,7 +225,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa = smem_base + stage * GEMM_STAGE_BYTES;
           mbar_arrive_expect_tx(fb, GEMM_STAGE_BYTES);
-          tma_load_2d(sa, &tmA, fb, kb * GEMM_BK, m0);
+          tma_load_2d(sa, &tmA, fb, a_block(args, kb) * GEMM_BK, m0);
 #pragma unroll
           for (int j = 0; j < GEMM_BN / 64; ++j)
             tma_load_2d(sa + GEMM_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);

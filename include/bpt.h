@@ -99,7 +99,11 @@ int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const v
                       const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                       int heads, int q_block, int kv_block, int causal, float* out, void* stream);
 
-/* fp32 inputs (same arguments, fp32 tensors). */
+/* fp32 inputs (same arguments, fp32 tensors). The GEMMs keep about 16
+ * significant bits of x and of the weights: each fp32 value v is split on the
+ * device into bf16 parts hi = bf16(v) and lo = bf16(v - hi), and the products
+ * x W_hi + x W_lo (projection: x_hi W_hi + x_hi W_lo + x_lo W_hi) accumulate in
+ * fp32. Attention and the FFN activations are bf16 as in the bf16 entry. */
 int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, const float* Wo, const float* bo,
                           const float* W1, const float* b1, const float* W2, const float* b2, int b, int s, int h,
                           int heads, int q_block, int kv_block, int causal, float* out, void* stream);

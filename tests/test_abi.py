@@ -127,11 +127,13 @@ def test_workspace_bytes_follow_the_layout():
     assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128, 2048) == expect(2, 2048, 1024, 2048)
     assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == expect(1, 16384, 2048, 2048)
     assert bpt.workspace_bytes(0, 1, 8192, 2048, 16, 512, 512) == expect(1, 8192, 2048, 4096)
-    # fp32 inputs add bf16 copies of x and the weights
+    # fp32 inputs add their bf16 parts: x as [x_hi | x_lo] rows, Wqkv as
+    # [hi; lo; hi], Wo, W1 and W2 as [hi; lo]
     f = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
     g = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)
     assert g == expect(1, 256, 256, 256)
-    assert f == g + up(256 * 256 * 2) + up(3 * 256 * 256 * 2) + up(256 * 256 * 2) + 2 * up(4 * 256 * 256 * 2)
+    assert f == g + up(256 * 512 * 2) + up(768 * 768 * 2) + up(512 * 256 * 2) + up(512 * 1024 * 2) + \
+        up(2048 * 256 * 2)
     assert bpt.workspace_bytes(0, 1, 256, 256, 3, 64, 64) == 0
     assert bpt.workspace_bytes(0, 0, 256, 256, 4, 64, 64) == 0
 
@@ -157,10 +159,11 @@ def test_ffn_width_entry_validates_and_sizes_its_workspace():
         max(2 * up(2048 * 1024 * 2), up(512 * 1024 * 4) + up(512 * 1024 * 2) + up(512 * 192 * 2))
     assert bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 256, ffn=4096) == \
         max(2 * up(256 * 256 * 2), up(256 * 256 * 4) + up(256 * 256 * 2) + up(256 * 4096 * 2))
-    # fp32 inputs add bf16 copies of W1 [h, f] and W2 [f, h]
+    # fp32 inputs add the bf16 parts, W1 [h, f] and W2 [f, h] as [hi; lo]
     f32 = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64, 256, ffn=640)
     b16 = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 256, ffn=640)
-    assert f32 == b16 + up(256 * 256 * 2) + up(3 * 256 * 256 * 2) + up(256 * 256 * 2) + 2 * up(256 * 640 * 2)
+    assert f32 == b16 + up(256 * 512 * 2) + up(768 * 768 * 2) + up(512 * 256 * 2) + up(512 * 640 * 2) + \
+        up(1280 * 256 * 2)
     # a too-small caller workspace and a misaligned one are refused
     need = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64, 0, ffn=512)
     ws = BASE + 30 * STEP

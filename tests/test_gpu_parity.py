@@ -209,10 +209,8 @@ def test_host_entry_equals_the_device_path(dtype):
     one = bpt.layer_forward_host(xs[1].pin_memory(), params, shape.heads, shape.q_block, shape.kv_block,
                                  shape.causal, n_inputs=4)
     assert torch.equal(one, got[1])
-    # and for bf16 the result is the oracle's layer (the fp32 entry's own
-    # accuracy is checked by the fp32 workload and FFN-width tests)
-    if dtype == "bf16":
-        assert_parity(got[0].numpy(), oracle_full(shape, inps[0]), "host entry bf16")
+    # and the result is the oracle's layer
+    assert_parity(got[0].numpy(), oracle_full(shape, inps[0]), f"host entry {dtype}")
 
 
 def test_convert_rounds_to_nearest_even_like_torch():

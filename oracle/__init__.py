@@ -1,4 +1,4 @@
-"""fp64 CPU oracle of the BPT layer forward.
+"""fp64 CPU oracle of the BPT layer forward (and its gradients).
 
 TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
 benchmark's CPU-baseline leg use it to produce expected values. The library
@@ -13,4 +13,9 @@ from .bpt_oracle import (  # noqa: F401
     layer_rows,
     qkv_projection,
     residual_ffn,
+)
+from .bpt_oracle_backward import (  # noqa: F401
+    attention_backward,
+    attention_backward_blockwise,
+    layer_backward,
 )

@@ -1,0 +1,186 @@
+"""Plain fp64 CPU oracle for the gradients of one BPT layer.
+
+TEST INFRASTRUCTURE ONLY, like bpt_oracle: only the test suite may import or
+call this module; the library's product path never does, and this module
+imports nothing from it.
+
+The pages train their models with the blockwise layer ("Blockwise Parallel
+Transformer for Large Context Models" paper review, sections 4-5: language
+modelling and reinforcement learning runs, with the blockwise FFN scanned and
+rematerialised, section 3 "blockwise FFN" listing). What the backward pass
+computes is fixed by the forward: the gradients of the layer's output with
+respect to its input and every parameter. `layer_backward` writes that chain
+rule out for the forward of bpt_oracle:
+
+    qkv = x Wqkv + bqkv;  S = Q K^T / sqrt(dh) (masked);  P = softmax(S)
+    O = P V;  hid = x + O Wo + bo;  a = hid W1 + b1;  u = max(0, a)
+    y = hid + u W2 + b2
+
+and, given dy = dL/dy,
+
+    db2 = sum dy;  dW2 = u^T dy;  da = (dy W2^T) [a > 0]
+    db1 = sum da;  dW1 = hid^T da;  dhid = dy + da W1^T
+    dbo = sum dhid;  dWo = O^T dhid;  dO = dhid Wo^T
+    per head: dV = P^T dO;  dP = dO V^T;  dS = P (dP - rowsum(dP P))
+              dQ = dS K / sqrt(dh);  dK = dS^T Q / sqrt(dh)
+    dqkv = [dQ | dK | dV];  dbqkv = sum dqkv;  dWqkv = x^T dqkv
+    dx = dhid + dqkv Wqkv^T
+
+`attention_backward_blockwise` computes the attention part block by block,
+the way a blockwise layer trains without storing P: per query block and
+key/value block it recomputes P from the forward's row statistics (running
+max m and sum l, as Algorithm 1 records them) and accumulates dQ, dK and dV,
+using D = rowsum(dO O) in place of rowsum(dP P) (the two are equal). It is
+checked equal to the plain gradient for every block pair.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import bpt_oracle as ob
+
+
+def _softmax_grad(P: np.ndarray, dP: np.ndarray) -> np.ndarray:
+    """dS for dP through a row softmax P (the softmax Jacobian applied per row)."""
+    return P * (dP - np.sum(dP * P, axis=-1, keepdims=True))
+
+
+def _relu_grad(a: np.ndarray) -> np.ndarray:
+    return (a > 0).astype(a.dtype)
+
+
+def _value_grad(P: np.ndarray, dO: np.ndarray) -> np.ndarray:
+    """dV = P^T dO of one head."""
+    return np.swapaxes(P, -1, -2) @ dO
+
+
+def _qk_grads(dS: np.ndarray, Q: np.ndarray, K: np.ndarray, scale: float):
+    """dQ = dS K scale and dK = dS^T Q scale of one head."""
+    return (dS @ K) * scale, (np.swapaxes(dS, -1, -2) @ Q) * scale
+
+
+def _dhid(dy: np.ndarray, da: np.ndarray, W1: np.ndarray) -> np.ndarray:
+    """Gradient reaching hid: through the second residual and through the FFN."""
+    return dy + da @ W1.T
+
+
+def _attention_probs(Q, K, dh, causal):
+    """Row softmax of the scaled, masked scores of one head: P [.., s, s]."""
+    s = Q.shape[-2]
+    t = np.arange(s)
+    allowed = ob._key_allowed(t, t, causal)
+    S = (Q @ np.swapaxes(K, -1, -2)) * ob._softmax_scale(dh)
+    S = np.where(allowed, S, -np.inf)
+    S = S - S.max(axis=-1, keepdims=True)
+    E = np.where(allowed, np.exp(S), 0.0)
+    return E / E.sum(axis=-1, keepdims=True)
+
+
+def attention_backward(Q, K, V, dO, heads: int, causal: bool):
+    """dQ, dK, dV [b, s, h] of O = softmax(Q K^T / sqrt(dh)) V per head, by the plain definition."""
+    h = Q.shape[-1]
+    dh = h // heads
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for k in range(heads):
+        c = ob._head_cols(k, dh)
+        P = _attention_probs(Q[..., c], K[..., c], dh, causal)
+        dV[..., c] = _value_grad(P, dO[..., c])
+        dP = dO[..., c] @ np.swapaxes(V[..., c], -1, -2)
+        dS = _softmax_grad(P, dP)
+        dQ[..., c], dK[..., c] = _qk_grads(dS, Q[..., c], K[..., c], ob._softmax_scale(dh))
+    return dQ, dK, dV
+
+
+def attention_backward_blockwise(Q, K, V, dO, heads: int, causal: bool, q_block: int, kv_block: int):
+    """dQ, dK, dV [b, s, h] block by block from the forward's row statistics.
+
+    Forward statistics per query row (over all of its key/value blocks): the
+    max m of the scaled scores and the sum l of exp(score - m); O itself. Then
+    for each query block i and key/value block j: P_ij = exp(S_ij - m_i) / l_i
+    (0 where masked), dV_j += P_ij^T dO_i, dP_ij = dO_i V_j^T, dS_ij = P_ij
+    (dP_ij - D_i) with D_i = rowsum(dO_i O_i), dQ_i += dS_ij K_j scale,
+    dK_j += dS_ij^T Q_i scale.
+    """
+    b, s, h = Q.shape
+    if s % q_block or s % kv_block:
+        raise ValueError("s must be a multiple of both block sizes")
+    dh = h // heads
+    scale = ob._softmax_scale(dh)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    t = np.arange(s)
+    for k in range(heads):
+        c = ob._head_cols(k, dh)
+        q, kk, v, do = Q[..., c], K[..., c], V[..., c], dO[..., c]
+        # forward statistics, block by block over the keys
+        m = np.full((b, s), -np.inf)
+        for j0 in range(0, s, kv_block):
+            tj = t[j0:j0 + kv_block]
+            Sj = np.where(ob._key_allowed(t, tj, causal), (q @ np.swapaxes(kk[:, j0:j0 + kv_block], -1, -2)) * scale,
+                          -np.inf)
+            m = np.maximum(m, Sj.max(axis=-1))
+        l = np.zeros((b, s))
+        o = np.zeros_like(q)
+        for j0 in range(0, s, kv_block):
+            tj = t[j0:j0 + kv_block]
+            allowed = ob._key_allowed(t, tj, causal)
+            Sj = (q @ np.swapaxes(kk[:, j0:j0 + kv_block], -1, -2)) * scale
+            Ej = np.where(allowed, np.exp(np.where(allowed, Sj, 0.0) - m[..., None]), 0.0)
+            l += Ej.sum(axis=-1)
+            o += Ej @ v[:, j0:j0 + kv_block]
+        o /= l[..., None]
+        D = np.sum(do * o, axis=-1)
+        for i0 in range(0, s, q_block):
+            ti = t[i0:i0 + q_block]
+            qi, doi = q[:, i0:i0 + q_block], do[:, i0:i0 + q_block]
+            mi, li, Di = m[:, i0:i0 + q_block], l[:, i0:i0 + q_block], D[:, i0:i0 + q_block]
+            for j0 in range(0, s, kv_block):
+                tj = t[j0:j0 + kv_block]
+                allowed = ob._key_allowed(ti, tj, causal)
+                kj, vj = kk[:, j0:j0 + kv_block], v[:, j0:j0 + kv_block]
+                Sij = (qi @ np.swapaxes(kj, -1, -2)) * scale
+                Pij = np.where(allowed, np.exp(np.where(allowed, Sij, 0.0) - mi[..., None]), 0.0) / li[..., None]
+                dV[:, j0:j0 + kv_block, c] += np.swapaxes(Pij, -1, -2) @ doi
+                dPij = doi @ np.swapaxes(vj, -1, -2)
+                dSij = Pij * (dPij - Di[..., None])
+                dQ[:, i0:i0 + q_block, c] += (dSij @ kj) * scale
+                dK[:, j0:j0 + kv_block, c] += (np.swapaxes(dSij, -1, -2) @ qi) * scale
+    return dQ, dK, dV
+
+
+def layer_backward(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, heads: int, causal: bool,
+                   q_block: int | None = None, kv_block: int | None = None) -> dict:
+    """Gradients of the layer output y with respect to x and every parameter,
+    for the upstream gradient dy [b, s, h]; attention blockwise when both
+    block sizes are given. Returns a dict keyed like the arguments: dx, dWqkv,
+    dbqkv, dWo, dbo, dW1, db1, dW2, db2."""
+    h = x.shape[-1]
+    Q, K, V = ob.qkv_projection(x, Wqkv, bqkv)
+    O = ob.attention(Q, K, V, heads, causal, threads=1)
+    hid = x + O @ Wo + bo
+    a = hid @ W1 + b1
+    u = ob._relu(a)
+
+    def flat(z):
+        return z.reshape(-1, z.shape[-1])
+
+    g = {}
+    g["db2"] = flat(dy).sum(axis=0)
+    g["dW2"] = flat(u).T @ flat(dy)
+    da = (dy @ W2.T) * _relu_grad(a)
+    g["db1"] = flat(da).sum(axis=0)
+    g["dW1"] = flat(hid).T @ flat(da)
+    dhid = _dhid(dy, da, W1)
+    g["dbo"] = flat(dhid).sum(axis=0)
+    g["dWo"] = flat(O).T @ flat(dhid)
+    dO = dhid @ Wo.T
+    if q_block is not None and kv_block is not None:
+        dQ, dK, dV = attention_backward_blockwise(Q, K, V, dO, heads, causal, q_block, kv_block)
+    else:
+        dQ, dK, dV = attention_backward(Q, K, V, dO, heads, causal)
+    dqkv = np.concatenate([dQ, dK, dV], axis=-1)
+    g["dbqkv"] = flat(dqkv).sum(axis=0)
+    g["dWqkv"] = flat(x).T @ flat(dqkv)
+    g["dx"] = dhid + dqkv @ Wqkv.T
+    assert g["dx"].shape == x.shape and h == x.shape[-1]
+    return g

@@ -1,0 +1,118 @@
+"""Pins of the backward oracle (oracle/bpt_oracle_backward.py) against things
+other than itself: central differences of the forward oracle, torch fp64
+autograd of a forward written here with torch's own attention, a conservation
+law of the value gradient, and the blockwise gradient equal to the plain one
+for every block pair."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import bpt_oracle_backward as obb
+from tests.test_oracle_pins import divisors, rand_layer
+
+NAMES = ("x", "Wqkv", "bqkv", "Wo", "bo", "W1", "b1", "W2", "b2")
+
+
+def grads(p, dy, heads, causal, **kw):
+    return obb.layer_backward(*(p[k] for k in NAMES), dy, heads=heads, causal=causal, **kw)
+
+
+def loss(p, dy, heads, causal):
+    y = oracle.layer_forward(*(p[k] for k in NAMES), heads=heads, causal=causal, threads=1)
+    return float(np.sum(y * dy))
+
+
+def pre_activations(p, heads, causal):
+    q, k, v = oracle.qkv_projection(p["x"], p["Wqkv"], p["bqkv"])
+    o = oracle.attention(q, k, v, heads, causal, threads=1)
+    hid = p["x"] + o @ p["Wo"] + p["bo"]
+    return hid @ p["W1"] + p["b1"]
+
+
+CASES = [(1, 3, 4, 2, 8, 3), (2, 4, 4, 1, 6, 4)]  # b, s, h, heads, ffn width, seed
+
+
+@pytest.mark.parametrize("b,s,h,heads,f,seed", CASES)
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradients_match_central_differences(b, s, h, heads, f, seed, causal):
+    p = rand_layer(b, s, h, heads, seed=seed, f=f)
+    dy = np.random.default_rng(seed + 100).standard_normal((b, s, h))
+    # no ReLU pre-activation within reach of the step, so the loss is smooth there
+    assert np.abs(pre_activations(p, heads, causal)).min() > 1e-4
+    g = grads(p, dy, heads, causal)
+    eps = 1e-6
+    for name in NAMES:
+        arr = p[name]
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + eps
+            up = loss(p, dy, heads, causal)
+            arr[idx] = old - eps
+            down = loss(p, dy, heads, causal)
+            arr[idx] = old
+            num[idx] = (up - down) / (2 * eps)
+        np.testing.assert_allclose(g["d" + name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def torch_layer(p, heads, causal):
+    """The layer in torch (fp64), attention by torch's scaled_dot_product_attention."""
+    x = p["x"]
+    b, s, h = x.shape
+    dh = h // heads
+    q, k, v = (x @ p["Wqkv"] + p["bqkv"]).split(h, dim=-1)
+
+    def split(z):
+        return z.reshape(b, s, heads, dh).transpose(1, 2)
+
+    o = torch.nn.functional.scaled_dot_product_attention(split(q), split(k), split(v), is_causal=causal)
+    o = o.transpose(1, 2).reshape(b, s, h)
+    hid = x + o @ p["Wo"] + p["bo"]
+    return hid + torch.relu(hid @ p["W1"] + p["b1"]) @ p["W2"] + p["b2"]
+
+
+@pytest.mark.parametrize("b,s,h,heads,f", [(1, 5, 8, 2, 32), (2, 7, 16, 4, 24), (1, 16, 8, 1, 16)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradients_match_torch_autograd(b, s, h, heads, f, causal):
+    p = rand_layer(b, s, h, heads, seed=s + h, f=f)
+    dy = np.random.default_rng(7).standard_normal((b, s, h))
+    tp = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True) for k, v in p.items()}
+    y = torch_layer(tp, heads, causal)
+    (y * torch.tensor(dy)).sum().backward()
+    g = grads(p, dy, heads, causal)
+    for name in NAMES:
+        np.testing.assert_allclose(g["d" + name], tp[name].grad.numpy(), rtol=1e-9, atol=1e-10, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_value_gradient_conserves_the_output_gradient(causal):
+    # every row of P sums to 1, so per head the key rows of dV = P^T dO add up
+    # to the query rows of dO
+    rng = np.random.default_rng(3)
+    Q, K, V, dO = (rng.standard_normal((2, 9, 8)) for _ in range(4))
+    _, _, dV = obb.attention_backward(Q, K, V, dO, heads=2, causal=causal)
+    np.testing.assert_allclose(dV.sum(axis=1), dO.sum(axis=1), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("s", [1, 2, 3, 8, 12])
+@pytest.mark.parametrize("causal", [False, True])
+def test_blockwise_attention_backward_equals_plain(s, causal):
+    rng = np.random.default_rng(s)
+    Q, K, V, dO = (rng.standard_normal((2, s, 8)) for _ in range(4))
+    ref = obb.attention_backward(Q, K, V, dO, heads=2, causal=causal)
+    for qb in divisors(s):
+        for kb in divisors(s):
+            got = obb.attention_backward_blockwise(Q, K, V, dO, heads=2, causal=causal, q_block=qb, kv_block=kb)
+            for a, r in zip(got, ref):
+                np.testing.assert_allclose(a, r, rtol=0, atol=1e-12)
+
+
+def test_layer_backward_blockwise_equals_plain():
+    p = rand_layer(2, 8, 8, 2, seed=11)
+    dy = np.random.default_rng(12).standard_normal((2, 8, 8))
+    ref = grads(p, dy, 2, True)
+    got = grads(p, dy, 2, True, q_block=4, kv_block=2)
+    for name in NAMES:
+        np.testing.assert_allclose(got["d" + name], ref["d" + name], rtol=0, atol=1e-12, err_msg=name)

@@ -297,11 +297,16 @@ def our_arm(args, shape, name):
         bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal, out=out,
                           stream=stream)
 
+    # device memory the library takes (its pool keeps the workspace between
+    # calls): free memory before the first call minus free memory after warm-up
+    torch.cuda.synchronize(device)
+    free_pre, _ = torch.cuda.mem_get_info(device)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
     if bpt.device_status() != 0:
         raise RuntimeError("device error during warm-up")
+    free_post, _ = torch.cuda.mem_get_info(device)
 
     # ---- timed region (device time, CUDA events on the launching stream)
     torch.cuda.reset_peak_memory_stats(device)
@@ -409,6 +414,7 @@ def our_arm(args, shape, name):
         "memory": {"workspace_bytes": ws_bytes, "ratio_bytes_vs_2bsh": ws_bytes / (2 * tokens * shape.h),
                    "ratio_elems_vs_2bsh": ws_bytes / 2 / (2 * tokens * shape.h),
                    "peak_torch_alloc_bytes_in_step": int(peak_bytes),
+                   "device_bytes_taken_by_library": int(free_pre - free_post),
                    "free_bytes_before": int(free0)},
     }
     print(json.dumps(line))

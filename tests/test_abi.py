@@ -5,6 +5,7 @@ checks run before any CUDA call, so these run on a CPU-only machine)."""
 import os
 import re
 
+import numpy as np
 import pytest
 
 import blockwise_attn_ffn_bpt_b200 as bpt
@@ -219,3 +220,32 @@ def test_kernel_timing_log_is_empty_without_launches():
     assert bpt.kernel_times() == {}
     bpt.set_kernel_timing(False)
     assert bpt.launch_count() >= 0
+
+
+def test_default_wave_keeps_to_its_memory_budget():
+    # over many valid shapes: the default workspace holds K and V, and its
+    # wave scratch stays within the larger of 1.5x the K/V bytes and the
+    # scratch of a ~4096-row wave (whole query blocks, or whole sequences)
+    rng = np.random.default_rng(0)
+
+    def up(v):
+        return (v + 1023) // 1024 * 1024
+
+    def scratch(wr, h, f):
+        return up(wr * h * 4) + up(wr * h * 2) + up(wr * f * 2)
+
+    for _ in range(300):
+        heads = int(rng.integers(1, 9))
+        h = heads * int(rng.choice([64, 128]))
+        q_block = int(rng.choice([1, 16, 64, 128, 512, 1024]))
+        s = q_block * int(rng.integers(1, 65))
+        b = int(rng.integers(1, 5))
+        f = 64 * int(rng.integers(1, 4 * h // 64 + 9))
+        ws = bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, ffn=f)
+        kv = 2 * up(b * s * h * 2)
+        floor_rows = max(q_block, 4096 // q_block * q_block) if s >= 4096 else min(b, 4096 // s) * s
+        budget = max(kv // 2 * 3, scratch(floor_rows, h, f))
+        assert ws >= kv
+        assert ws <= max(kv, budget + 3 * 1024), (b, s, h, heads, q_block, f)
+        # and no smaller than the explicit one-block wave
+        assert ws >= bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, q_block, ffn=f)

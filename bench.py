@@ -423,6 +423,18 @@ def our_arm(args, shape, name):
     return 0
 
 
+def largest_fitting(need, budget: int, unit: int) -> int:
+    """The largest multiple n * unit (n >= 1) with need(n * unit) <= budget, for
+    a need that grows with its argument; unit when even that does not fit."""
+    lo, hi = 1, 2
+    while need(hi * unit) <= budget:
+        lo, hi = hi, hi * 2
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if need(mid * unit) <= budget else (lo, mid)
+    return lo * unit
+
+
 def max_context_arm(args):
     """The longest single sequence one 7B-class BPT layer forward (h 4096, 32
     heads, causal, q_block 1024, kv_block 2048) fits on this GPU, measured by
@@ -456,13 +468,7 @@ def max_context_arm(args):
     def need(s):
         return s * h * 2 + s * h * 4 + bpt.workspace_bytes(0, 1, s, h, heads, qb, kvb)
 
-    lo, hi = 1, (free - margin) // (10 * h * kvb) + 2
-    while need(hi * kvb) <= free - margin:
-        hi *= 2
-    while hi - lo > 1:
-        mid = (lo + hi) // 2
-        lo, hi = (mid, hi) if need(mid * kvb) <= free - margin else (lo, mid)
-    s = lo * kvb
+    s = largest_fitting(need, free - margin, kvb)
     x = torch.empty((1, s, h), dtype=torch.bfloat16, device=device)
     chunk = 1 << 16
     for r0 in range(0, s, chunk):

@@ -95,3 +95,18 @@ def test_reference_arm_runs_on_rank_zero_only():
                   env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("unit", [1, 7, 2048])
+def test_largest_fitting_length_is_the_largest_that_fits(unit):
+    # need grows with the length, like the layer's bytes (x + out + workspace)
+    def need(s):
+        return 10 * s + (s // 3) * 2 + 1000
+
+    for budget in (1000, 1010 + 10 * unit, 5_000, 123_457, 10_000_000):
+        s = bench.largest_fitting(need, budget, unit)
+        assert s % unit == 0 and s >= unit
+        if need(unit) <= budget:
+            assert need(s) <= budget < need(s + unit)
+        else:
+            assert s == unit  # nothing fits: the smallest length is reported

@@ -746,6 +746,11 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
     if (!aligned16(q)) return BPT_ERR_ALIGN;
   if (x_stride < 0 || out_stride < 0 || (x_stride && (size_t)x_stride < xb) || (out_stride && (size_t)out_stride < ob))
     return BPT_ERR_SHAPE;
+  // the host ranges must be addressable: stride * (n - 1) + size without overflow
+  const size_t lim = (size_t)1 << 62;
+  if ((x_stride && (size_t)(n - 1) > (lim - xb) / (size_t)x_stride) ||
+      (out_stride && (size_t)(n - 1) > (lim - ob) / (size_t)out_stride))
+    return BPT_ERR_SHAPE;
   // host ranges: every input against every output (both are arithmetic progressions)
   const Range xr = rng(x_host, (size_t)x_stride * (n - 1) + xb), orr = rng(out_host, (size_t)out_stride * (n - 1) + ob);
   if (overlap(xr, orr)) return BPT_ERR_ALIAS;
@@ -919,7 +924,7 @@ int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, co
 }
 
 int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stream) {
-  if (n < 0) return BPT_ERR_SHAPE;
+  if (n < 0 || n > (1LL << 60)) return BPT_ERR_SHAPE;
   if (n == 0) return BPT_OK;
   if (!src || !dst) return BPT_ERR_NULL;
   if (!aligned16(src) || !aligned16(dst)) return BPT_ERR_ALIGN;

@@ -189,6 +189,7 @@ def test_host_entry_validates_before_touching_memory():
     assert L.bpt_layer_forward_host(0, xh, xb, *w, *shp, xh + xb, ob, 2, None) == ALIAS  # out inside the inputs
     assert L.bpt_layer_forward_host(0, xh, 0, *w, *shp, xh, 0, 3, None) == ALIAS
     assert L.bpt_layer_forward_host(5, xh, xb, *w, *shp, oh, ob, 2, None) == DTYPE
+    assert L.bpt_layer_forward_host(0, xh, 1 << 40, *w, *shp, oh, ob, 1 << 30, None) == SHAPE  # range overflows
     assert L.bpt_layer_forward_host(0, xh, xb, *w, 1, 256, 256, 3, 64, 64, 1, oh, ob, 2, None) == SHAPE
     assert L.bpt_layer_forward_host(0, xh, xb, *w, 1, 256, 256, 4, 48, 64, 1, oh, ob, 2, None) == BLOCK
 
@@ -203,6 +204,7 @@ def test_convert_entry_validates():
     assert L.bpt_convert_f32_to_bf16(a + 4, b, 8, None) == ALIGN
     assert L.bpt_convert_f32_to_bf16(a, b + 8, 8, None) == ALIGN
     assert L.bpt_convert_f32_to_bf16(a, a + 16, 8, None) == ALIAS
+    assert L.bpt_convert_f32_to_bf16(a, b, (1 << 60) + 1, None) == SHAPE
 
 
 def test_stage_entry_points_validate():

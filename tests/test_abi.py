@@ -251,3 +251,27 @@ def test_default_wave_keeps_to_its_memory_budget():
         assert ws <= max(kv, budget + 3 * 1024), (b, s, h, heads, q_block, f)
         # and no smaller than the explicit one-block wave
         assert ws >= bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, q_block, ffn=f)
+
+
+def test_binding_checks_parameters_before_calling_the_library():
+    # shape and dtype checks run in Python, before any pointer reaches the C ABI
+    import torch
+
+    b, s, h = 1, 8, 64
+    x = torch.zeros((b, s, h), dtype=torch.bfloat16)
+    good = {"Wqkv": (h, 3 * h), "bqkv": (3 * h,), "Wo": (h, h), "bo": (h,), "W1": (h, 4 * h), "b1": (4 * h,),
+            "W2": (4 * h, h), "b2": (h,)}
+    params = {k: torch.zeros(shp, dtype=torch.bfloat16) for k, shp in good.items()}
+    bad = dict(params, W2=torch.zeros((4 * h, h + 64), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="W2"):
+        bpt.layer_forward(x, bad, 1, 8, 8, True, out=torch.empty((b, s, h)))
+    bad = dict(params, bo=torch.zeros((h,), dtype=torch.float32))
+    with pytest.raises(TypeError, match="bo"):
+        bpt.layer_forward(x, bad, 1, 8, 8, True, out=torch.empty((b, s, h)))
+    with pytest.raises(TypeError):
+        bpt.layer_forward(x.to(torch.float16), params, 1, 8, 8, True, out=torch.empty((b, s, h)))
+    # the host entry wants host inputs and CUDA weights
+    with pytest.raises(ValueError):
+        bpt.layer_forward_host(x, params, 1, 8, 8, True, out_host=torch.empty((b, s, h)))
+    with pytest.raises(TypeError):
+        bpt.convert_f32_to_bf16(torch.zeros(4))

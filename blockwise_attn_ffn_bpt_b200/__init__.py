@@ -24,8 +24,8 @@ EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
     "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
     "bpt_layer_forward_host", "bpt_convert_f32_to_bf16",
-    "bpt_qkv_projection", "bpt_attention", "bpt_device_status", "bpt_launch_count", "bpt_set_kernel_timing",
-    "bpt_kernel_times",
+    "bpt_qkv_projection", "bpt_attention", "bpt_stream_status", "bpt_device_status", "bpt_wait_flag",
+    "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
 )
 
 
@@ -74,8 +74,12 @@ def lib() -> ctypes.CDLL:
     L.bpt_qkv_projection.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
     L.bpt_attention.restype = i
     L.bpt_attention.argtypes = [vp] * 3 + [i] * 7 + [vp, vp]
+    L.bpt_stream_status.restype = i
+    L.bpt_stream_status.argtypes = [vp]
     L.bpt_device_status.restype = i
     L.bpt_device_status.argtypes = []
+    L.bpt_wait_flag.restype = i
+    L.bpt_wait_flag.argtypes = [vp, i, i, vp]
     L.bpt_launch_count.restype = ctypes.c_uint64
     L.bpt_launch_count.argtypes = []
     L.bpt_set_kernel_timing.restype = i
@@ -214,13 +218,6 @@ def layer_forward_host(x_host: torch.Tensor, params: dict, heads: int, q_block: 
     return out_host
 
 
-def layer_forward_from_host(x_host: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int,
-                            causal: bool, out_host: Optional[torch.Tensor] = None,
-                            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """One input [b, s, h] from host memory to a host fp32 result (see layer_forward_host)."""
-    return layer_forward_host(x_host, params, heads, q_block, kv_block, causal, out_host=out_host, stream=stream)
-
-
 def convert_f32_to_bf16(src: torch.Tensor, out: Optional[torch.Tensor] = None,
                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """src (fp32, CUDA) rounded to bf16 by the library's kernel."""
@@ -273,8 +270,26 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int, q_b
     return o
 
 
+def stream_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise `stream` (default: the current stream) and return, then
+    clear, the status word of the library's work queued on it (0 = BPT_OK)."""
+    return int(lib().bpt_stream_status(_stream(stream)))
+
+
 def device_status() -> int:
+    """Synchronise the whole device and return, then clear, the status words
+    of every stream of it (0 = BPT_OK). Stalls every stream; prefer
+    stream_status."""
     return int(lib().bpt_device_status())
+
+
+def wait_flag(flag: torch.Tensor, value: int, timeout_us: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Queue a bounded wait on `stream` until flag[0] (an int32 CUDA tensor)
+    equals value; if it gives up after timeout_us, the stream's status word
+    records BPT_ERR_TIMEOUT (a check of the status path)."""
+    if flag.dtype != torch.int32 or not flag.is_cuda:
+        raise TypeError("flag must be an int32 CUDA tensor")
+    _check(lib().bpt_wait_flag(_ptr(flag), int(value), int(timeout_us), _stream(stream)), "bpt_wait_flag")
 
 
 def launch_count() -> int:

@@ -74,6 +74,7 @@ struct AttnArgs {
   __nv_bfloat16* o; // output rows: (beta - beta0) * t_len + (t - t_start)
   long long ldo;
   float scale_log2; // log2(e) / sqrt(dh)
+  int* status;      // status word of the launching stream
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]: bf16 A read from tensor memory (K-major).
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const uint32_t o_done0 = smem_addr(bars + 5);   // [2] per query tile
   const uint32_t mma_done = smem_addr(bars + 9);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  const Abort abort_flag{reinterpret_cast<volatile int*>(bars + 11), args.status};
   const uint32_t ring_full0 = smem_addr(bars + 12);             // [RING]
   const uint32_t ring_empty0 = smem_addr(bars + 12 + C::RING);  // [RING]
 
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(ring_empty0 + 8 * i, 1);
     }
     mbar_init(mma_done, 1);
-    *abort_flag = 0;
+    *abort_flag.flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -192,9 +193,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         // never leave with copies still landing in shared memory
         volatile int dummy = 0;
-        mbar_wait(q_full, 0, &dummy);
+        const Abort drain{&dummy, args.status};
+        mbar_wait(q_full, 0, drain);
         for (int i = 0; i < C::RING; ++i)
-          if (issued & (1u << i)) mbar_wait(ring_full0 + 8 * i, (par >> i) & 1u, &dummy);
+          if (issued & (1u << i)) mbar_wait(ring_full0 + 8 * i, (par >> i) & 1u, drain);
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -371,7 +373,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 1) {
     if (lane == 0) {
       volatile int dummy = 0;
-      mbar_wait(mma_done, 0, &dummy);
+      mbar_wait(mma_done, 0, Abort{&dummy, args.status});
     }
     __syncwarp();
     tc_fence_after();

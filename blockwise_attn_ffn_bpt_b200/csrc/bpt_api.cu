@@ -175,6 +175,73 @@ int check_device(int* sms) {
   return BPT_OK;
 }
 
+// ------------------------------------------------------------- stream status
+// Each (device, stream) that launches this library's kernels owns one word of
+// g_status_slots on that device, assigned at its first call and kept for the
+// life of the process; word 0 is shared by every stream past the first
+// kStatusSlots - 1 of a device. The table of stream handles is a fixed array
+// (open addressing), so assigning a word allocates nothing. The device address
+// of the array is looked up on every call (a symbol lookup, no allocation), so
+// it stays right after a cudaDeviceReset recreates the module.
+std::mutex g_status_mu;
+uintptr_t g_status_key[64][kStatusSlots];
+bool g_status_used[64][kStatusSlots];
+
+int status_base(int** base) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_slots) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  *base = reinterpret_cast<int*>(p);
+  return BPT_OK;
+}
+
+// Index of the stream's word on the current device; -1 if it has none and
+// `create` is false.
+int status_index(int dev, cudaStream_t st, bool create) {
+  const uintptr_t key = reinterpret_cast<uintptr_t>(st);
+  constexpr int n = kStatusSlots - 1;  // words 1 .. kStatusSlots - 1
+  const int start = (int)((key >> 4) * 0x9E3779B97F4A7C15ull >> 40) % n;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  for (int i = 0; i < n; ++i) {
+    const int idx = 1 + (start + i) % n;
+    if (!g_status_used[dev][idx]) {
+      if (!create) return -1;
+      g_status_used[dev][idx] = true;
+      g_status_key[dev][idx] = key;
+      return idx;
+    }
+    if (g_status_key[dev][idx] == key) return idx;
+  }
+  return 0;  // table full: the shared word
+}
+
+// Device address of the status word of `st` on the current device.
+int stream_status_word(cudaStream_t st, int** word) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  int* base = nullptr;
+  const int r = status_base(&base);
+  if (r != BPT_OK) return r;
+  *word = base + status_index(dev, st, true);
+  return BPT_OK;
+}
+
+// A single thread waits until *flag == value, at most timeout_ns; if it gives
+// up it records BPT_ERR_TIMEOUT in the stream's status word.
+__global__ void wait_flag_kernel(const int* flag, int value, unsigned long long timeout_ns, int* status) {
+  if (threadIdx.x != 0) return;
+  const unsigned long long t0 = global_timer_ns();
+  while (*reinterpret_cast<const volatile int*>(flag) != value) {
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicExch(status, (int)BPT_ERR_TIMEOUT);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
 // ------------------------------------------------------------- workspace pool
 // The allocating entry points take their workspace from a library-owned,
 // stream-ordered memory pool per device that keeps freed memory for the next
@@ -278,16 +345,23 @@ int default_wave_rows(int b, int s, int h, int ffn, int q_block) {
                                          : (long long)std::min(b, 4096 / s) * s;
   const size_t budget = std::max(kv_bytes(b, s, h) / 2 * 3, wave_scratch_bytes(floor_rows, h, ffn));
   const long long max_rows = std::max<long long>(q_block, (long long)(budget / per_row));
-  std::vector<std::pair<long long, long long>> cand;  // (modelled steps, wave rows)
-  for (long long wr = q_block; wr < s && wr <= max_rows; wr += q_block)
-    cand.push_back({b * ((s / wr) * wave_steps(wr, h, ffn) + wave_steps(s % wr, h, ffn)), wr});
-  for (long long g = 1; g <= b && (g * s <= max_rows || cand.empty()); ++g)
-    cand.push_back({(b / g) * wave_steps(g * s, h, ffn) + wave_steps((b % g) * s, h, ffn), g * s});
-  long long best = cand[0].first;
-  for (const auto& c : cand) best = std::min(best, c.first);
+  // candidates (modelled steps, wave rows): whole numbers of query blocks
+  // shorter than a sequence, then whole numbers of sequences; two passes over
+  // them (the best time, then the smallest wave within 1% of it) keep this
+  // free of allocations
+  auto visit = [&](auto&& f) {
+    bool any = false;
+    for (long long wr = q_block; wr < s && wr <= max_rows; wr += q_block, any = true)
+      f(b * ((s / wr) * wave_steps(wr, h, ffn) + wave_steps(s % wr, h, ffn)), wr);
+    for (long long g = 1; g <= b && (g * s <= max_rows || !any); ++g, any = true)
+      f((b / g) * wave_steps(g * s, h, ffn) + wave_steps((b % g) * s, h, ffn), g * s);
+  };
+  long long best = -1;
+  visit([&](long long steps, long long) { best = best < 0 ? steps : std::min(best, steps); });
   long long pick = 0;
-  for (const auto& c : cand)
-    if (c.first * 100 <= best * 101 && (pick == 0 || c.second < pick)) pick = c.second;
+  visit([&](long long steps, long long wr) {
+    if (steps * 100 <= best * 101 && (pick == 0 || wr < pick)) pick = wr;
+  });
   return (int)std::min<long long>(pick, 0x7fffffffLL);
 }
 
@@ -301,18 +375,25 @@ int wave_rows_for(int b, int s, int h, int ffn, int q_block, int wave_rows) {
   return (int)wr;
 }
 
-std::vector<Wave> plan_waves(int b, int s, int h, int ffn, int q_block, int wave_rows) {
-  std::vector<Wave> w;
+// Calls f(wave) for each wave of the FFN side in order and returns the first
+// status other than BPT_OK (or BPT_OK).
+template <class F>
+int for_each_wave(int b, int s, int h, int ffn, int q_block, int wave_rows, F&& f) {
   const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
   if (wr >= s) {
     const int g = wr / s;
-    for (int beta = 0; beta < b; beta += g) w.push_back(Wave{(long long)beta * s, beta, std::min(g, b - beta), 0, s});
+    for (int beta = 0; beta < b; beta += g) {
+      const int r = f(Wave{(long long)beta * s, beta, std::min(g, b - beta), 0, s});
+      if (r != BPT_OK) return r;
+    }
   } else {
     for (int beta = 0; beta < b; ++beta)
-      for (int ts = 0; ts < s; ts += wr)
-        w.push_back(Wave{(long long)beta * s + ts, beta, 1, ts, std::min(wr, s - ts)});
+      for (int ts = 0; ts < s; ts += wr) {
+        const int r = f(Wave{(long long)beta * s + ts, beta, 1, ts, std::min(wr, s - ts)});
+        if (r != BPT_OK) return r;
+      }
   }
-  return w;
+  return BPT_OK;
 }
 
 // ------------------------------------------------------------- workspace layout
@@ -358,8 +439,10 @@ Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave
 // blocks of B pair with A's blocks as a_block() maps them (split products).
 template <int MODE>
 int launch_gemm_split(const void* A, long long M, long long a_cols, long long lda, const void* B, long long K,
-                      long long N, int a_split, int a_kb, GemmArgs args, int sms, cudaStream_t st, const char* name) {
+                      long long N, int a_split, int a_kb, GemmArgs args, int sms, cudaStream_t st, int* status,
+                      const char* name) {
   if (M <= 0) return BPT_OK;
+  args.status = status;
   CUtensorMap ta, tb;
   if (!map_rows(&ta, A, M, a_cols, lda, GEMM_BM)) return BPT_ERR_CUDA;
   if (!map_rows(&tb, B, K, N, N, 64)) return BPT_ERR_CUDA;
@@ -381,15 +464,15 @@ int launch_gemm_split(const void* A, long long M, long long a_cols, long long ld
 
 template <int MODE>
 int launch_gemm(const void* A, long long M, long long K, long long lda, const void* B, long long N,
-                GemmArgs args, int sms, cudaStream_t st, const char* name) {
-  return launch_gemm_split<MODE>(A, M, K, lda, B, K, N, 0, 0, args, sms, st, name);
+                GemmArgs args, int sms, cudaStream_t st, int* status, const char* name) {
+  return launch_gemm_split<MODE>(A, M, K, lda, B, K, N, 0, 0, args, sms, st, status, name);
 }
 
 // Attention of the query rows [t_start, t_start + t_len) of sequences
 // beta0 .. beta0 + n_seq - 1; q rows have `ldq` elements between them.
 int launch_attention(const void* q, long long ldq, const void* k, const void* v, int b, int s, int h, int heads,
                      int causal, int beta0, int n_seq, int t_start, int t_len, __nv_bfloat16* o, long long ldo,
-                     cudaStream_t st) {
+                     cudaStream_t st, int* status) {
   const int dh = h / heads;
   CUtensorMap tq, tk, tv;
   if (!map_seq(&tq, q, b, s, h, ldq) || !map_seq(&tk, k, b, s, h, h) || !map_seq(&tv, v, b, s, h, h))
@@ -403,6 +486,7 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
   a.n_pairs = (t_len + 2 * ATT_BM - 1) / (2 * ATT_BM);
   a.ldo = ldo;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  a.status = status;
   for (int z0 = 0; z0 < n_seq; z0 += 65535) {
     const int nz = std::min(65535, n_seq - z0);
     a.beta0 = beta0 + z0;
@@ -524,6 +608,8 @@ int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads
 
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
               int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms) {
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
   const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
   const long long tok = (long long)b * s;
   __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(ws + L.k);
@@ -571,17 +657,17 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.h = h;
     if (f32)
       BPT_TRY(launch_gemm_split<EPI_QKV>(xa, tok, 2LL * h, 2LL * h, wqkv, 3LL * h, 3LL * h, 2, h / GEMM_BK, a, sms,
-                                         st, "gemm_qkv"));
+                                         st, status, "gemm_qkv"));
     else
-      BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, "gemm_qkv"));
+      BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, status, "gemm_qkv"));
   }
 
   // steps 4-10 for every query block at once: each CTA overwrites the Q of its
   // own rows and head with their attention output
-  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st));
+  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st, status));
 
   // step 11 per wave of query blocks: out-projection, residuals and FFN
-  for (const Wave& w : plan_waves(b, s, h, ffn, q_block, wave_rows)) {
+  return for_each_wave(b, s, h, ffn, q_block, wave_rows, [&](const Wave& w) -> int {
     const long long rows = w.rows();
     GemmArgs a{};
     a.resid = p.x;
@@ -598,17 +684,16 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.ld_dst = h;
     const int sp = f32 ? 1 : 0, kf = f32 ? 2 : 1;  // fp32 inputs: A against [W_hi; W_lo]
     BPT_TRY(launch_gemm_split<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, (long long)kf * h, h, sp,
-                                           h / GEMM_BK, a, sms, st, "gemm_outproj"));
+                                           h / GEMM_BK, a, sms, st, status, "gemm_outproj"));
     a.bias = p.b1;
     a.dst = U;
     a.ld_dst = ffn;
     BPT_TRY(launch_gemm_split<EPI_FFN_UP>(HB, rows, h, h, w1, (long long)kf * h, ffn, sp, h / GEMM_BK, a, sms, st,
-                                          "gemm_ffn_up"));
+                                          status, "gemm_ffn_up"));
     a.bias = p.b2;
-    BPT_TRY(launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
-                                            st, "gemm_ffn_down"));
-  }
-  return BPT_OK;
+    return launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
+                                           st, status, "gemm_ffn_down");
+  });
 }
 
 int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int kv_block,
@@ -652,27 +737,21 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
 
 // Scratch of bpt_layer_forward_noalloc: one fixed array in device memory,
 // created with the library image on every device that loads it. In host code
-// the name g_static_ws denotes a host-side stand-in, never the device address:
-// the address is looked up per device with cudaGetSymbolAddress.
+// the name g_static_ws denotes a host-side stand-in, never the device address.
 static __device__ __align__(256) unsigned char g_static_ws[BPT_STATIC_WORKSPACE_BYTES];
 
-std::mutex g_static_mu;
-void* g_static_ptr[64] = {};
-
-// Device address of g_static_ws on the current device (looked up once per device).
+// Device address of g_static_ws on the current device. It is looked up on
+// every call, with the device current: a symbol lookup allocates nothing, and
+// an address saved from an earlier call would be stale once cudaDeviceReset
+// (or a new context on the device) has recreated the module. The first call
+// on a device also loads the library's device image there.
 int static_workspace(void** ptr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_static_mu);
-  if (!g_static_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return BPT_ERR_CUDA;
-    }
-    g_static_ptr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
   }
-  *ptr = g_static_ptr[dev];
+  *ptr = p;
   return BPT_OK;
 }
 
@@ -953,8 +1032,10 @@ int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b,
   a.v = reinterpret_cast<__nv_bfloat16*>(v);
   a.ldkv = h;
   a.h = h;
-  return launch_gemm<EPI_QKV>(x, (long long)b * s, h, h, Wqkv, 3LL * h, a, sms,
-                              reinterpret_cast<cudaStream_t>(stream), "gemm_qkv");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  return launch_gemm<EPI_QKV>(x, (long long)b * s, h, h, Wqkv, 3LL * h, a, sms, st, status, "gemm_qkv");
 }
 
 int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int q_block,
@@ -969,16 +1050,81 @@ int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int
     if (!aligned16(p)) return BPT_ERR_ALIGN;
   int sms = 0;
   BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
   return launch_attention(q, h, k, v, b, s, h, heads, causal, 0, b, 0, s, reinterpret_cast<__nv_bfloat16*>(o), h,
-                          reinterpret_cast<cudaStream_t>(stream));
+                          st, status);
+}
+
+int bpt_stream_status(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  const int idx = status_index(dev, st, false);
+  if (idx < 0) return BPT_OK;  // no call of this library ever ran on the stream
+  int* base = nullptr;
+  BPT_TRY(status_base(&base));
+  int v = 0;
+  if (cudaMemcpyAsync(&v, base + idx, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  if (v != BPT_OK && (cudaMemsetAsync(base + idx, 0, sizeof(int), st) != cudaSuccess ||
+                      cudaStreamSynchronize(st) != cudaSuccess)) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  return v;
 }
 
 int bpt_device_status(void) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return BPT_ERR_CUDA;
-  int v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return BPT_ERR_CUDA;
-  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BPT_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  static int words[kStatusSlots];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cudaMemcpyFromSymbol(words, g_status_slots, sizeof(words)) != cudaSuccess) {
+    cudaGetLastError();
+    return BPT_ERR_CUDA;
+  }
+  int v = BPT_OK;
+  for (int w : words)
+    if (w != BPT_OK && v == BPT_OK) v = w;
+  if (v != BPT_OK) {
+    std::memset(words, 0, sizeof(words));
+    if (cudaMemcpyToSymbol(g_status_slots, words, sizeof(words)) != cudaSuccess) {
+      cudaGetLastError();
+      return BPT_ERR_CUDA;
+    }
+  }
   return v;
+}
+
+int bpt_wait_flag(const int* flag, int value, int timeout_us, void* stream) {
+  if (!flag) return BPT_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(flag) & 3u) != 0) return BPT_ERR_ALIGN;
+  if (timeout_us < 0 || timeout_us > 10000000) return BPT_ERR_SHAPE;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  {
+    LaunchScope ls("wait_flag", st);
+    wait_flag_kernel<<<1, 32, 0, st>>>(flag, value, (unsigned long long)timeout_us * 1000ull, status);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
 uint64_t bpt_launch_count(void) { return g_launches.load(); }

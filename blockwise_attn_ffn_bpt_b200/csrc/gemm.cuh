@@ -66,6 +66,7 @@ struct GemmArgs {
   // 2 a_kb blocks, then kb - a_kb (A = [x_hi | x_lo] against [W_hi; W_lo; W_hi]).
   int a_split;
   int a_kb;  // K blocks of one copy of A
+  int* status;  // status word of the launching stream
 };
 
 // K block of A that pairs with K block kb of B
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t tempty0 = smem_addr(bars + 2 * GEMM_STAGES + 2);
   const uint32_t mma_done = smem_addr(bars + 2 * GEMM_STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * GEMM_STAGES + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * GEMM_STAGES + 6);
+  const Abort abort_flag{reinterpret_cast<volatile int*>(bars + 2 * GEMM_STAGES + 6), args.status};
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(tempty0 + 8 * i, 4);
     }
     mbar_init(mma_done, 1);
-    *abort_flag = 0;
+    *abort_flag.flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       for (int i = 0; i < GEMM_STAGES; ++i)
         if (issued & (1u << i)) {
           volatile int dummy = 0;
-          mbar_wait(full0 + 8 * i, (last_parity >> i) & 1u, &dummy);
+          mbar_wait(full0 + 8 * i, (last_parity >> i) & 1u, Abort{&dummy, args.status});
         }
     }
   } else if (warp == 1) {
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 1) {
     if (lane == 0) {
       volatile int dummy = 0;
-      mbar_wait(mma_done, 0, &dummy);
+      mbar_wait(mma_done, 0, Abort{&dummy, args.status});
     }
     __syncwarp();
     tc_fence_after();

@@ -11,10 +11,14 @@
 
 namespace bpt {
 
-// Device-side error word of the library: kernels that give up a wait record
-// BPT_ERR_TIMEOUT here; the host reads it with bpt_device_status(). The
-// library is one translation unit, which holds this definition.
-__device__ int g_device_error = 0;
+// Device-side status words, one per (device, stream) that has run this
+// library's kernels: a kernel that gives up a wait records BPT_ERR_TIMEOUT in
+// the word of the stream it was launched on (its address comes in the
+// kernel's arguments), and bpt_stream_status() reads and clears that word.
+// Zero at module load. The library is one translation unit, which holds this
+// definition.
+constexpr int kStatusSlots = 1024;
+__device__ int g_status_slots[kStatusSlots];
 
 // A wait that makes no progress for this long is abandoned (the kernel then
 // records BPT_ERR_TIMEOUT, skips its remaining work and exits cleanly).
@@ -63,20 +67,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Where a kernel that gives up records it: the CTA's abort flag (shared
+// memory, seen by every role of the CTA) and the status word of the launching
+// stream (global memory, read by the host).
+struct Abort {
+  volatile int* flag;
+  int* status;
+};
+
 // Wait for the phase with the given parity to complete. Returns false (and
-// raises the CTA's abort flag and the device error word) if the wait made no
-// progress for kWaitTimeoutNs, or if another thread of the CTA already gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// raises the CTA's abort flag and the stream's status word) if the wait made
+// no progress for kWaitTimeoutNs, or if another thread of the CTA already
+// gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
+    if (*ab.flag) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-      *abort_flag = 1;
-      atomicExch(&g_device_error, (int)BPT_ERR_TIMEOUT);
+      *ab.flag = 1;
+      atomicExch(ab.status, (int)BPT_ERR_TIMEOUT);
       return false;
     }
   }
@@ -86,8 +99,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // resumes about 100 clocks after the phase completes; one whose lane 0 polls
 // alone and then broadcasts takes over twice as long, and several times that
 // while other warps of the SM are busy. The outcome is warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
+  const bool ok = mbar_wait(bar, parity, ab);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -49,10 +49,11 @@
  *   nothing launched and nothing written. Otherwise the call is asynchronous on
  *   `stream` (a cudaStream_t; NULL means the legacy default stream) and
  *   returns BPT_OK once all kernels are queued. Device-side failures (a
- *   bounded wait that gave up) are reported by bpt_device_status().
- * - Reentrancy: calls on different streams may run concurrently; the only
- *   process-wide state is the device error word, the launch counter and the
- *   optional kernel timing log.
+ *   bounded wait that gave up) are recorded in a status word owned by the
+ *   stream the kernels ran on, and bpt_stream_status(stream) reports them.
+ * - Reentrancy: calls on different streams may run concurrently; each stream
+ *   has its own device status word. The other process-wide state is the
+ *   launch counter and the optional kernel timing log.
  */
 #ifndef BPT_H_
 #define BPT_H_
@@ -83,14 +84,20 @@ typedef enum bpt_dtype {
   BPT_DTYPE_F32 = 1
 } bpt_dtype;
 
-/* Human-readable name of a status code (static string, never NULL). */
+/* Human-readable name of a status code (static string, never NULL). A library
+ * utility; the pages have no counterpart. */
 const char* bpt_status_string(int status);
 
 /* ------------------------------------------------------------------------
  * The layer forward (Algorithm 1 of the BPT paper review, section 3).
  * ------------------------------------------------------------------------ */
 
-/* bf16 inputs. Allocates its workspace stream-ordered on `stream` from a
+/* The layer as the pages define it: Algorithm 1 steps 1-12 with Eq. 3 and its
+ * scaling operation for the attention and the blockwise FFN-with-residuals
+ * formula (paper review section 3), bf16 matmul inputs with fp32
+ * accumulation (paper review section 5, precision).
+ *
+ * bf16 inputs. Allocates its workspace stream-ordered on `stream` from a
  * library-owned memory pool of the current device and frees it stream-ordered
  * after the last kernel; the pool keeps freed memory for later calls (so
  * repeated calls do not map device memory again). Returns BPT_ERR_NOMEM if the
@@ -99,7 +106,12 @@ int bpt_layer_forward(const void* x, const void* Wqkv, const void* bqkv, const v
                       const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                       int heads, int q_block, int kv_block, int causal, float* out, void* stream);
 
-/* fp32 inputs (same arguments, fp32 tensors). The GEMMs keep about 16
+/* The same layer (Algorithm 1, paper review section 3) for fp32 inputs; the
+ * small fp32 workload of the test suite uses it. The pages fix bf16 matmul
+ * inputs with fp32 accumulation (section 5); this entry keeps more of the fp32
+ * inputs' precision than a plain bf16 rounding would.
+ *
+ * fp32 inputs (same arguments, fp32 tensors). The GEMMs keep about 16
  * significant bits of x and of the weights: each fp32 value v is split on the
  * device into bf16 parts hi = bf16(v) and lo = bf16(v - hi), and the products
  * x W_hi + x W_lo (projection: x_hi W_hi + x_hi W_lo + x_lo W_hi) accumulate in
@@ -108,7 +120,13 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
                           const float* W1, const float* b1, const float* W2, const float* b2, int b, int s, int h,
                           int heads, int q_block, int kv_block, int causal, float* out, void* stream);
 
-/* Bytes of workspace a caller must pass to bpt_layer_forward_ws for these
+/* Workspace of one layer call. The pages' memory analysis (paper review
+ * section 3, "memory analysis": 2bsh of activations per layer, FFN scratch
+ * per chunk of c rows, never per sequence) is what it is sized against.
+ * Departure from the plain (b, s, h, heads, q_block, kv_block) signature:
+ * dtype selects the element type of the inputs and wave_rows the FFN chunk.
+ *
+ * Bytes of workspace a caller must pass to bpt_layer_forward_ws for these
  * arguments (0 if they are invalid or b*s == 0): one region that holds the bf16
  * K and V of the whole input (2 * b*s*h * 2 bytes) until attention is done and
  * then the FFN scratch of one wave (14 * h bytes per wave row: fp32 residual
@@ -124,7 +142,11 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows);
 
-/* The layer with an FFN of any width ffn (the pages fix ffn = 4h; every
+/* The standard FFN max(0, x W1 + b1) W2 + b2 (paper review section 3, core
+ * formulas) has a hidden width the formula leaves open; the memory analysis'
+ * 8bch activation input implies 4h, which every other entry point uses.
+ *
+ * The layer with an FFN of any width ffn (the pages fix ffn = 4h; every
  * other entry point uses 4h): W1 is [h, ffn], b1 [ffn], W2 [ffn, h], in the
  * element type dtype. ffn must be a positive multiple of 64 (BPT_ERR_SHAPE
  * otherwise). workspace == NULL with ws_bytes == 0 takes the workspace from
@@ -139,7 +161,10 @@ int bpt_layer_forward_ffn(int dtype, const void* x, const void* Wqkv, const void
                           int s, int h, int heads, int ffn, int q_block, int kv_block, int causal, int wave_rows,
                           void* workspace, size_t ws_bytes, float* out, void* stream);
 
-/* The layer with a caller-owned workspace (device memory, 256-byte aligned,
+/* Algorithm 1 (paper review section 3) with the caller's workspace; same
+ * departure as bpt_layer_workspace_bytes (dtype, wave_rows).
+ *
+ * The layer with a caller-owned workspace (device memory, 256-byte aligned,
  * at least bpt_layer_workspace_bytes(...) bytes, not overlapping any argument;
  * BPT_ERR_NOMEM if ws_bytes is too small). dtype is a bpt_dtype and gives the
  * element type of x, the weights and the biases. Allocates nothing. */
@@ -148,7 +173,11 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
                          int s, int h, int heads, int q_block, int kv_block, int causal, int wave_rows,
                          void* workspace, size_t ws_bytes, float* out, void* stream);
 
-/* End to end from host memory: for i in [0, n_inputs), out_host + i *
+/* Algorithm 1 (paper review section 3) from its input sequence x in host
+ * memory to the layer's output in host memory; the copy pipeline has no
+ * counterpart in the pages.
+ *
+ * End to end from host memory: for i in [0, n_inputs), out_host + i *
  * out_stride receives the layer applied to x_host + i * x_stride (strides in
  * bytes; 0 reuses the same input, or writes every result to the same place).
  * x is [b, s, h] of dtype (bf16 or fp32) in host memory; out is fp32 [b, s, h]
@@ -168,7 +197,11 @@ int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, co
                            const void* b2, int b, int s, int h, int heads, int q_block, int kv_block, int causal,
                            float* out_host, long long out_stride, int n_inputs, void* stream);
 
-/* dst[i] = src[i] rounded to bf16 (nearest, ties to even), i < n; device
+/* Between the layers of a stack (the pages' models are stacks of BPT layers:
+ * paper review section 6, 1B-70B models) the fp32 output becomes the next
+ * layer's bf16 input, the matmul input precision of section 5.
+ *
+ * dst[i] = src[i] rounded to bf16 (nearest, ties to even), i < n; device
  * pointers, 16-byte aligned, not overlapping; asynchronous on `stream`.
  * Chains layers: one layer's fp32 out becomes the next layer's bf16 x (a
  * stack of BPT layers, as the pages' models are). Errors: BPT_ERR_SHAPE for
@@ -186,15 +219,17 @@ int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stre
  * which the library is loaded holds that array until the process exits.
  *
  * - Allocates nothing: no cudaMalloc / cudaMallocAsync / cudaFree, and no
- *   allocating library routine. The caller still owns x, the weights, the
- *   biases and out.
+ *   allocating library routine (nor host heap memory). The caller still owns
+ *   x, the weights, the biases and out.
  * - Size limit: returns BPT_ERR_NOMEM, with nothing launched, when the
  *   workspace the layer needs (bpt_layer_workspace_bytes(BPT_DTYPE_BF16, b, s,
  *   h, heads, q_block, kv_block, 0)) exceeds BPT_STATIC_WORKSPACE_BYTES; for
  *   example b=1, s=2048, h=1024 needs 28 MiB and fits, s=8192, h=2048 does not.
- * - The first call on each device looks up that device's address of the array
- *   (one cudaGetSymbolAddress, with that device current). Make that first call
- *   before any stream capture on the device.
+ * - Every call looks up the current device's address of the array (one
+ *   cudaGetSymbolAddress with that device current, which allocates nothing),
+ *   so the address is right even after cudaDeviceReset has recreated the
+ *   library's device image. The first call of this library on a device also
+ *   loads that image there; make it before any stream capture on the device.
  * - Every call on a device uses the same array, and it keeps whatever the last
  *   call left in it. No part of it needs to start at zero: each byte a call
  *   reads was written earlier in the same call. Calls whose work overlaps on
@@ -211,12 +246,19 @@ int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv,
  * Single steps of Algorithm 1, for checking intermediate results.
  * ------------------------------------------------------------------------ */
 
-/* Step 1: [Q | K | V] = x Wqkv + bqkv with bf16 x [b*s, h], Wqkv [h, 3h],
+/* Algorithm 1 step 1 (paper review section 3), with the fused projection of
+ * "Transformer QKV matrix computation and 3 parallel strategies", section 2.
+ *
+ * Step 1: [Q | K | V] = x Wqkv + bqkv with bf16 x [b*s, h], Wqkv [h, 3h],
  * bqkv [3h]; writes bf16 q, k, v, each [b*s, h] row-major. */
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,
                        void* v, void* stream);
 
-/* Steps 2-10: O = concat_k softmax(Q_k K_k^T / sqrt(dh)) V_k over all key
+/* Algorithm 1 steps 2-10 with Eq. 3 and its scaling operation (paper review
+ * section 3); heads split and concatenated as in "PyTorch 2.3 multi-head
+ * self-attention from QKV to 8 heads", sections 2-4.
+ *
+ * Steps 2-10: O = concat_k softmax(Q_k K_k^T / sqrt(dh)) V_k over all key
  * blocks with online-softmax rescaling; bf16 q, k, v [b, s, h] in, bf16 o
  * [b, s, h] out. q_block / kv_block are validated as for the layer. */
 int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int q_block,
@@ -226,14 +268,43 @@ int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int
  * Status and measurement.
  * ------------------------------------------------------------------------ */
 
-/* Synchronise the current device, return the device error word (BPT_OK or
- * BPT_ERR_TIMEOUT) and reset it to BPT_OK. BPT_ERR_CUDA if the sync failed. */
+/* Status of the work queued on one stream (library plumbing; the pages have
+ * no counterpart). Synchronises `stream` only (other streams keep running),
+ * then returns the status word owned by that stream on the current device --
+ * BPT_OK, or BPT_ERR_TIMEOUT if a kernel of this library launched on it gave
+ * up a bounded wait since the word was last read -- and resets the word to
+ * BPT_OK. A status recorded on another stream is neither returned nor cleared.
+ * Call it with the device current on which the work was queued. Returns
+ * BPT_ERR_CUDA if the synchronisation or the read fails (for example when no
+ * GPU is present). Words are assigned to streams at their first call and kept
+ * for the life of the process; past 1023 distinct streams on one device the
+ * further ones share one word. A destroyed stream's word passes to a later
+ * stream that gets the same handle, so read a stream's status before
+ * destroying it. */
+int bpt_stream_status(void* stream);
+
+/* Every stream of the current device at once: synchronises the whole device,
+ * returns the first status word that is not BPT_OK (or BPT_OK) and resets all
+ * words of the device. It stalls every stream of the device; prefer
+ * bpt_stream_status. */
 int bpt_device_status(void);
 
-/* Number of kernels this library has launched in this process. */
+/* A check of the status path (library plumbing; the pages have no
+ * counterpart): one thread, queued on `stream`, waits until the int at `flag`
+ * (device or host-mapped memory, 4-byte aligned) equals `value`, for at most
+ * timeout_us microseconds; if it gives up it records BPT_ERR_TIMEOUT in the
+ * stream's status word, exactly as the layer's kernels do when one of their
+ * bounded waits runs out. The wait ends either way, so it never hangs the
+ * stream. Errors: BPT_ERR_NULL, BPT_ERR_ALIGN, BPT_ERR_SHAPE (timeout_us
+ * outside [0, 10^7]), with nothing launched. */
+int bpt_wait_flag(const int* flag, int value, int timeout_us, void* stream);
+
+/* Number of kernels this library has launched in this process (measurement
+ * support; the pages have no counterpart). */
 uint64_t bpt_launch_count(void);
 
-/* Kernel timing log: while enabled, every launch is bracketed by CUDA events
+/* Kernel timing log (measurement support; the pages have no counterpart).
+ * While enabled, every launch is bracketed by CUDA events
  * recorded on its own stream. bpt_kernel_times synchronises and writes, for at
  * most `max` kernel kinds, the name, launch count and summed milliseconds,
  * then clears the log; it returns the number of kinds written. */

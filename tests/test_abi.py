@@ -217,6 +217,28 @@ def test_stage_entry_points_validate():
     assert L.bpt_attention(p[0], p[1], p[2] + 4, 1, 128, 256, 2, 64, 64, 1, p[3], None) == ALIGN
 
 
+def test_status_entry_points_without_a_gpu():
+    # bpt_stream_status synchronises the stream it is given before it reads
+    # that stream's word: with no GPU the synchronisation fails, which it
+    # reports as BPT_ERR_CUDA instead of a status word (and it must not crash)
+    L = bpt.lib()
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("checks the no-GPU answer")
+    assert L.bpt_stream_status(None) == -7
+    assert L.bpt_stream_status(0x2) == -7  # the per-thread default stream handle
+    assert L.bpt_device_status() == -7
+
+
+def test_wait_flag_entry_validates():
+    L = bpt.lib()
+    f = BASE
+    assert L.bpt_wait_flag(None, 1, 1000, None) == NULL
+    assert L.bpt_wait_flag(f + 2, 1, 1000, None) == ALIGN
+    assert L.bpt_wait_flag(f, 1, -1, None) == SHAPE
+    assert L.bpt_wait_flag(f, 1, 10_000_001, None) == SHAPE
+
+
 def test_kernel_timing_log_is_empty_without_launches():
     bpt.set_kernel_timing(True)
     assert bpt.kernel_times() == {}

@@ -19,7 +19,6 @@ import argparse
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import tempfile
@@ -54,26 +53,34 @@ def layer_flops(shape: bi.LayerShape) -> dict:
     }
 
 
-def profiled_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, or None when there is none for this workload or the kernel's
-    source changed since the counters were taken."""
-    if kernel != "attention":
-        return None
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+
+
+def kernel_source_hash(files=("attention.cuh", "ptx.cuh")) -> str:
     import hashlib
-    path = os.path.join(ROOT, "profiles", "attention_s16384_h2048_causal.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    m_t = re.search(rf"traffic_per_launch_{re.escape(workload)}_bytes: (\d+)", text)
-    m_h = re.search(r"kernel_source_sha256_16: ([0-9a-f]+)", text)
-    if not (m_t and m_h):
-        return None
     h = hashlib.sha256()
-    for f in ("attention.cuh", "ptx.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "blockwise_attn_ffn_bpt_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    return int(m_t.group(1)) if h.hexdigest()[:16] == m_h.group(1) else None
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str, path: str = TRAFFIC_FILE):
+    """DRAM bytes per launch of the dominant kernel, from the data file written
+    beside its ncu summary; None when there is none for this workload or the
+    kernel's source changed since the counters were taken."""
+    if kernel != "attention" or not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    v = d.get("traffic_per_launch_bytes", {}).get(workload)
+    return int(v) if v is not None else None
+
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "bf16_tflops_sustained_sm_mhz": 1300.0}
 
 
 def measured_peaks() -> tuple[dict, str]:
@@ -81,7 +88,41 @@ def measured_peaks() -> tuple[dict, str]:
     if os.path.exists(path):
         with open(path) as f:
             return json.load(f), "measured"
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sustained_clock_mhz(peaks: dict):
+    """SM clock (MHz) at which the sustained bf16 peak was taken: a key of the
+    peaks record that names both 'sustain' and a clock, else the fallback's."""
+    stack = [peaks]
+    while stack:
+        d = stack.pop()
+        for k, v in d.items():
+            if isinstance(v, dict):
+                stack.append(v)
+            elif isinstance(v, (int, float)) and "sustain" in k.lower() and ("mhz" in k.lower() or "clock" in k.lower()):
+                return float(v)
+    return FALLBACK_PEAKS["bf16_tflops_sustained_sm_mhz"]
+
+
+def tensor_roofline(kernel: str, achieved: float, peaks: dict, src: str, sm_mhz, traffic) -> dict:
+    """Roofline object of a tensor-core kernel timed with CUDA events.
+
+    frac is against the burst bf16 peak (the denominator of a kernel that runs
+    at full clock, as this one does inside a step of tens of ms); the
+    sustained peak, scaled from the clock it was taken at to the clock sampled
+    during this run, is reported beside it."""
+    burst = float(peaks["bf16_tflops"])
+    sus = float(peaks.get("bf16_tflops_sustained", burst))
+    sus_mhz = sustained_clock_mhz(peaks)
+    scaled = sus * (sm_mhz / sus_mhz) if sm_mhz else None
+    return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+            "frac": achieved / burst, "traffic": traffic,
+            "peak_source": f"{src} bf16_tflops (burst, cuBLAS bf16 GEMM timed alone)",
+            "peak_sustained_at_sampled_clock": scaled,
+            "frac_vs_sustained_at_sampled_clock": (achieved / scaled) if scaled else None,
+            "sustained_peak_note": f"{src} bf16_tflops_sustained {sus} taken at {sus_mhz:.0f} MHz, scaled by the "
+                                   f"median SM clock sampled in this run ({sm_mhz} MHz)"}
 
 
 # ---------------------------------------------------------------------------
@@ -208,23 +249,67 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_sample(shape: bi.LayerShape, inp: dict, budget_s: float = 10.0, max_rows: int | None = None):
-    """Time the oracle on the first n rows of sequence 0 (n doubled until the
-    budget is spent). Returns (tokens/s, rows, seconds)."""
-    import oracle
-    args = bi.oracle_args(inp)
-    n = 64
-    cap = min(shape.s, max_rows or shape.s)
-    best = None
-    while True:
-        rows = np.arange(min(n, cap), dtype=np.int64)
+def spread_rows(s: int, n: int, offset: int = 0) -> np.ndarray:
+    """n query positions spread evenly over [0, s), the last one always s - 1
+    (so the oracle projects the keys/values of the whole sequence)."""
+    n = max(1, min(n, s))
+    idx = (np.arange(n, dtype=np.int64) * s) // n + (offset % max(1, s // n))
+    idx = np.minimum(idx, s - 1)
+    idx[-1] = s - 1
+    return np.unique(idx)
+
+
+class OracleTimer:
+    """Time of the fp64 oracle on one whole layer forward of a workload,
+    extrapolated from rows spread over the sequence.
+
+    The oracle's row function (layer_rows) costs a fixed part, the key/value
+    projection of the visible prefix (the whole sequence once the last row is
+    asked for), plus a part per row (its query projection, its attention over
+    its visible keys, the output projection and the FFN). A calibration call on
+    the last row alone gives fixed + one row; a call on n rows spread evenly
+    over the sequence (their causal prefixes average s/2, as over all rows)
+    gives fixed + n rows; the whole forward of one sequence is then
+    fixed + s rows, and b sequences take b times that."""
+
+    def __init__(self, shape: bi.LayerShape, inp: dict):
+        import oracle
+        self.oracle = oracle
+        self.shape = shape
+        self.args = bi.oracle_args(inp)
+        self.t_one = self._time(np.array([shape.s - 1], dtype=np.int64))
+
+    def _time(self, rows: np.ndarray) -> float:
         t0 = time.perf_counter()
-        oracle.layer_rows(*args, heads=shape.heads, causal=shape.causal, rows=rows)
-        dt = time.perf_counter() - t0
-        best = (rows.size / dt, int(rows.size), dt)
-        if dt >= budget_s or rows.size >= cap:
-            return best
-        n = min(cap, max(n * 2, int(n * budget_s / max(dt, 1e-3) * 0.6)))
+        self.oracle.layer_rows(*self.args, heads=self.shape.heads, causal=self.shape.causal, rows=rows)
+        return time.perf_counter() - t0
+
+    def rows_for_budget(self, budget_s: float) -> int:
+        """How many spread rows take about budget_s beyond the fixed part."""
+        probe = spread_rows(self.shape.s, 32)
+        per_row = max((self._time(probe) - self.t_one) / max(1, probe.size - 1), 1e-6)
+        return int(max(2, min(self.shape.s, budget_s / per_row)))
+
+    def sample(self, n: int, offset: int = 0):
+        """(tokens/s of the whole forward, rows timed, seconds spent, est. seconds of one forward)."""
+        s = self.shape.s
+        rows = spread_rows(s, n, offset)
+        t_n = self._time(rows)
+        if rows.size >= s:
+            t_seq = t_n
+        else:
+            per_row = max(t_n - self.t_one, 0.0) / max(1, rows.size - 1)
+            t_seq = self.t_one + (s - 1) * per_row
+        t_full = self.shape.b * t_seq
+        return self.shape.b * s / t_full, int(rows.size), t_n, t_full
+
+
+def sample_text(timer: OracleTimer, rows: int) -> str:
+    s = timer.shape.s
+    return (f"fp64 numpy/BLAS oracle (layer_rows) on {rows} query rows spread evenly over sequence 0 (s={s}, "
+            f"incl. row {s - 1}, so the whole key/value projection), after a calibration call on row {s - 1} "
+            f"alone ({timer.t_one:.2f} s); the whole forward of all {timer.shape.b} sequence(s) is extrapolated "
+            f"as b * (fixed + s * per-row)")
 
 
 def reference_arm(args, shape, name):
@@ -232,24 +317,25 @@ def reference_arm(args, shape, name):
     if rank != 0:
         return 0
     inp = bi.make_inputs(shape, seed=0)
-    per_step = []
+    # warm-up: the oracle on a short prefix (its threads and BLAS come up)
     for _ in range(args.warmup):
-        oracle_sample(shape, inp, budget_s=2.0, max_rows=256)
-    for _ in range(args.steps):
-        per_step.append(oracle_sample(shape, inp, budget_s=args.ref_budget))
+        import oracle
+        oracle.layer_rows(*bi.oracle_args(inp), heads=shape.heads, causal=shape.causal,
+                          rows=np.arange(min(shape.s, 64), dtype=np.int64))
+    timer = OracleTimer(shape, inp)
+    n = timer.rows_for_budget(args.ref_budget)
+    per_step = [timer.sample(n, offset=i) for i in range(args.steps)]
     tps = float(np.mean([p[0] for p in per_step]))
-    rows = per_step[-1][1]
     secs = float(sum(p[2] for p in per_step))
     cores = blas_threads()
-    sample = (f"oracle rows t=0..{rows - 1} of sequence 0 (their keys/values projected), fp64 numpy/BLAS; "
-              f"early causal rows attend to short prefixes, so this favours the CPU")
     line = {
         "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([p[3] for p in per_step])) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases)",
         "config": config_of(shape, name),
-        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample_text(timer, per_step[-1][1]) + f"; {secs:.1f} s timed over the steps"},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -260,8 +346,11 @@ def config_of(shape: bi.LayerShape, name: str) -> dict:
     return {"workload": name, "batch": shape.b, "seq_len": shape.s, "d_model": shape.h, "heads": shape.heads,
             "head_dim": shape.dh, "ffn_hidden": shape.f, "causal": shape.causal, "q_block": shape.q_block,
             "kv_block": shape.kv_block, "input_dtype": shape.dtype,
+            "block_sizes": "q_block sets the FFN wave (a whole number of query blocks); kv_block is validated but "
+                           "does not change the GPU schedule (attention tiles keys by 128)",
             "l2": "inputs larger than L2 (x, K/V and weights each exceed 126 MB)"
-            if shape.b * shape.s * shape.h * 2 > L2_BYTES else "L2 flushed between steps",
+            if shape.b * shape.s * shape.h * 2 > L2_BYTES else
+            "L2 flushed between steps (a 252 MB write, outside each step's event pair)",
             "parallelism": "independent sequences per GPU"}
 
 
@@ -269,80 +358,165 @@ def config_of(shape: bi.LayerShape, name: str) -> dict:
 # our arm
 # ---------------------------------------------------------------------------
 
+class Layer:
+    """Device-resident inputs of one workload and the call that runs it."""
+
+    def __init__(self, shape: bi.LayerShape, seed: int, device, inp: dict | None = None):
+        import torch
+        import blockwise_attn_ffn_bpt_b200 as bpt
+        self.bpt = bpt
+        self.shape = shape
+        self.inp = inp if inp is not None else bi.make_inputs(shape, seed=seed)
+        self.x = bi.to_torch(self.inp["x"], device)
+        self.params = {k: bi.to_torch(self.inp[k], device) for k in bi.PARAM_NAMES}
+        self.out = torch.empty((shape.b, shape.s, shape.h), dtype=torch.float32, device=device)
+        self.flush = None
+        if shape.b * shape.s * shape.h * 2 <= L2_BYTES:
+            self.flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    def run(self, stream):
+        sh = self.shape
+        self.bpt.layer_forward(self.x, self.params, sh.heads, sh.q_block, sh.kv_block, sh.causal, out=self.out,
+                               stream=stream)
+
+    def timed_steps(self, steps: int, stream) -> float:
+        """Device milliseconds of `steps` layer forwards: each forward between
+        its own pair of CUDA events on the launching stream (an L2 flush, when
+        the inputs fit in L2, runs between the pairs and is not counted)."""
+        import torch
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            if self.flush is not None:
+                self.flush.zero_()
+            e0.record(stream)
+            self.run(stream)
+            e1.record(stream)
+        torch.cuda.synchronize(stream.device)
+        return float(sum(e0.elapsed_time(e1) for e0, e1 in evs))
+
+
+def gpu_index(local: int) -> int:
+    if "CUDA_VISIBLE_DEVICES" in os.environ:
+        return int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    return local
+
+
+def kernel_split(layer: Layer, steps: int, stream) -> dict:
+    """Per-kernel device time over `steps` forwards, in a pass of its own with
+    the library's per-launch CUDA-event log on (never the headline pass)."""
+    bpt = layer.bpt
+    bpt.set_kernel_timing(True)
+    bpt.kernel_times()
+    for _ in range(steps):
+        if layer.flush is not None:
+            layer.flush.zero_()
+        layer.run(stream)
+    kt = bpt.kernel_times()
+    bpt.set_kernel_timing(False)
+    return kt
+
+
+def measure(args, shape: bi.LayerShape, name: str, layer: Layer, device, dist, steps: int) -> dict:
+    """Headline timing of one workload: warm-up, then `steps` forwards timed
+    with the kernel log off, barrier + sync on both sides, max over ranks;
+    clocks sampled during the timed region; then the per-kernel split in a
+    second pass."""
+    import torch
+    bpt = layer.bpt
+    world, rank, local = dist_env()
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        layer.run(stream)
+    if bpt.stream_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    launches0 = bpt.launch_count()
+    with ClockSampler(gpu_index(local)) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        ms = layer.timed_steps(steps, stream)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+    launches = bpt.launch_count() - launches0
+    if bpt.stream_status(stream) != 0:
+        raise RuntimeError("device error during the timed region")
+    ms_max = max_over_ranks(ms, dist, device)
+    ksteps = max(1, min(steps, 10))
+    ktimes = kernel_split(layer, ksteps, stream)
+    if bpt.stream_status(stream) != 0:
+        raise RuntimeError("device error during the kernel-split pass")
+    flops = layer_flops(shape)
+    clk = clocks.summary()
+    peaks, src = measured_peaks()
+    tokens = shape.b * shape.s
+    value = whole_job_throughput(tokens, steps, world, ms_max)
+    tflops = sum(flops.values()) * steps * world / (ms_max / 1e3) / 1e12
+    total_k = sum(v[1] for v in ktimes.values()) or 1.0
+    kernels = {}
+    for k, (n, t) in ktimes.items():
+        kf = flops.get(k, 0.0) * ksteps
+        kernels[k] = {"launches": n, "ms": t, "share": t / total_k, "avg_launch_ms": t / n,
+                      "tflops": (kf / (t / 1e3) / 1e12) if (kf and t > 0) else None}
+    roof = None
+    if ktimes:
+        kname = max(ktimes.items(), key=lambda kv: kv[1][1])[0]
+        kn, kms = ktimes[kname]
+        achieved = flops.get(kname, 0.0) * ksteps / (kms / 1e3) / 1e12 if kms > 0 else 0.0
+        roof = tensor_roofline(kname, achieved, peaks, src, clk.get("sm_mhz"), profiled_traffic(name, kname))
+        roof.update({"launches": kn, "avg_launch_ms": kms / kn,
+                     "timing": f"per-launch CUDA events on the launching stream, in a separate pass of {ksteps} "
+                               f"forwards after the headline pass"})
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32-in/bf16-mma",
+        "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases; random-init layer)",
+        "config": config_of(shape, name),
+        "tflops": tflops, "frac_of_bf16_peak": tflops / float(peaks["bf16_tflops"]),
+        "peak_source": f"{src} bf16_tflops (burst)",
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "kernels": kernels,
+        "kernels_pass": f"separate pass of {ksteps} forwards with per-launch CUDA events",
+        "clocks": clk,
+    }
+
+
 def our_arm(args, shape, name):
     import torch
-
-    import blockwise_attn_ffn_bpt_b200 as bpt
 
     world, rank, local = dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist = init_dist("nccl", world)
-
-    inp = bi.make_inputs(shape, seed=rank_seed(rank))
-    x = bi.to_torch(inp["x"], device)
-    params = {k: bi.to_torch(inp[k], device) for k in bi.PARAM_NAMES}
-    out = torch.empty((shape.b, shape.s, shape.h), dtype=torch.float32, device=device)
+    layer = Layer(shape, rank_seed(rank), device)
+    bpt = layer.bpt
     dtype_code = bpt.BPT_DTYPE_F32 if shape.dtype == "f32" else bpt.BPT_DTYPE_BF16
     ws_bytes = bpt.workspace_bytes(dtype_code, shape.b, shape.s, shape.h, shape.heads, shape.q_block,
                                    shape.kv_block)
-    flush = None
-    if shape.b * shape.s * shape.h * 2 <= L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step():
-        if flush is not None:
-            flush.zero_()
-        bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal, out=out,
-                          stream=stream)
-
     # device memory the library takes (its pool keeps the workspace between
-    # calls): free memory before the first call minus free memory after warm-up
+    # calls): free memory before the first call minus free memory after it
     torch.cuda.synchronize(device)
     free_pre, _ = torch.cuda.mem_get_info(device)
-    for _ in range(args.warmup):
-        step()
+    layer.run(stream)
     torch.cuda.synchronize(device)
-    if bpt.device_status() != 0:
-        raise RuntimeError("device error during warm-up")
     free_post, _ = torch.cuda.mem_get_info(device)
-
-    # ---- timed region (device time, CUDA events on the launching stream)
     torch.cuda.reset_peak_memory_stats(device)
     mem0 = torch.cuda.memory_allocated(device)
-    free0, _ = torch.cuda.mem_get_info(device)
-    bpt.set_kernel_timing(True)
-    bpt.kernel_times()
-    launches0 = bpt.launch_count()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                      int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])) as clocks:
-        barrier(dist, device)
-        torch.cuda.synchronize(device)
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(dist, device)
-    launches = bpt.launch_count() - launches0
-    ktimes = bpt.kernel_times()
-    bpt.set_kernel_timing(False)
-    if bpt.device_status() != 0:
-        raise RuntimeError("device error during the timed region")
-    ms = ev0.elapsed_time(ev1)
-    ms_max = max_over_ranks(ms, dist, device)
+
+    line = measure(args, shape, name, layer, device, dist, args.steps)
+    peak_bytes = torch.cuda.max_memory_allocated(device) - mem0
 
     # ---- end to end through the C ABI's host-memory entry (bpt_layer_forward_host):
     # every step copies its input from pinned host memory and its result back;
     # the library overlaps step i's copies with the compute of steps i -/+ 1
+    x, out = layer.x, layer.out
     x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     x_host.copy_(x)
     out_host = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
     torch.cuda.synchronize(device)
-    bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+    bpt.layer_forward_host(x_host, layer.params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
                            out_host=out_host, n_inputs=max(1, args.warmup // 2), stream=stream)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -350,21 +524,23 @@ def our_arm(args, shape, name):
     torch.cuda.synchronize(device)
     e2e_steps = max(1, args.steps)
     e0.record(stream)
-    bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
+    bpt.layer_forward_host(x_host, layer.params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
                            out_host=out_host, n_inputs=e2e_steps, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier(dist, device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    if bpt.stream_status(stream) != 0:
+        raise RuntimeError("device error during the end-to-end pass")
 
-    peak_bytes = torch.cuda.max_memory_allocated(device) - mem0
-
-    # ---- CPU baseline (rank 0, N = 1 only)
+    # ---- CPU baseline (rank 0, N = 1 only): the oracle as it stands
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, rows, secs = oracle_sample(shape, inp, budget_s=args.ref_budget)
+        timer = OracleTimer(shape, layer.inp)
+        n = timer.rows_for_budget(args.ref_budget)
+        tps, rows, secs, _ = timer.sample(n)
         cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"first {rows} rows of sequence 0 with their keys/values, fp64 numpy/BLAS, {secs:.1f} s"}
+               "sample": sample_text(timer, rows) + f"; {secs:.1f} s for the spread rows"}
 
     if dist is not None:
         barrier(dist, device)
@@ -374,53 +550,60 @@ def our_arm(args, shape, name):
         return 0
 
     tokens = shape.b * shape.s
-    flops = layer_flops(shape)
-    total_flops = sum(flops.values())
-    value = whole_job_throughput(tokens, args.steps, world, ms_max)
-    tflops = total_flops * args.steps * world / (ms_max / 1e3) / 1e12
-    peaks, peak_src = measured_peaks()
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-
-    # dominant kernel: largest share of the timed kernel time
-    dom = max(ktimes.items(), key=lambda kv: kv[1][1]) if ktimes else None
-    roof = None
-    if dom is not None:
-        kname, (nl, kms) = dom
-        kflops = flops.get(kname, 0.0) * args.steps
-        achieved = kflops / (kms / 1e3) / 1e12 if kms > 0 else 0.0
-        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(name, kname), "launches": nl,
-                "avg_launch_ms": kms / nl,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"}
-    kernel_table = {k: {"launches": n, "ms": t, "share": t / sum(v[1] for v in ktimes.values())}
-                    for k, (n, t) in ktimes.items()}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases; random-init layer)",
-        "config": config_of(shape, name),
-        "tflops": tflops, "frac_of_bf16_peak": tflops / peak,
-        "roofline": roof,
-        "cpu_baseline": cpu,
-        "e2e": {"value": tokens * e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
-                "d2h_bytes_per_step": int(out.numel() * out.element_size()),
-                "steps": e2e_steps, "api": "bpt_layer_forward_host (pinned host buffers)"},
-        "gpu_launches": int(launches),
-        "kernels": kernel_table,
-        "clocks": clocks.summary(),
-        "memory": {"workspace_bytes": ws_bytes, "ratio_bytes_vs_2bsh": ws_bytes / (2 * tokens * shape.h),
-                   "ratio_elems_vs_2bsh": ws_bytes / 2 / (2 * tokens * shape.h),
-                   "peak_torch_alloc_bytes_in_step": int(peak_bytes),
-                   "device_bytes_taken_by_library": int(free_pre - free_post),
-                   "free_bytes_before": int(free0)},
+    line["cpu_baseline"] = cpu
+    line["e2e"] = {"value": tokens * e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                   "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+                   "steps": e2e_steps, "api": "bpt_layer_forward_host (pinned host buffers)"}
+    two_bsh_bytes = 2 * tokens * shape.h
+    line["memory"] = {
+        "workspace_bytes": ws_bytes, "ratio_bytes_vs_2bsh": ws_bytes / two_bsh_bytes,
+        "ratio_elems_vs_2bsh": ws_bytes / 2 / two_bsh_bytes,
+        "reading": "target: 2bsh read as elements (<= 1.5x); read as bf16 bytes the bound is not met (2.0x), "
+                   "which is inherent to materialising K and V (Algorithm 1 step 1: 4bsh bytes)",
+        "peak_torch_alloc_bytes_in_step": int(peak_bytes),
+        "device_bytes_taken_by_library": int(free_pre - free_post),
     }
     print(json.dumps(line))
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def all_configs_arm(args):
+    """One JSON line per configuration of the layer's workloads (the four
+    fixed workloads and every point of the block-size sweep, causal and not):
+    device time, tokens/s, TFLOP/s, fraction of the bf16 peak, kernel split,
+    SM clock. One GPU; no e2e or CPU legs."""
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    names = list(bi.WORKLOADS) + [f"sweep_{blk}_{c}" for c in ("causal", "noncausal") for blk in bi.SWEEP_BLOCKS]
+    if args.only:
+        names = [n for n in names if any(o in n for o in args.only.split(","))]
+    cache = {}
+    for name in names:
+        shape = shape_of(name)
+        key = ("sweep", shape.causal) if name.startswith("sweep_") else name
+        if key not in cache:
+            cache.clear()
+            cache[key] = bi.make_inputs(shape, seed=0)
+        layer = Layer(shape, 0, device, inp=cache[key])
+        steps = args.steps if shape.s * shape.b >= 32768 else max(args.steps, 20)
+        line = measure(args, shape, name, layer, device, None, steps)
+        line["cpu_baseline"] = None
+        line["e2e"] = None
+        print(json.dumps(line), flush=True)
+        del layer
+        torch.cuda.empty_cache()
+    return 0
+
+
+def shape_of(name: str) -> bi.LayerShape:
+    if name.startswith("sweep_"):
+        _, blk, c = name.split("_")
+        return bi.sweep_shape(int(blk), c == "causal")
+    return bi.WORKLOADS[name]
 
 
 def largest_fitting(need, budget: int, unit: int) -> int:
@@ -488,7 +671,7 @@ def max_context_arm(args):
         torch.cuda.synchronize(device)
     ms = ev0.elapsed_time(ev1)
     free_after, _ = torch.cuda.mem_get_info(device)
-    status = bpt.device_status()
+    status = bpt.stream_status(stream)
     # oracle check of the first rows, and finiteness of rows spread over the sequence
     R = 256
     p64 = {k: v.float().cpu().numpy().astype(np.float64) for k, v in params.items()}
@@ -527,21 +710,22 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="one of: " + ", ".join(list(bi.WORKLOADS) + ["sweep_<block>_<causal|noncausal>"]))
-    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per sample")
+    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work per sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--max-context", action="store_true",
                     help="instead: the longest sequence one 7B-class layer forward fits on the GPU, run once")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="instead: one line per workload and block-size sweep point (one GPU)")
+    ap.add_argument("--only", default="", help="with --all-configs: comma-separated name fragments to keep")
     args = ap.parse_args(argv)
     if args.max_context:
         return max_context_arm(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.all_configs:
+        return all_configs_arm(args)
     name = args.workload
-    if name.startswith("sweep_"):
-        _, blk, c = name.split("_")
-        shape = bi.sweep_shape(int(blk), c == "causal")
-    else:
-        shape = bi.WORKLOADS[name]
+    shape = shape_of(name)
     world, _, _ = dist_env()
     if world != args.gpus:
         print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)

@@ -7,6 +7,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -110,3 +111,52 @@ def test_largest_fitting_length_is_the_largest_that_fits(unit):
             assert need(s) <= budget < need(s + unit)
         else:
             assert s == unit  # nothing fits: the smallest length is reported
+
+
+def test_spread_rows_cover_the_sequence_and_end_on_its_last_row():
+    for s, n in [(256, 8), (32768, 100), (1000, 1), (64, 500), (5, 3)]:
+        r = bench.spread_rows(s, n)
+        assert r[-1] == s - 1 and r.min() >= 0 and np.all(np.diff(r) > 0)
+        assert r.size == min(n, s) or r.size == min(n, s) - 1  # the last slot moved onto s - 1
+        if n < s:
+            # evenly spread: the mean position is near the middle, so causal
+            # rows average a prefix of about s/2
+            assert abs(r.mean() - (s - 1) / 2) <= s / n + 1
+
+
+def test_oracle_timer_extrapolates_a_whole_forward():
+    import bpt_inputs as bi
+    shape = bi.LayerShape(2, 128, 128, 2, 64, 64, True)
+    inp = bi.make_inputs(shape, seed=0)
+    timer = bench.OracleTimer(shape, inp)
+    assert timer.t_one > 0
+    tps, rows, secs, t_full = timer.sample(16)
+    assert rows == 16 and secs > 0 and t_full > 0
+    assert tps == pytest.approx(shape.b * shape.s / t_full)
+    # asking for every row times the whole sequence directly
+    tps_all, rows_all, secs_all, t_all = timer.sample(10_000)
+    assert rows_all == shape.s and t_all == pytest.approx(shape.b * secs_all)
+
+
+def test_traffic_comes_from_the_data_file_only_while_the_source_matches(tmp_path):
+    p = tmp_path / "traffic.json"
+    good = {"kernel_source_sha256_16": bench.kernel_source_hash(), "traffic_per_launch_bytes": {"w": 123}}
+    p.write_text(json.dumps(good))
+    assert bench.profiled_traffic("w", "attention", str(p)) == 123
+    assert bench.profiled_traffic("other", "attention", str(p)) is None
+    assert bench.profiled_traffic("w", "gemm_qkv", str(p)) is None
+    p.write_text(json.dumps(dict(good, kernel_source_sha256_16="0" * 16)))
+    assert bench.profiled_traffic("w", "attention", str(p)) is None
+    assert bench.profiled_traffic("w", "attention", str(tmp_path / "missing.json")) is None
+
+
+def test_roofline_frac_is_against_the_burst_peak():
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1300.0, "bf16_tflops_sustained_sm_mhz": 1300.0}
+    r = bench.tensor_roofline("attention", 1000.0, peaks, "measured", 1950.0, None)
+    assert r["peak"] == 1600.0 and r["frac"] == pytest.approx(1000.0 / 1600.0)
+    # the sustained figure scaled to the sampled clock
+    assert r["peak_sustained_at_sampled_clock"] == pytest.approx(1300.0 * 1950.0 / 1300.0)
+    assert r["frac_vs_sustained_at_sampled_clock"] == pytest.approx(1000.0 / 1950.0)
+    # without a clock key the fallback's clock is used
+    assert bench.sustained_clock_mhz({"bf16_tflops": 1.0}) == bench.FALLBACK_PEAKS["bf16_tflops_sustained_sm_mhz"]
+    assert bench.sustained_clock_mhz({"x": {"sustained_clock_mhz": 1234}}) == 1234.0

@@ -63,7 +63,7 @@ def run_layer(shape, inp, wave_rows=0, workspace=False):
         out = bpt.layer_forward(x, params, shape.heads, shape.q_block, shape.kv_block, shape.causal,
                                 wave_rows=wave_rows)
     torch.cuda.synchronize()
-    assert bpt.device_status() == 0
+    assert bpt.stream_status() == 0
     return out.cpu().numpy()
 
 
@@ -201,7 +201,7 @@ def test_host_entry_equals_the_device_path(dtype):
     xs = [bi.to_torch(i["x"], device="cpu") for i in inps]
     x_host = torch.stack(xs).pin_memory()
     got = bpt.layer_forward_host(x_host, params, shape.heads, shape.q_block, shape.kv_block, shape.causal)
-    assert bpt.device_status() == 0
+    assert bpt.stream_status() == 0
     for k in range(3):
         ref = bpt.layer_forward(xs[k].cuda(), params, shape.heads, shape.q_block, shape.kv_block, shape.causal)
         torch.cuda.synchronize()
@@ -234,7 +234,7 @@ def test_two_layer_stack_matches_the_oracle_applied_twice():
     x2 = bpt.convert_f32_to_bf16(y1).view(x.shape)
     y2 = bpt.layer_forward(x2, d2, s1.heads, s1.q_block, s1.kv_block, s1.causal)
     torch.cuda.synchronize()
-    assert bpt.device_status() == 0
+    assert bpt.stream_status() == 0
     assert torch.equal(got, y2)
     # layer 2 on that bf16 input is the oracle's layer (the usual bound)
     x2_64 = x2.float().cpu().numpy().astype(np.float64)
@@ -336,15 +336,29 @@ def test_workload_causal_b2_s2048_full():
     assert_parity(got, ref, "b2 s2048 h1024 causal")
 
 
-@pytest.mark.parametrize("name", ["gpt1b_s8192_h2048", "gpt7b_s32768_h4096"])
-def test_workload_full_size_sampled_rows(name):
-    shape = bi.WORKLOADS[name]
+def test_workload_gpt1b_s8192_every_row():
+    # the 1B-class workload (s = 8192, h = 2048, causal) compared on every row
+    shape = bi.WORKLOADS["gpt1b_s8192_h2048"]
+    inp = bi.make_inputs(shape, seed=0)
+    got = run_layer(shape, inp)
+    assert_parity(got, oracle_full(shape, inp), "gpt1b s8192 h2048, every row")
+
+
+def test_workload_gpt7b_s32768_first_and_last_query_blocks_and_sampled_rows():
+    # the 7B-class workload: every row of the first and of the last query
+    # block (rows 31744-32767 attend to the longest prefixes, where the running
+    # max has moved most), plus rows spread over every other query block
+    shape = bi.WORKLOADS["gpt7b_s32768_h4096"]
     inp = bi.make_inputs(shape, seed=0)
     got = run_layer(shape, inp)
     assert np.isfinite(got).all()
-    rows = sample_rows(shape)
+    qb = shape.q_block
+    rows = np.unique(np.concatenate([np.arange(qb), np.arange(shape.s - qb, shape.s), sample_rows(shape)]))
     ref = oracle.layer_rows(*bi.oracle_args(inp), heads=shape.heads, causal=shape.causal, rows=rows)
-    assert_parity(got.reshape(-1, shape.h)[rows], ref, name)
+    flat = got.reshape(-1, shape.h)
+    assert_parity(flat[:qb], ref[:qb], "gpt7b first query block")
+    assert_parity(flat[shape.s - qb:], ref[-qb:], "gpt7b last query block")
+    assert_parity(flat[rows], ref, "gpt7b first, last and sampled rows")
 
 
 @pytest.mark.parametrize("causal", [True, False])
@@ -362,3 +376,7 @@ def test_block_size_sweep_sampled_rows(causal):
     # every block size computes the same layer
     for o in outs[1:]:
         assert np.abs(o - outs[0]).max() <= MAX_ABS
+    # and one sweep point (q_block = kv_block = 2048) on every row
+    assert shapes[-1].q_block == 2048
+    full = oracle_full(shapes[-1], inp).reshape(-1, shapes[-1].h)
+    assert_parity(outs[-1], full, f"sweep block 2048 causal={causal}, every row")

@@ -41,16 +41,24 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------
 
 def layer_flops(shape: bi.LayerShape) -> dict:
-    b, s, h = shape.b, shape.s, shape.h
+    """Matmul flops of one forward per kernel name of the library's timing log
+    (ffn_chain runs the three FFN-side GEMMs in one launch)."""
+    b, s, h, f = shape.b, shape.s, shape.h, shape.f
     tok = b * s
     att = 4.0 * b * s * s * h * (0.5 if shape.causal else 1.0)
     return {
         "gemm_qkv": 2.0 * tok * h * 3 * h,
         "attention": att,
         "gemm_outproj": 2.0 * tok * h * h,
-        "gemm_ffn_up": 2.0 * tok * h * 4 * h,
-        "gemm_ffn_down": 2.0 * tok * 4 * h * h,
+        "gemm_ffn_up": 2.0 * tok * h * f,
+        "gemm_ffn_down": 2.0 * tok * f * h,
     }
+
+
+def kernel_flops(shape: bi.LayerShape) -> dict:
+    f = layer_flops(shape)
+    f["ffn_chain"] = f["gemm_outproj"] + f["gemm_ffn_up"] + f["gemm_ffn_down"]
+    return f
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
@@ -265,35 +273,48 @@ class OracleTimer:
 
     The oracle's row function (layer_rows) costs a fixed part, the key/value
     projection of the visible prefix (the whole sequence once the last row is
-    asked for), plus a part per row (its query projection, its attention over
-    its visible keys, the output projection and the FFN). A calibration call on
-    the last row alone gives fixed + one row; a call on n rows spread evenly
-    over the sequence (their causal prefixes average s/2, as over all rows)
-    gives fixed + n rows; the whole forward of one sequence is then
-    fixed + s rows, and b sequences take b times that."""
+    asked for), plus a part per row (its query projection, its scores against
+    every projected key with the invisible ones masked, the output projection
+    and the FFN), as its plain whole-sequence forward does. A calibration call
+    on the last row alone (after one untimed warm-up call) gives fixed + one
+    row; a call on n rows spread evenly over the sequence gives fixed + n rows;
+    the whole forward of one sequence is then fixed + s rows, and b sequences
+    take b times that."""
 
     def __init__(self, shape: bi.LayerShape, inp: dict):
         import oracle
         self.oracle = oracle
         self.shape = shape
         self.args = bi.oracle_args(inp)
-        self.t_one = self._time(np.array([shape.s - 1], dtype=np.int64))
+        last = np.array([shape.s - 1], dtype=np.int64)
+        self._time(last)  # warm-up: BLAS threads, page faults of the fp64 copies
+        self.t_one = self._time(last)
 
     def _time(self, rows: np.ndarray) -> float:
         t0 = time.perf_counter()
         self.oracle.layer_rows(*self.args, heads=self.shape.heads, causal=self.shape.causal, rows=rows)
         return time.perf_counter() - t0
 
+    # host memory the oracle's score matrices of one call may take: it holds,
+    # per head and worker thread, a few fp64 arrays of (rows x visible keys)
+    MEM_BUDGET = 4 << 30
+
+    def max_rows(self) -> int:
+        threads = max(1, min(self.shape.heads, os.cpu_count() or 1))
+        per_row = self.shape.s * 8 * 4 * threads
+        return int(max(2, min(self.shape.s, self.MEM_BUDGET // per_row)))
+
     def rows_for_budget(self, budget_s: float) -> int:
-        """How many spread rows take about budget_s beyond the fixed part."""
-        probe = spread_rows(self.shape.s, 32)
+        """How many spread rows take about budget_s beyond the fixed part
+        (never more than the memory bound allows)."""
+        probe = spread_rows(self.shape.s, min(64, self.max_rows()))
         per_row = max((self._time(probe) - self.t_one) / max(1, probe.size - 1), 1e-6)
-        return int(max(2, min(self.shape.s, budget_s / per_row)))
+        return int(max(2, min(self.max_rows(), budget_s / per_row)))
 
     def sample(self, n: int, offset: int = 0):
         """(tokens/s of the whole forward, rows timed, seconds spent, est. seconds of one forward)."""
         s = self.shape.s
-        rows = spread_rows(s, n, offset)
+        rows = spread_rows(s, min(n, self.max_rows()), offset)
         t_n = self._time(rows)
         if rows.size >= s:
             t_seq = t_n
@@ -445,6 +466,7 @@ def measure(args, shape: bi.LayerShape, name: str, layer: Layer, device, dist, s
     if bpt.stream_status(stream) != 0:
         raise RuntimeError("device error during the kernel-split pass")
     flops = layer_flops(shape)
+    kflops = kernel_flops(shape)
     clk = clocks.summary()
     peaks, src = measured_peaks()
     tokens = shape.b * shape.s
@@ -453,14 +475,14 @@ def measure(args, shape: bi.LayerShape, name: str, layer: Layer, device, dist, s
     total_k = sum(v[1] for v in ktimes.values()) or 1.0
     kernels = {}
     for k, (n, t) in ktimes.items():
-        kf = flops.get(k, 0.0) * ksteps
+        kf = kflops.get(k, 0.0) * ksteps
         kernels[k] = {"launches": n, "ms": t, "share": t / total_k, "avg_launch_ms": t / n,
                       "tflops": (kf / (t / 1e3) / 1e12) if (kf and t > 0) else None}
     roof = None
     if ktimes:
         kname = max(ktimes.items(), key=lambda kv: kv[1][1])[0]
         kn, kms = ktimes[kname]
-        achieved = flops.get(kname, 0.0) * ksteps / (kms / 1e3) / 1e12 if kms > 0 else 0.0
+        achieved = kflops.get(kname, 0.0) * ksteps / (kms / 1e3) / 1e12 if kms > 0 else 0.0
         roof = tensor_roofline(kname, achieved, peaks, src, clk.get("sm_mhz"), profiled_traffic(name, kname))
         roof.update({"launches": kn, "avg_launch_ms": kms / kn,
                      "timing": f"per-launch CUDA events on the launching stream, in a separate pass of {ksteps} "
@@ -710,7 +732,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="one of: " + ", ".join(list(bi.WORKLOADS) + ["sweep_<block>_<causal|noncausal>"]))
-    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work per sample")
+    ap.add_argument("--ref-budget", type=float, default=4.0, help="seconds of oracle work per sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--max-context", action="store_true",
                     help="instead: the longest sequence one 7B-class layer forward fits on the GPU, run once")

@@ -134,6 +134,7 @@ def test_oracle_timer_extrapolates_a_whole_forward():
     assert rows == 16 and secs > 0 and t_full > 0
     assert tps == pytest.approx(shape.b * shape.s / t_full)
     # asking for every row times the whole sequence directly
+    assert timer.max_rows() == shape.s  # a tiny problem is never memory-bound
     tps_all, rows_all, secs_all, t_all = timer.sample(10_000)
     assert rows_all == shape.s and t_all == pytest.approx(shape.b * secs_all)
 

@@ -33,6 +33,8 @@ import bpt_inputs as bi  # noqa: E402
 
 METRIC = "BPT layer fwd tokens/s and TFLOP/s (% BF16 peak) on 1 B200, vs fp64 oracle"
 DEFAULT_WORKLOAD = "gpt7b_s32768_h4096"
+# wave_rows values of the library's FFN-side schedules (BPT_WAVE_* in include/bpt.h)
+FFN_SCHEDULES = {"default": 0, "chained": -1, "waves": -2}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -382,11 +384,12 @@ def config_of(shape: bi.LayerShape, name: str) -> dict:
 class Layer:
     """Device-resident inputs of one workload and the call that runs it."""
 
-    def __init__(self, shape: bi.LayerShape, seed: int, device, inp: dict | None = None):
+    def __init__(self, shape: bi.LayerShape, seed: int, device, inp: dict | None = None, wave_rows: int = 0):
         import torch
         import blockwise_attn_ffn_bpt_b200 as bpt
         self.bpt = bpt
         self.shape = shape
+        self.wave_rows = wave_rows
         self.inp = inp if inp is not None else bi.make_inputs(shape, seed=seed)
         self.x = bi.to_torch(self.inp["x"], device)
         self.params = {k: bi.to_torch(self.inp[k], device) for k in bi.PARAM_NAMES}
@@ -398,7 +401,7 @@ class Layer:
     def run(self, stream):
         sh = self.shape
         self.bpt.layer_forward(self.x, self.params, sh.heads, sh.q_block, sh.kv_block, sh.causal, out=self.out,
-                               stream=stream)
+                               wave_rows=self.wave_rows, stream=stream)
 
     def timed_steps(self, steps: int, stream) -> float:
         """Device milliseconds of `steps` layer forwards: each forward between
@@ -492,7 +495,7 @@ def measure(args, shape: bi.LayerShape, name: str, layer: Layer, device, dist, s
         "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32-in/bf16-mma",
         "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights, N(0,0.02^2) biases; random-init layer)",
-        "config": config_of(shape, name),
+        "config": dict(config_of(shape, name), ffn_schedule=args.ffn),
         "tflops": tflops, "frac_of_bf16_peak": tflops / float(peaks["bf16_tflops"]),
         "peak_source": f"{src} bf16_tflops (burst)",
         "roofline": roof,
@@ -510,7 +513,7 @@ def our_arm(args, shape, name):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist = init_dist("nccl", world)
-    layer = Layer(shape, rank_seed(rank), device)
+    layer = Layer(shape, rank_seed(rank), device, wave_rows=FFN_SCHEDULES[args.ffn])
     bpt = layer.bpt
     dtype_code = bpt.BPT_DTYPE_F32 if shape.dtype == "f32" else bpt.BPT_DTYPE_BF16
     ws_bytes = bpt.workspace_bytes(dtype_code, shape.b, shape.s, shape.h, shape.heads, shape.q_block,
@@ -610,7 +613,7 @@ def all_configs_arm(args):
         if key not in cache:
             cache.clear()
             cache[key] = bi.make_inputs(shape, seed=0)
-        layer = Layer(shape, 0, device, inp=cache[key])
+        layer = Layer(shape, 0, device, inp=cache[key], wave_rows=FFN_SCHEDULES[args.ffn])
         steps = args.steps if shape.s * shape.b >= 32768 else max(args.steps, 20)
         line = measure(args, shape, name, layer, device, None, steps)
         line["cpu_baseline"] = None
@@ -739,6 +742,8 @@ def main(argv=None):
     ap.add_argument("--all-configs", action="store_true",
                     help="instead: one line per workload and block-size sweep point (one GPU)")
     ap.add_argument("--only", default="", help="with --all-configs: comma-separated name fragments to keep")
+    ap.add_argument("--ffn", choices=list(FFN_SCHEDULES), default="default",
+                    help="FFN-side schedule: the library's default, one chained launch, or per-GEMM waves")
     args = ap.parse_args(argv)
     if args.max_context:
         return max_context_arm(args)

@@ -319,21 +319,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m_new, -m_new);
       float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
+      auto exp_phase = [&]() {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-          const int i = 32 * half + i2;
-          const uint64_t x2 = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), sl2x2, negm2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
-          pk[i2] = pp;
-          add_bf16x2_to(pp, sum4[i & 3], sum4[(i + 2) & 3]);
+          for (int i2 = 0; i2 < 32; ++i2) {
+            const int i = 32 * half + i2;
+            const uint64_t x2 = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), sl2x2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+            pk[i2] = pp;
+            add_bf16x2_to(pp, sum4[i & 3], sum4[(i + 2) & 3]);
+          }
+          tmem_store32(tS + 32 * half, pk);
         }
-        tmem_store32(tS + 32 * half, pk);
-      }
+      };
+      exp_phase();
       // hand P to the MMA issuer
       tc_fence_before();
       __syncwarp();

@@ -30,6 +30,7 @@
 
 #include "attention.cuh"
 #include "bpt.h"
+#include "ffn_chain.cuh"
 #include "gemm.cuh"
 
 namespace bpt {
@@ -154,6 +155,8 @@ int check_device(int* sms) {
                                         GEMM_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_FFN_DOWN>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(ffn_chain_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GEMM_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         AttnCfg<64>::SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -366,7 +369,7 @@ int default_wave_rows(int b, int s, int h, int ffn, int q_block) {
 }
 
 int wave_rows_for(int b, int s, int h, int ffn, int q_block, int wave_rows) {
-  if (wave_rows <= 0) return default_wave_rows(b, s, h, ffn, q_block);
+  if (wave_rows <= 0) return default_wave_rows(b, s, h, ffn, q_block);  // BPT_WAVE_DEFAULT(_WAVES)
   long long wr = std::max<long long>(q_block, ((long long)wave_rows / q_block) * q_block);
   if (wr >= s) {
     const long long g = std::max<long long>(1, std::min<long long>(b, wr / s));
@@ -396,26 +399,85 @@ int for_each_wave(int b, int s, int h, int ffn, int q_block, int wave_rows, F&& 
   return BPT_OK;
 }
 
-// ------------------------------------------------------------- workspace layout
-// Region 0 holds K and V during the projection and attention, then the wave
-// scratch (hid, hb, U) of the FFN side; the f32 entry's bf16 copies of x and
-// the weights follow it.
-struct Layout {
-  size_t k, v, hid, hb, u, xb, wqkv, wo, w1, w2, total;
-  int wave_rows;
+// ------------------------------------------------------------- FFN chain plan
+// Groups of the one-launch FFN side (ffn_chain.cuh): the largest group of
+// 16, 8, 4, 2 or 1 M-tiles whose slots (fp32 hid, its bf16 copy, bf16 U) take
+// at most 1.5x the K/V bytes (or 32 MiB, for small problems); one M-tile
+// when none does. The slots alias the K/V region, dead once attention has
+// run, so the workspace is the larger of the two. Slots are 1 KB aligned.
+struct ChainPlan {
+  int m_tiles, gm, groups, hs, us;
+  size_t hid, hb, u, bytes;
 };
+
+ChainPlan chain_plan(int b, int s, int h, int ffn) {
+  const long long M = (long long)b * s;
+  const size_t kv = kv_bytes(b, s, h);
+  const size_t budget = std::max(kv / 2 * 3, (size_t)32 << 20);
+  ChainPlan p{};
+  p.m_tiles = (int)((M + GEMM_BM - 1) / GEMM_BM);
+  for (int gm = CHAIN_GROUP_MT; gm >= 1; gm /= 2) {
+    p.gm = gm;
+    p.groups = (p.m_tiles + gm - 1) / gm;
+    p.hs = std::min(CHAIN_HID_SLOTS, p.groups);
+    p.us = std::min(CHAIN_U_SLOTS, p.groups);
+    const size_t rows = (size_t)gm * GEMM_BM;
+    p.hid = 0;
+    p.hb = align_up((size_t)p.hs * rows * h * 4, 1024);
+    p.u = p.hb + align_up((size_t)p.hs * rows * h * 2, 1024);
+    p.bytes = p.u + align_up((size_t)p.us * rows * ffn * 2, 1024);
+    if (p.bytes <= budget) break;
+  }
+  return p;
+}
+
+// ------------------------------------------------------------- workspace layout
+// Region 0 holds K and V during the projection and attention, then the
+// scratch of the FFN side: the chain's group slots (default bf16 path) or one
+// wave's hid, hb and U (explicit wave size, fp32 inputs); the chain's
+// completion counters, then the f32 entry's bf16 copies of x and the weights
+// follow it.
+struct Layout {
+  size_t k, v, hid, hb, u, xb, wqkv, wo, w1, w2, cnt, total;
+  int wave_rows;
+  bool chain;
+  ChainPlan cp;
+};
+
+// wave_rows selects the FFN side's schedule: BPT_WAVE_CHAINED runs it in one
+// launch (bf16 inputs), BPT_WAVE_DEFAULT_WAVES and any positive size in one
+// launch per GEMM and wave, and BPT_WAVE_DEFAULT (0) takes kChainByDefault.
+// fp32 inputs (split products) always run per wave.
+constexpr bool kChainByDefault = false;
+bool use_chain(int dtype, int wave_rows) {
+  if (dtype != BPT_DTYPE_BF16) return false;
+  return wave_rows == BPT_WAVE_CHAINED || (wave_rows == BPT_WAVE_DEFAULT && kChainByDefault);
+}
 
 Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave_rows) {
   Layout L{};
   const size_t tok = (size_t)b * s;
-  const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
-  L.wave_rows = wr;
   L.k = 0;
   L.v = align_up(tok * h * 2, 1024);
-  L.hid = 0;
-  L.hb = align_up((size_t)wr * h * 4, 1024);
-  L.u = L.hb + align_up((size_t)wr * h * 2, 1024);
-  size_t off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h, ffn));
+  size_t off;
+  if (use_chain(dtype, wave_rows)) {
+    L.chain = true;
+    L.cp = chain_plan(b, s, h, ffn);
+    L.wave_rows = L.cp.gm * GEMM_BM;
+    L.hid = L.cp.hid;
+    L.hb = L.cp.hb;
+    L.u = L.cp.u;
+    off = std::max(kv_bytes(b, s, h), L.cp.bytes);
+    L.cnt = off;
+    off = align_up(off + 3 * (size_t)L.cp.groups * sizeof(unsigned), 1024);
+  } else {
+    const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
+    L.wave_rows = wr;
+    L.hid = 0;
+    L.hb = align_up((size_t)wr * h * 4, 1024);
+    L.u = L.hb + align_up((size_t)wr * h * 2, 1024);
+    off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h, ffn));
+  }
   auto take = [&](size_t bytes) {
     size_t at = off;
     off = align_up(off + bytes, 1024);
@@ -435,6 +497,10 @@ Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave
 }
 
 // ------------------------------------------------------------- launches
+struct LayerPtrs {
+  const void *x, *Wqkv, *bqkv, *Wo, *bo, *W1, *b1, *W2, *b2;
+};
+
 // A [M, a_cols] (row stride lda) times B [K, N]; with a_split != 0 the K
 // blocks of B pair with A's blocks as a_block() maps them (split products).
 template <int MODE>
@@ -497,6 +563,54 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
       attention_fwd_tcgen05<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);
     else
       attention_fwd_tcgen05<128><<<grid, ATT_THREADS, AttnCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+// The FFN side of every query block in one launch (ffn_chain.cuh): O (bf16
+// rows inside out, `ldq` elements apart) -> hid, U -> out.
+int launch_chain(const __nv_bfloat16* O, long long ldq, const LayerPtrs& p, long long M, int h, int ffn,
+                 const Layout& L, uint8_t* ws, float* out, int sms, cudaStream_t st, int* status) {
+  if (M <= 0) return BPT_OK;
+  const ChainPlan& cp = L.cp;
+  const long long rows = (long long)cp.gm * GEMM_BM;
+  ChainArgs a{};
+  a.M = M;
+  a.h = h;
+  a.f = ffn;
+  a.m_tiles = cp.m_tiles;
+  a.gm = cp.gm;
+  a.groups = cp.groups;
+  a.hid_slots = cp.hs;
+  a.u_slots = cp.us;
+  a.n_op = (h + GEMM_BN - 1) / GEMM_BN;
+  a.n_up = (ffn + GEMM_BN - 1) / GEMM_BN;
+  a.n_dn = a.n_op;
+  a.x = reinterpret_cast<const __nv_bfloat16*>(p.x);
+  a.bo = reinterpret_cast<const __nv_bfloat16*>(p.bo);
+  a.b1 = reinterpret_cast<const __nv_bfloat16*>(p.b1);
+  a.b2 = reinterpret_cast<const __nv_bfloat16*>(p.b2);
+  a.hid = reinterpret_cast<float*>(ws + L.hid);
+  a.hb = reinterpret_cast<__nv_bfloat16*>(ws + L.hb);
+  a.u = reinterpret_cast<__nv_bfloat16*>(ws + L.u);
+  a.out = out;
+  unsigned* cnt = reinterpret_cast<unsigned*>(ws + L.cnt);
+  a.op_cnt = cnt;
+  a.up_cnt = cnt + cp.groups;
+  a.dn_cnt = cnt + 2 * (size_t)cp.groups;
+  a.status = status;
+  CUtensorMap tO, tHb, tU, tWo, tW1, tW2;
+  if (!map_rows(&tO, O, M, h, ldq, GEMM_BM) || !map_rows(&tHb, a.hb, cp.hs * rows, h, h, GEMM_BM) ||
+      !map_rows(&tU, a.u, cp.us * rows, ffn, ffn, GEMM_BM) || !map_rows(&tWo, p.Wo, h, h, h, 64) ||
+      !map_rows(&tW1, p.W1, h, ffn, ffn, 64) || !map_rows(&tW2, p.W2, ffn, h, h, 64))
+    return BPT_ERR_CUDA;
+  if (cudaMemsetAsync(cnt, 0, 3 * (size_t)cp.groups * sizeof(unsigned), st) != cudaSuccess)
+    return BPT_ERR_CUDA;
+  const long long tiles = (long long)cp.m_tiles * (a.n_op + a.n_up + a.n_dn);
+  const int grid = (int)std::min<long long>(tiles, sms);
+  {
+    LaunchScope ls("ffn_chain", st);
+    ffn_chain_tcgen05<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(tO, tHb, tU, tWo, tW1, tW2, a);
   }
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
@@ -576,9 +690,6 @@ int launch_split_rows(const float* src, long long rows, int cols, void* dst, int
     if (_r != BPT_OK) return _r; \
   } while (0)
 
-struct LayerPtrs {
-  const void *x, *Wqkv, *bqkv, *Wo, *bo, *W1, *b1, *W2, *b2;
-};
 
 // FFN width: a positive multiple of 64 (one K step of the GEMMs, one TMA box)
 int check_ffn(int ffn) { return (ffn <= 0 || ffn % 64) ? BPT_ERR_SHAPE : BPT_OK; }
@@ -666,7 +777,8 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   // own rows and head with their attention output
   BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st, status));
 
-  // step 11 per wave of query blocks: out-projection, residuals and FFN
+  // step 11 for every query block: out-projection, residuals and FFN
+  if (L.chain) return launch_chain(QO, ldq, p, tok, h, ffn, L, ws, out, sms, st, status);
   return for_each_wave(b, s, h, ffn, q_block, wave_rows, [&](const Wave& w) -> int {
     const long long rows = w.rows();
     GemmArgs a{};

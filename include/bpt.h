@@ -40,9 +40,10 @@
  *   dh in {64, 128}, b*s <= 2^31 - 1. The FFN width is fixed at 4h.
  * - Blocks: 1 <= q_block <= s, 1 <= kv_block <= s, s % q_block == 0,
  *   s % kv_block == 0 (equal-length blocks). The result does not depend on the
- *   block sizes (the blockwise computation is exact); q_block sets the rows of
- *   each FFN wave, which is a whole number of query blocks (or of whole
- *   sequences).
+ *   block sizes (the blockwise computation is exact). The kernels tile by the
+ *   hardware instead: attention by 128 query rows x 128 keys, the FFN side by
+ *   waves of whole query blocks (or, on request, by groups of 128-row tiles
+ *   that all run in one launch: BPT_WAVE_CHAINED).
  * - causal != 0: key u is visible to query t iff u <= t in the same sequence.
  * - Pointers must be 16-byte aligned (tensor-memory-access tiles).
  * - Errors: argument errors return a negative bpt_status synchronously, with
@@ -83,6 +84,13 @@ typedef enum bpt_dtype {
   BPT_DTYPE_BF16 = 0,
   BPT_DTYPE_F32 = 1
 } bpt_dtype;
+
+/* Schedules of the FFN side (the wave_rows argument of the _ws and _ffn entry
+ * points and of bpt_layer_workspace_bytes(_ffn)); any positive value is an
+ * explicit wave of that many rows, one launch per GEMM and wave. */
+#define BPT_WAVE_DEFAULT 0         /* the library's choice (per-GEMM waves) */
+#define BPT_WAVE_CHAINED (-1)      /* every query block's FFN side in one launch (bf16 inputs) */
+#define BPT_WAVE_DEFAULT_WAVES (-2) /* one launch per GEMM and wave, waves of the library's default size */
 
 /* Human-readable name of a status code (static string, never NULL). A library
  * utility; the pages have no counterpart. */
@@ -129,16 +137,25 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
  * Bytes of workspace a caller must pass to bpt_layer_forward_ws for these
  * arguments (0 if they are invalid or b*s == 0): one region that holds the bf16
  * K and V of the whole input (2 * b*s*h * 2 bytes) until attention is done and
- * then the FFN scratch of one wave (14 * h bytes per wave row: fp32 residual
- * stream, its bf16 copy and the 4h-wide bf16 intermediate), so its size is the
- * larger of the two; the fp32 entry adds bf16 copies of x and the weights.
- * wave_rows <= 0 selects the library's default FFN wave: the whole number of
- * query blocks (or of whole sequences) that the library's model of its GEMM
- * tile rounds finds fastest, with scratch of at most 1.5x the K/V bytes (or of
- * about 4096 rows, where that is more); 8192 rows at b=1, s=32768, h=4096,
- * q_block=1024, where the scratch fits inside the K/V region. Otherwise
- * wave_rows is rounded down to a multiple of q_block (at least q_block), and a
- * value of s or more groups whole sequences. */
+ * then the FFN scratch, so its size is the larger of the two, plus a few KiB.
+ * wave_rows = BPT_WAVE_CHAINED with bf16 inputs runs the FFN side of every
+ * query block in one launch over groups of 128-row tiles: the scratch is 3
+ * slots of a group's fp32 residual stream and its bf16 copy and 2 slots of
+ * its FFN intermediate (ffn wide, bf16), with the largest group of 16, 8, 4,
+ * 2 or 1 tiles whose slots take at most 1.5x the K/V bytes (or 32 MiB); at
+ * b=1, s=32768, h=4096 that is 2048-row groups inside the K/V region, 512 MiB
+ * in all (1.0x 2bsh read as elements). BPT_WAVE_DEFAULT (the library's
+ * choice: per-GEMM waves, which measured as fast as the chained launch at
+ * the large workloads and faster at the small ones), BPT_WAVE_DEFAULT_WAVES,
+ * wave_rows > 0 and fp32 inputs run one launch per GEMM and FFN wave: the
+ * scratch is one
+ * wave's (14 * h bytes per wave row: fp32 residual stream, its bf16 copy and
+ * the 4h-wide bf16 intermediate); wave_rows is rounded down to a multiple of
+ * q_block (at least q_block), and a value of s or more groups whole
+ * sequences; otherwise the library picks the whole number of query
+ * blocks (or of whole sequences) that its model of its GEMM tile
+ * rounds finds fastest, with scratch of at most 1.5x the K/V bytes (or of
+ * about 4096 rows). The fp32 entry adds bf16 copies of x and the weights. */
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows);
 

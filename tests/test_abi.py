@@ -105,36 +105,61 @@ def test_ws_entry_checks_dtype_and_workspace():
     assert L.bpt_layer_forward_ws(0, *p, *args, p[3], need, out, None) == ALIAS
 
 
-def test_workspace_bytes_follow_the_layout():
-    # bf16: one region holds K and V for the whole sequence during projection
-    # and attention, then the FFN wave scratch (fp32 hid, its bf16 copy and the
-    # bf16 intermediate U, wave rows x 4h), each piece rounded up to 1 KiB
-    def up(v):
-        return (v + 1023) // 1024 * 1024
+def _up(v):
+    return (v + 1023) // 1024 * 1024
 
-    def expect(b, s, h, wr):
-        return max(up(b * s * h * 2) * 2, up(wr * h * 4) + up(wr * h * 2) + up(wr * 4 * h * 2))
+
+def chain_workspace(b, s, h, f):
+    """Default bf16 workspace: one region holds K and V for the whole sequence
+    during projection and attention, then the slots of the one-launch FFN side
+    (3 slots of a row group's fp32 hid and bf16 hid copy, 2 of its bf16 U; the
+    largest group of 16, 8, 4, 2 or 1 128-row tiles whose slots take at most
+    1.5x the K/V bytes or 32 MiB), each piece rounded up to 1 KiB; then the
+    chain's counters (three per group)."""
+    M = b * s
+    mt = -(-M // 128)
+    kv = 2 * _up(M * h * 2)
+    for gm in (16, 8, 4, 2, 1):
+        groups = -(-mt // gm)
+        hs, us, rows = min(3, groups), min(2, groups), gm * 128
+        slots = _up(hs * rows * h * 4) + _up(hs * rows * h * 2) + _up(us * rows * f * 2)
+        if slots <= max(kv // 2 * 3, 32 << 20):
+            break
+    return _up(max(kv, slots) + 3 * groups * 4), kv, slots
+
+
+def test_workspace_bytes_follow_the_layout():
+    def wave(b, s, h, wr):
+        # explicit wave: K/V region, or one wave's fp32 hid, its bf16 copy and the bf16 U (wave rows x 4h)
+        return max(_up(b * s * h * 2) * 2, _up(wr * h * 4) + _up(wr * h * 2) + _up(wr * 4 * h * 2))
 
     b, s, h = 1, 32768, 4096
     ws = bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048)
-    # default wave at the 32k-token 7B shape: 8192 rows (8 query blocks), whose
-    # scratch fits inside the K/V region
-    assert ws == expect(b, s, h, 8192) == 2 * b * s * h * 2
-    assert bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048, 12288) == expect(b, s, h, 12288) > ws
-    # element ratio against 2bsh
-    assert ws / 2 / (2 * b * s * h) <= 1.0
-    # wave rows are whole query blocks; a whole-sequence wave covers whole sequences
-    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == expect(2, 2048, 1024, 4096)
-    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128, 2048) == expect(2, 2048, 1024, 2048)
-    assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == expect(1, 16384, 2048, 2048)
-    assert bpt.workspace_bytes(0, 1, 8192, 2048, 16, 512, 512) == expect(1, 8192, 2048, 4096)
-    # fp32 inputs add their bf16 parts: x as [x_hi | x_lo] rows, Wqkv as
-    # [hi; lo; hi], Wo, W1 and W2 as [hi; lo]
+    # the 32k-token 7B shape, default (per-GEMM waves): 8192-row waves (8 query
+    # blocks) whose scratch fits inside the K/V region
+    assert ws == wave(b, s, h, 8192) == 2 * b * s * h * 2
+    assert ws / 2 / (2 * b * s * h) <= 1.0  # element ratio against 2bsh
+    assert bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048, -2) == ws  # BPT_WAVE_DEFAULT_WAVES
+    assert bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048, 12288) == wave(b, s, h, 12288) > ws
+    # the chained schedule: its 2048-row slots fit inside the K/V region too
+    exp, kv, slots = chain_workspace(b, s, h, 4 * h)
+    assert bpt.workspace_bytes(0, b, s, h, 32, 1024, 2048, -1) == exp and slots < kv == ws
+    assert exp / 2 / (2 * b * s * h) <= 1.0001  # the counters add a few KiB
+    for args in [(2, 2048, 1024, 16, 128, 128), (1, 16384, 2048, 16, 2048, 2048), (1, 8192, 2048, 16, 512, 512),
+                 (1, 256, 256, 4, 64, 64), (3, 1000, 192, 3, 200, 125)]:
+        b_, s_, h_ = args[:3]
+        assert bpt.workspace_bytes(0, *args, -1) == chain_workspace(b_, s_, h_, 4 * h_)[0], args
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128) == wave(2, 2048, 1024, 4096)
+    assert bpt.workspace_bytes(0, 1, 8192, 2048, 16, 512, 512) == wave(1, 8192, 2048, 4096)
+    # explicit waves: whole query blocks; a whole-sequence wave covers whole sequences
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128, 2048) == wave(2, 2048, 1024, 2048)
+    assert bpt.workspace_bytes(0, 1, 16384, 2048, 16, 2048, 2048, 1000) == wave(1, 16384, 2048, 2048)
+    assert bpt.workspace_bytes(0, 2, 2048, 1024, 16, 128, 128, 100000) == wave(2, 2048, 1024, 4096)
+    # fp32 inputs keep one launch per GEMM and wave and add their bf16 parts: x
+    # as [x_hi | x_lo] rows, Wqkv as [hi; lo; hi], Wo, W1 and W2 as [hi; lo]
     f = bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
-    g = bpt.workspace_bytes(0, 1, 256, 256, 4, 64, 64)
-    assert g == expect(1, 256, 256, 256)
-    assert f == g + up(256 * 512 * 2) + up(768 * 768 * 2) + up(512 * 256 * 2) + up(512 * 1024 * 2) + \
-        up(2048 * 256 * 2)
+    assert f == wave(1, 256, 256, 256) + _up(256 * 512 * 2) + _up(768 * 768 * 2) + _up(512 * 256 * 2) + \
+        _up(512 * 1024 * 2) + _up(2048 * 256 * 2)
     assert bpt.workspace_bytes(0, 1, 256, 256, 3, 64, 64) == 0
     assert bpt.workspace_bytes(0, 0, 256, 256, 4, 64, 64) == 0
 
@@ -246,18 +271,14 @@ def test_kernel_timing_log_is_empty_without_launches():
     assert bpt.launch_count() >= 0
 
 
-def test_default_wave_keeps_to_its_memory_budget():
-    # over many valid shapes: the default workspace holds K and V, and its
-    # wave scratch stays within the larger of 1.5x the K/V bytes and the
-    # scratch of a ~4096-row wave (whole query blocks, or whole sequences)
+def test_workspaces_keep_to_their_memory_budgets():
+    # over many valid shapes: the default workspace (per-GEMM waves) holds K
+    # and V, and its wave scratch stays within the larger of 1.5x the K/V
+    # bytes and the scratch of a ~4096-row wave (whole query blocks, or whole
+    # sequences); the chained schedule's slots stay within 1.5x the K/V region
+    # (or 32 MiB) whenever a one-tile group does (otherwise the one-tile
+    # group's slots set the size), and its counters add a few KiB
     rng = np.random.default_rng(0)
-
-    def up(v):
-        return (v + 1023) // 1024 * 1024
-
-    def scratch(wr, h, f):
-        return up(wr * h * 4) + up(wr * h * 2) + up(wr * f * 2)
-
     for _ in range(300):
         heads = int(rng.integers(1, 9))
         h = heads * int(rng.choice([64, 128]))
@@ -265,14 +286,20 @@ def test_default_wave_keeps_to_its_memory_budget():
         s = q_block * int(rng.integers(1, 65))
         b = int(rng.integers(1, 5))
         f = 64 * int(rng.integers(1, 4 * h // 64 + 9))
-        ws = bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, ffn=f)
-        kv = 2 * up(b * s * h * 2)
+        ws_waves = bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, ffn=f)
+        kv = 2 * _up(b * s * h * 2)
         floor_rows = max(q_block, 4096 // q_block * q_block) if s >= 4096 else min(b, 4096 // s) * s
-        budget = max(kv // 2 * 3, scratch(floor_rows, h, f))
+        wave_budget = max(kv // 2 * 3, _up(floor_rows * h * 4) + _up(floor_rows * h * 2) + _up(floor_rows * f * 2))
+        assert kv <= ws_waves <= max(kv, wave_budget + 3 * 1024), (b, s, h, heads, q_block, f)
+        assert ws_waves >= bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, q_block, ffn=f)
+        ws = bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, -1, ffn=f)
+        exp, kv, slots = chain_workspace(b, s, h, f)
+        assert ws == exp, (b, s, h, heads, q_block, f)
         assert ws >= kv
-        assert ws <= max(kv, budget + 3 * 1024), (b, s, h, heads, q_block, f)
-        # and no smaller than the explicit one-block wave
-        assert ws >= bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, q_block, ffn=f)
+        mt = -(-b * s // 128)
+        one_tile = min(3, mt) * 128 * h * 6 + min(2, mt) * 128 * f * 2 + 3 * 1024
+        assert ws <= max(kv // 2 * 3, 32 << 20, one_tile) + _up(3 * mt * 4) + 1024, (b, s, h, heads, q_block, f)
+        assert bpt.workspace_bytes(0, b, s, h, heads, q_block, q_block, -2, ffn=f) == ws_waves
 
 
 def test_binding_checks_parameters_before_calling_the_library():

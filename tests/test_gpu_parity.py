@@ -261,6 +261,17 @@ def test_layer_result_does_not_depend_on_the_wave(wave_rows):
     assert_parity(got, ref, f"wave_rows={wave_rows}")
 
 
+@pytest.mark.parametrize("schedule", [-1, -2], ids=["chained", "default-waves"])
+def test_both_ffn_schedules_match_the_oracle(schedule):
+    # the FFN side in one launch (BPT_WAVE_CHAINED: four 2048-row groups here,
+    # so both scratch slots are reused) and in one launch per GEMM and wave
+    # (BPT_WAVE_DEFAULT_WAVES) compute the same layer
+    shape = bi.LayerShape(2, 4096, 256, 2, 128, 256, True)
+    inp = bi.make_inputs(shape, seed=9)
+    got = run_layer(shape, inp, wave_rows=schedule, workspace=True)
+    assert_parity(got, oracle_full(shape, inp), f"ffn schedule {schedule}")
+
+
 @pytest.mark.parametrize("q_scale,max_abs", [(2.0, MAX_ABS), (8.0, 0.1)])
 def test_layer_sharp_attention_matches_oracle(q_scale, max_abs):
     # query weights scaled: attention far from uniform, so attention errors are

@@ -148,16 +148,18 @@ def attention_backward_blockwise(Q, K, V, dO, heads: int, causal: bool, q_block:
     return dQ, dK, dV
 
 
-def layer_backward(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, heads: int, causal: bool,
-                   q_block: int | None = None, kv_block: int | None = None) -> dict:
-    """Gradients of the layer output y with respect to x and every parameter,
-    for the upstream gradient dy [b, s, h]; attention blockwise when both
-    block sizes are given. Returns a dict keyed like the arguments: dx, dWqkv,
-    dbqkv, dWo, dbo, dW1, db1, dW2, db2."""
-    h = x.shape[-1]
-    Q, K, V = ob.qkv_projection(x, Wqkv, bqkv)
-    O = ob.attention(Q, K, V, heads, causal, threads=1)
-    hid = x + O @ Wo + bo
+def ffn_backward(hid, W1, b1, W2, dy) -> dict:
+    """Gradients of the FFN block with its residual, y = hid + max(0, hid W1 +
+    b1) W2 + b2 (the standard FFN of the BPT paper review, section 3, with the
+    second residual of its blockwise FFN formula), for the upstream gradient
+    dy: dhid, dW1, db1, dW2, db2. The blockwise FFN is rematerialised in the
+    backward pass (paper review section 3, the scanned blockwise FFN):
+    u = max(0, a) is recomputed from hid here rather than stored.
+
+        a = hid W1 + b1;  u = max(0, a)
+        db2 = sum dy;  dW2 = u^T dy;  da = (dy W2^T) [a > 0]
+        db1 = sum da;  dW1 = hid^T da;  dhid = dy + da W1^T
+    """
     a = hid @ W1 + b1
     u = ob._relu(a)
 
@@ -170,7 +172,26 @@ def layer_backward(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, heads: int, causal
     da = (dy @ W2.T) * _relu_grad(a)
     g["db1"] = flat(da).sum(axis=0)
     g["dW1"] = flat(hid).T @ flat(da)
-    dhid = _dhid(dy, da, W1)
+    g["dhid"] = _dhid(dy, da, W1)
+    return g
+
+
+def layer_backward(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, heads: int, causal: bool,
+                   q_block: int | None = None, kv_block: int | None = None) -> dict:
+    """Gradients of the layer output y with respect to x and every parameter,
+    for the upstream gradient dy [b, s, h]; attention blockwise when both
+    block sizes are given. Returns a dict keyed like the arguments: dx, dWqkv,
+    dbqkv, dWo, dbo, dW1, db1, dW2, db2."""
+    h = x.shape[-1]
+    Q, K, V = ob.qkv_projection(x, Wqkv, bqkv)
+    O = ob.attention(Q, K, V, heads, causal, threads=1)
+    hid = x + O @ Wo + bo
+
+    def flat(z):
+        return z.reshape(-1, z.shape[-1])
+
+    g = ffn_backward(hid, W1, b1, W2, dy)
+    dhid = g.pop("dhid")
     g["dbo"] = flat(dhid).sum(axis=0)
     g["dWo"] = flat(O).T @ flat(dhid)
     dO = dhid @ Wo.T

@@ -116,3 +116,53 @@ def test_layer_backward_blockwise_equals_plain():
     got = grads(p, dy, 2, True, q_block=4, kv_block=2)
     for name in NAMES:
         np.testing.assert_allclose(got["d" + name], ref["d" + name], rtol=0, atol=1e-12, err_msg=name)
+
+
+# ---------------------------------------------------------------------------
+# the FFN block alone (ffn_backward): pinned to central differences of the
+# forward oracle's FFN-with-residual (residual_ffn with O = 0, Wo = 0, bo = 0
+# gives y = hid + max(0, hid W1 + b1) W2 + b2), and to torch fp64 autograd
+# ---------------------------------------------------------------------------
+
+def ffn_forward(hid, W1, b1, W2, b2):
+    z = np.zeros_like(hid)
+    return oracle.residual_ffn(hid, z, np.zeros((hid.shape[-1], hid.shape[-1])), np.zeros(hid.shape[-1]),
+                               W1, b1, W2, b2)
+
+
+@pytest.mark.parametrize("rows,h,f,seed", [(5, 4, 8, 1), (7, 6, 3, 2), (1, 3, 5, 3)])
+def test_ffn_backward_matches_central_differences(rows, h, f, seed):
+    rng = np.random.default_rng(seed)
+    hid = rng.standard_normal((rows, h))
+    W1, b1 = rng.standard_normal((h, f)), rng.standard_normal(f)
+    W2, b2 = rng.standard_normal((f, h)), rng.standard_normal(h)
+    dy = rng.standard_normal((rows, h))
+    assert np.abs(hid @ W1 + b1).min() > 1e-4  # away from the ReLU kink
+    g = obb.ffn_backward(hid, W1, b1, W2, dy)
+    params = {"hid": hid, "W1": W1, "b1": b1, "W2": W2, "b2": b2}
+    eps = 1e-6
+    for name, arr in params.items():
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + eps
+            up = float(np.sum(ffn_forward(**params) * dy))
+            arr[idx] = old - eps
+            down = float(np.sum(ffn_forward(**params) * dy))
+            arr[idx] = old
+            num[idx] = (up - down) / (2 * eps)
+        np.testing.assert_allclose(g["d" + name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_ffn_backward_matches_torch_autograd():
+    rng = np.random.default_rng(11)
+    rows, h, f = 37, 16, 48
+    t = {k: torch.tensor(v, requires_grad=True) for k, v in {
+        "hid": rng.standard_normal((rows, h)), "W1": rng.standard_normal((h, f)) / 4, "b1": rng.standard_normal(f),
+        "W2": rng.standard_normal((f, h)) / 7, "b2": rng.standard_normal(h)}.items()}
+    dy = rng.standard_normal((rows, h))
+    y = t["hid"] + torch.relu(t["hid"] @ t["W1"] + t["b1"]) @ t["W2"] + t["b2"]
+    y.backward(torch.tensor(dy))
+    g = obb.ffn_backward(*(t[k].detach().numpy() for k in ("hid", "W1", "b1", "W2")), dy)
+    for k in ("hid", "W1", "b1", "W2", "b2"):
+        np.testing.assert_allclose(g["d" + k], t[k].grad.numpy(), rtol=1e-10, atol=1e-10, err_msg=k)

@@ -727,6 +727,47 @@ def max_context_arm(args):
     return 0 if (status == 0 and finite) else 1
 
 
+def ffn_backward_arm(args):
+    """Throughput of the FFN block's backward (bpt_ffn_backward) at the 7B-class
+    layer's shapes (rows 32768, h 4096, ffn 16384; 4096-row chunks): five
+    products of 2 rows h ffn flops each (the recomputed intermediate, da,
+    dhid, dW1, dW2). Seeded synthetic inputs drawn on the device."""
+    import torch
+    import blockwise_attn_ffn_bpt_b200 as bpt
+    rows, h, f = 32768, 4096, 16384
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    g = torch.Generator(device=device).manual_seed(0)
+    hid = torch.randn((rows, h), generator=g, device=device)
+    dy = torch.randn((rows, h), generator=g, device=device)
+    W1 = (torch.randn((h, f), generator=g, device=device) / math.sqrt(h)).to(torch.bfloat16)
+    b1 = (torch.randn(f, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((f, h), generator=g, device=device) / math.sqrt(f)).to(torch.bfloat16)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        bpt.ffn_backward(hid, W1, b1, W2, dy, stream=stream)
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(gpu_index(0)) as clocks:
+        for e0, e1 in evs:
+            e0.record(stream)
+            bpt.ffn_backward(hid, W1, b1, W2, dy, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    status = bpt.stream_status(stream)
+    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    flops = 5 * 2.0 * rows * h * f
+    peaks, src = measured_peaks()
+    line = {"metric": "FFN block backward (bpt_ffn_backward) TFLOP/s on 1 B200", "value": flops / (ms / 1e3) / 1e12,
+            "unit": "TFLOP/s", "ms": ms, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+            "config": {"workload": "ffn_backward_rows32768_h4096_f16384", "chunk_rows": 4096},
+            "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
+            "peak_source": f"{src} bf16_tflops (burst)", "device_status": status, "clocks": clocks.summary(),
+            "data": "synthetic (torch generator on the device)"}
+    print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -744,9 +785,13 @@ def main(argv=None):
     ap.add_argument("--only", default="", help="with --all-configs: comma-separated name fragments to keep")
     ap.add_argument("--ffn", choices=list(FFN_SCHEDULES), default="default",
                     help="FFN-side schedule: the library's default, one chained launch, or per-GEMM waves")
+    ap.add_argument("--ffn-backward", action="store_true",
+                    help="instead: throughput of the FFN block's backward at the 7B-class layer's shapes")
     args = ap.parse_args(argv)
     if args.max_context:
         return max_context_arm(args)
+    if args.ffn_backward:
+        return ffn_backward_arm(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.all_configs:

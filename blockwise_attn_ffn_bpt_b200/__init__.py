@@ -24,7 +24,8 @@ EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",
     "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
     "bpt_layer_forward_host", "bpt_convert_f32_to_bf16",
-    "bpt_qkv_projection", "bpt_attention", "bpt_stream_status", "bpt_device_status", "bpt_wait_flag",
+    "bpt_qkv_projection", "bpt_attention", "bpt_ffn_backward_workspace_bytes", "bpt_ffn_backward",
+    "bpt_stream_status", "bpt_device_status", "bpt_wait_flag",
     "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
 )
 
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
     L.bpt_qkv_projection.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
     L.bpt_attention.restype = i
     L.bpt_attention.argtypes = [vp] * 3 + [i] * 7 + [vp, vp]
+    L.bpt_ffn_backward_workspace_bytes.restype = sz
+    L.bpt_ffn_backward_workspace_bytes.argtypes = [i] * 4
+    L.bpt_ffn_backward.restype = i
+    L.bpt_ffn_backward.argtypes = [vp] * 5 + [i] * 4 + [vp] * 6 + [sz, vp]
     L.bpt_stream_status.restype = i
     L.bpt_stream_status.argtypes = [vp]
     L.bpt_device_status.restype = i
@@ -268,6 +273,33 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int, q_b
                             _ptr(o), _stream(stream))
     _check(r, "bpt_attention")
     return o
+
+
+def ffn_backward(hid: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, W2: torch.Tensor, dy: torch.Tensor,
+                 chunk_rows: int = 0, stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of the FFN block out = hid + max(0, hid W1 + b1) W2 + b2 for
+    dy = dL/dout (bpt_ffn_backward): hid, dy fp32 [..., h] on the GPU; W1, b1,
+    W2 bf16. Returns {"dhid", "dW1", "db1", "dW2", "db2"} (fp32)."""
+    h = hid.shape[-1]
+    ffn = W1.shape[-1]
+    rows = hid.numel() // h
+    if hid.dtype != torch.float32 or dy.dtype != torch.float32 or dy.shape != hid.shape:
+        raise TypeError("hid and dy must be fp32 tensors of the same shape")
+    for name, t, shape in (("W1", W1, (h, ffn)), ("b1", b1, (ffn,)), ("W2", W2, (ffn, h))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be bf16 of shape {shape}")
+    dev = hid.device
+    g = {"dhid": torch.empty_like(hid), "dW1": torch.empty((h, ffn), dtype=torch.float32, device=dev),
+         "db1": torch.empty(ffn, dtype=torch.float32, device=dev),
+         "dW2": torch.empty((ffn, h), dtype=torch.float32, device=dev),
+         "db2": torch.empty(h, dtype=torch.float32, device=dev)}
+    nbytes = int(lib().bpt_ffn_backward_workspace_bytes(rows, h, ffn, chunk_rows))
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    r = lib().bpt_ffn_backward(_ptr(hid), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(dy), rows, h, ffn, chunk_rows,
+                               _ptr(g["dhid"]), _ptr(g["dW1"]), _ptr(g["db1"]), _ptr(g["dW2"]), _ptr(g["db2"]),
+                               _ptr(ws), ws.numel(), _stream(stream))
+    _check(r, "bpt_ffn_backward")
+    return g
 
 
 def stream_status(stream: Optional[torch.cuda.Stream] = None) -> int:

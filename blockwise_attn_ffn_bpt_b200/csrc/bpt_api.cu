@@ -32,6 +32,16 @@
 #include "bpt.h"
 #include "ffn_chain.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
+
+// The bf16 forward GEMMs run on SM pairs (gemm_pair.cuh) when this is 1, on
+// single SMs (gemm.cuh) when it is 0. Measured on B200 at b=1, s=32768,
+// h=4096: QKV 2.46 -> 2.15 ms, FFN-up 3.39 -> 2.92 ms, FFN-down 3.34 -> 2.90
+// ms, out-projection 1.03 -> 0.95 ms (the single-SM kernel's copies and MMA
+// reads exceed what shared memory delivers per clock; a pair halves B's).
+#ifndef BPT_PAIR_GEMM
+#define BPT_PAIR_GEMM 1
+#endif
 
 namespace bpt {
 namespace {
@@ -155,6 +165,20 @@ int check_device(int* sms) {
                                         GEMM_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_FFN_DOWN>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_BWD_DA, 0, 0>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_BWD_DHID, 0, 0>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI_GRAD, 1, 1>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_OUTPROJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_FFN_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_FFN_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GP_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(ffn_chain_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         GEMM_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -399,6 +423,13 @@ int for_each_wave(int b, int s, int h, int ffn, int q_block, int wave_rows, F&& 
   return BPT_OK;
 }
 
+// Rows per chunk of the FFN block's backward: the caller's, rounded down to a
+// multiple of 128 (at least 128), or 4096 by default; never more than rows.
+long long ffn_bwd_chunk(int rows, int chunk_rows) {
+  long long r = chunk_rows > 0 ? std::max(128, chunk_rows / 128 * 128) : 4096;
+  return std::min<long long>(r, rows);
+}
+
 // ------------------------------------------------------------- FFN chain plan
 // Groups of the one-launch FFN side (ffn_chain.cuh): the largest group of
 // 16, 8, 4, 2 or 1 M-tiles whose slots (fp32 hid, its bf16 copy, bf16 U) take
@@ -519,6 +550,20 @@ int launch_gemm_split(const void* A, long long M, long long a_cols, long long ld
   args.K = (int)K;
   args.m_tiles = (int)((M + GEMM_BM - 1) / GEMM_BM);
   args.n_tiles = (int)((N + GEMM_BN - 1) / GEMM_BN);
+  if (BPT_PAIR_GEMM && a_split == 0) {
+    // 256 x 256 tiles on SM pairs: each CTA maps its own 128 rows of A and its
+    // 128-column half of B
+    CUtensorMap tb2;
+    if (!map_rows(&ta, A, M, a_cols, lda, 128) || !map_rows(&tb2, B, K, N, N, 64)) return BPT_ERR_CUDA;
+    args.m_tiles = (int)((M + GP_BM - 1) / GP_BM);
+    args.n_tiles = (int)((N + GP_BN - 1) / GP_BN);
+    const int pairs = std::min(args.m_tiles * args.n_tiles, sms / 2);
+    {
+      LaunchScope ls(name, st);
+      gemm_pair_tcgen05<MODE><<<2 * pairs, GEMM_THREADS, GP_SMEM_BYTES, st>>>(ta, tb2, args);
+    }
+    return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+  }
   const int tiles = args.m_tiles * args.n_tiles;
   const int grid = std::min(tiles, sms);
   {
@@ -532,6 +577,57 @@ template <int MODE>
 int launch_gemm(const void* A, long long M, long long K, long long lda, const void* B, long long N,
                 GemmArgs args, int sms, cudaStream_t st, int* status, const char* name) {
   return launch_gemm_split<MODE>(A, M, K, lda, B, K, N, 0, 0, args, sms, st, status, name);
+}
+
+// D[M, N] = A B for the backward's products: A is [M, K] (lda elements apart)
+// or, with A_MN, stored [K, M]; B is [K, N] (ldb apart) with B_MN or stored
+// [N, K] without. K need not be a multiple of 64: the copies zero-fill past
+// the last row of an operand.
+template <int MODE, int A_MN, int B_MN>
+int launch_gemm_t(const void* A, long long lda, const void* B, long long ldb, long long M, long long N, long long K,
+                  GemmArgs args, int sms, cudaStream_t st, int* status, const char* name) {
+  if (M <= 0 || N <= 0) return BPT_OK;
+  CUtensorMap ta, tb;
+  const bool ok_a = A_MN ? map_rows(&ta, A, K, M, lda, 64) : map_rows(&ta, A, M, K, lda, GEMM_BM);
+  const bool ok_b = B_MN ? map_rows(&tb, B, K, N, ldb, 64) : map_rows(&tb, B, N, K, ldb, GEMM_BN);
+  if (!ok_a || !ok_b) return BPT_ERR_CUDA;
+  args.status = status;
+  args.M = (int)M;
+  args.N = (int)N;
+  args.K = (int)((K + GEMM_BK - 1) / GEMM_BK * GEMM_BK);
+  args.m_tiles = (int)((M + GEMM_BM - 1) / GEMM_BM);
+  args.n_tiles = (int)((N + GEMM_BN - 1) / GEMM_BN);
+  const int grid = std::min(args.m_tiles * args.n_tiles, sms);
+  {
+    LaunchScope ls(name, st);
+    gemm_bf16_tcgen05<MODE, A_MN, B_MN><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+// out[c] (+)= sum over rows r of src[r * ld + c], fp32 accumulation in row
+// order (deterministic): one thread per column.
+template <typename T>
+__global__ void colsum_kernel(const T* __restrict__ src, long long rows, int cols, long long ld, float* out,
+                              int accumulate) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  float acc = 0.0f;
+  for (long long r = 0; r < rows; ++r) {
+    if constexpr (sizeof(T) == 2)
+      acc += __bfloat162float(src[r * ld + c]);
+    else
+      acc += src[r * ld + c];
+  }
+  out[c] = accumulate ? out[c] + acc : acc;
+}
+
+template <typename T>
+int launch_colsum(const T* src, long long rows, int cols, long long ld, float* out, int accumulate, cudaStream_t st) {
+  if (cols <= 0) return BPT_OK;
+  LaunchScope ls("colsum", st);
+  colsum_kernel<T><<<(cols + 127) / 128, 128, 0, st>>>(src, rows, cols, ld, out, accumulate);
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
 // Attention of the query rows [t_start, t_start + t_len) of sequences
@@ -1123,6 +1219,88 @@ int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stre
   int sms = 0;
   BPT_TRY(check_device(&sms));
   return launch_convert(src, dst, n, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t bpt_ffn_backward_workspace_bytes(int rows, int h, int ffn, int chunk_rows) {
+  if (rows <= 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return 0;
+  const long long R = ffn_bwd_chunk(rows, chunk_rows);
+  return 2 * align_up((size_t)R * h * 2, 1024) + 2 * align_up((size_t)R * ffn * 2, 1024);
+}
+
+int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy, int rows,
+                     int h, int ffn, int chunk_rows, float* dhid, float* dW1, float* db1, float* dW2, float* db2,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (rows < 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return BPT_ERR_SHAPE;
+  if ((long long)h * ffn > 0x7fffffffLL || (long long)rows * std::max(h, ffn) > (1LL << 40)) return BPT_ERR_SHAPE;
+  if (rows == 0) return BPT_OK;
+  const void* ptrs[12] = {hid, W1, b1, W2, dy, dhid, dW1, db1, dW2, db2, workspace, nullptr};
+  for (int i = 0; i < 11; ++i)
+    if (!ptrs[i]) return BPT_ERR_NULL;
+  for (int i = 0; i < 11; ++i)
+    if (!aligned16(ptrs[i])) return BPT_ERR_ALIGN;
+  const long long R = ffn_bwd_chunk(rows, chunk_rows);
+  const size_t need = bpt_ffn_backward_workspace_bytes(rows, h, ffn, chunk_rows);
+  if (ws_bytes < need) return BPT_ERR_NOMEM;
+  // outputs must not overlap the inputs or one another
+  const Range in[5] = {rng(hid, (size_t)rows * h * 4), rng(W1, (size_t)h * ffn * 2), rng(b1, (size_t)ffn * 2),
+                       rng(W2, (size_t)ffn * h * 2), rng(dy, (size_t)rows * h * 4)};
+  const Range outs[6] = {rng(dhid, (size_t)rows * h * 4), rng(dW1, (size_t)h * ffn * 4), rng(db1, (size_t)ffn * 4),
+                         rng(dW2, (size_t)ffn * h * 4), rng(db2, (size_t)h * 4), rng(workspace, need)};
+  for (int i = 0; i < 6; ++i) {
+    for (const Range& r : in)
+      if (overlap(outs[i], r)) return BPT_ERR_ALIAS;
+    for (int j = i + 1; j < 6; ++j)
+      if (overlap(outs[i], outs[j])) return BPT_ERR_ALIAS;
+  }
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(ws + align_up((size_t)R * h * 2, 1024));
+  __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + 2 * align_up((size_t)R * h * 2, 1024));
+  __nv_bfloat16* da = reinterpret_cast<__nv_bfloat16*>(ws + 2 * align_up((size_t)R * h * 2, 1024) +
+                                                       align_up((size_t)R * ffn * 2, 1024));
+  for (long long r0 = 0; r0 < rows; r0 += R) {
+    const long long n = std::min<long long>(R, rows - r0);
+    const int acc = r0 > 0 ? 1 : 0;
+    BPT_TRY(launch_convert(hid + r0 * h, hb, n * h, sms, st));
+    BPT_TRY(launch_convert(dy + r0 * h, dyb, n * h, sms, st));
+    // the chunk's FFN intermediate again (rematerialised, not stored by the forward)
+    GemmArgs a{};
+    a.bias = b1;
+    a.dst = U;
+    a.ld_dst = ffn;
+    BPT_TRY((launch_gemm_t<EPI_FFN_UP, 0, 1>(hb, h, W1, ffn, n, ffn, h, a, sms, st, status, "bwd_ffn_up")));
+    // da = (dy W2^T) [U > 0]
+    a = GemmArgs{};
+    a.mask_u = U;
+    a.ld_mask = ffn;
+    a.dst = da;
+    a.ld_dst = ffn;
+    BPT_TRY((launch_gemm_t<EPI_BWD_DA, 0, 0>(dyb, h, W2, h, n, ffn, h, a, sms, st, status, "bwd_da")));
+    // dhid = dy + da W1^T
+    a = GemmArgs{};
+    a.dy = dy + r0 * h;
+    a.ld_dy = h;
+    a.out = dhid + r0 * h;
+    a.ld_out = h;
+    BPT_TRY((launch_gemm_t<EPI_BWD_DHID, 0, 0>(da, ffn, W1, ffn, n, h, ffn, a, sms, st, status, "bwd_dhid")));
+    // dW1 (+)= hid^T da and dW2 (+)= U^T dy over the chunk's rows
+    a = GemmArgs{};
+    a.accumulate = acc;
+    a.out = dW1;
+    a.ld_out = ffn;
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(hb, h, da, ffn, h, ffn, n, a, sms, st, status, "bwd_dW1")));
+    a.out = dW2;
+    a.ld_out = h;
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(U, ffn, dyb, h, ffn, h, n, a, sms, st, status, "bwd_dW2")));
+    BPT_TRY(launch_colsum(da, n, ffn, ffn, db1, acc, st));
+    BPT_TRY(launch_colsum(dy + r0 * h, n, h, h, db2, acc, st));
+  }
+  return BPT_OK;
 }
 
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,

@@ -1,7 +1,10 @@
 // Persistent tcgen05 GEMM with fused epilogues for the projections of the BPT
-// layer: D[M, N] = A[M, K] * B[K, N] with A bf16 row-major (K-major operand),
-// B bf16 row-major [in, out] weights (MN-major operand), fp32 accumulation in
-// tensor memory.
+// layer and of its FFN block's backward: D[M, N] = A[M, K] * B[K, N], bf16
+// operands, fp32 accumulation in tensor memory. Forward: A row-major [M, K]
+// (K-major operand), B = [in, out] weights row-major [K, N] (MN-major
+// operand). Backward: B = a weight used transposed, stored [N, K] (K-major,
+// B_MN = 0), and, for weight gradients, A = an activation used transposed,
+// stored [K, M] (MN-major, A_MN = 1).
 //
 // Roles (192 threads): warp 0 issues TMA tile loads into a STAGES-deep ring,
 // one thread of warp 1 issues tcgen05.mma into one of two TMEM accumulators,
@@ -32,6 +35,9 @@ enum EpiMode {
   EPI_OUTPROJ = 1,   // + bo + x (first residual) -> fp32 hid and its bf16 copy (wave scratch)
   EPI_FFN_UP = 2,    // + b1, ReLU -> bf16 U
   EPI_FFN_DOWN = 3,  // + b2 + hid (second residual) -> fp32 out
+  EPI_BWD_DA = 4,    // (dy W2^T) masked by U > 0 (the ReLU's derivative) -> bf16 da
+  EPI_BWD_DHID = 5,  // + dy (the residual's gradient) -> fp32 dhid
+  EPI_GRAD = 6,      // -> fp32 weight gradient, added to what is there when accumulate is set
 };
 
 struct GemmArgs {
@@ -66,6 +72,12 @@ struct GemmArgs {
   // 2 a_kb blocks, then kb - a_kb (A = [x_hi | x_lo] against [W_hi; W_lo; W_hi]).
   int a_split;
   int a_kb;  // K blocks of one copy of A
+  // backward: U (EPI_BWD_DA's mask), dy fp32 (EPI_BWD_DHID), accumulate (EPI_GRAD)
+  const __nv_bfloat16* mask_u;
+  long long ld_mask;
+  const float* dy;
+  long long ld_dy;
+  int accumulate;
   int* status;  // status word of the launching stream
 };
 
@@ -123,7 +135,7 @@ __device__ __forceinline__ void store32_f32(float* dst, const float (&v)[32]) {
 template <int MODE>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int col, float (&v)[32]) {
   float bias[32];
-  load32(a.bias, a.bias_f32, col, bias);
+  if constexpr (MODE <= EPI_FFN_DOWN) load32(a.bias, a.bias_f32, col, bias);
   if constexpr (MODE == EPI_QKV) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += bias[i];
@@ -144,12 +156,33 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int co
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i] + bias[i], 0.0f);
     store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
-  } else {
+  } else if constexpr (MODE == EPI_FFN_DOWN) {
     float hid[32];
     load32(a.hid + (long long)row * a.ld_hid + col, 1, 0, hid);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += bias[i] + hid[i];
     float* o = a.out + (a.row0 + row) * a.ld_out + col;
+    store32_f32(o, v);
+  } else if constexpr (MODE == EPI_BWD_DA) {
+    float u[32];
+    load32(a.mask_u, 0, (long long)row * a.ld_mask + col, u);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = u[i] > 0.0f ? v[i] : 0.0f;
+    store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
+  } else if constexpr (MODE == EPI_BWD_DHID) {
+    float dy[32];
+    load32(a.dy, 1, (long long)row * a.ld_dy + col, dy);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += dy[i];
+    store32_f32(a.out + (long long)row * a.ld_out + col, v);
+  } else {
+    float* o = a.out + (long long)row * a.ld_out + col;
+    if (a.accumulate) {
+      float old[32];
+      load32(o, 1, 0, old);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += old[i];
+    }
     store32_f32(o, v);
   }
 }
@@ -164,7 +197,11 @@ __device__ __forceinline__ void gemm_tile_coords(int t, int m_tiles, int n_tiles
   nt = r / gm;
 }
 
-template <int MODE>
+// A_MN = 1: A stored [K, M] (M contiguous), loaded as two [64 k][64 m] boxes
+// per stage; otherwise [M, K], one [128 m][64 k] box. B_MN = 1: B stored [K,
+// N], four [64 k][64 n] boxes; otherwise [N, K], one [256 n][64 k] box. Both
+// are 128-byte swizzled; the descriptors follow the operand's majorness.
+template <int MODE, int A_MN = 0, int B_MN = 1>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmArgs args) {
@@ -226,10 +263,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa = smem_base + stage * GEMM_STAGE_BYTES;
           mbar_arrive_expect_tx(fb, GEMM_STAGE_BYTES);
-          tma_load_2d(sa, &tmA, fb, a_block(args, kb) * GEMM_BK, m0);
+          if constexpr (A_MN) {
 #pragma unroll
-          for (int j = 0; j < GEMM_BN / 64; ++j)
-            tma_load_2d(sa + GEMM_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);
+            for (int j = 0; j < GEMM_BM / 64; ++j)
+              tma_load_2d(sa + j * GEMM_B_BOX_BYTES, &tmA, fb, m0 + 64 * j, kb * GEMM_BK);
+          } else {
+            tma_load_2d(sa, &tmA, fb, a_block(args, kb) * GEMM_BK, m0);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int j = 0; j < GEMM_BN / 64; ++j)
+              tma_load_2d(sa + GEMM_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);
+          } else {
+            tma_load_2d(sa + GEMM_A_BYTES, &tmB, fb, kb * GEMM_BK, n0);
+          }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
@@ -246,7 +293,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, 0, 1);
+      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -264,8 +311,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sb = sa + GEMM_A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(sb + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024);
+            // K-major: the 16-deep slice starts 32 bytes further along each
+            // 128-byte row; MN-major: 16 rows (of 128 bytes) further, with the
+            // 64-wide boxes GEMM_B_BOX_BYTES apart
+            const uint64_t adesc = A_MN ? smem_desc_sw128(sa + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024)
+                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bdesc = B_MN ? smem_desc_sw128(sb + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024)
+                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
             mma_bf16_ss(d, adesc, bdesc, idesc, (kb | kk) != 0);
           }
           mma_commit(empty0 + 8 * stage);

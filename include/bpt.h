@@ -282,6 +282,42 @@ int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int
                   int kv_block, int causal, void* o, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Backward of the FFN block (part of the layer's backward pass).
+ * ------------------------------------------------------------------------ */
+
+/* Gradients of the FFN block with its residual, out = hid + max(0, hid W1 +
+ * b1) W2 + b2 (paper review section 3: the standard FFN and the second
+ * residual of the blockwise FFN formula), for the upstream gradient dy =
+ * dL/dout. The pages train with this layer and rematerialise the blockwise
+ * FFN in the backward pass (the scanned blockwise FFN of section 3): the
+ * intermediate max(0, hid W1 + b1) is recomputed here, chunk by chunk of
+ * rows, never stored for the whole sequence.
+ *
+ *     u = max(0, hid W1 + b1)       (recomputed per chunk)
+ *     da = (dy W2^T) * [u > 0]
+ *     dhid = dy + da W1^T           dW1 = hid^T da    db1 = sum_rows da
+ *     dW2 = u^T dy                  db2 = sum_rows dy
+ *
+ * hid, dy: fp32 [rows, h] device memory; W1 [h, ffn], b1 [ffn], W2 [ffn, h]
+ * bf16 (the layer's weights). Outputs, fp32, written entirely (not
+ * accumulated into): dhid [rows, h], dW1 [h, ffn], db1 [ffn], dW2 [ffn, h],
+ * db2 [h]. The matrix products take bf16 operands (hid and dy rounded to
+ * nearest even) with fp32 accumulation; the weight gradients sum the chunks
+ * in fp32. chunk_rows: rows per chunk, rounded down to a multiple of 128 (0 =
+ * 4096). workspace: device memory of at least
+ * bpt_ffn_backward_workspace_bytes(...) bytes (bf16 copies of a chunk's hid
+ * and dy, its recomputed intermediate and da). h and ffn must be multiples of
+ * 64. Errors: BPT_ERR_SHAPE, BPT_ERR_NULL, BPT_ERR_ALIGN (16 bytes),
+ * BPT_ERR_NOMEM (workspace too small), BPT_ERR_ALIAS (an output or the
+ * workspace overlaps an input or another output); nothing launched then.
+ * Asynchronous on `stream`; device-side failures through
+ * bpt_stream_status. */
+size_t bpt_ffn_backward_workspace_bytes(int rows, int h, int ffn, int chunk_rows);
+int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy, int rows,
+                     int h, int ffn, int chunk_rows, float* dhid, float* dW1, float* db1, float* dW2, float* db2,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Status and measurement.
  * ------------------------------------------------------------------------ */
 

@@ -324,3 +324,32 @@ def test_binding_checks_parameters_before_calling_the_library():
         bpt.layer_forward_host(x, params, 1, 8, 8, True, out_host=torch.empty((b, s, h)))
     with pytest.raises(TypeError):
         bpt.convert_f32_to_bf16(torch.zeros(4))
+
+
+def test_ffn_backward_entry_validates_before_touching_memory():
+    L = bpt.lib()
+    p = fake_ptrs(11)
+    hid, W1, b1, W2, dy, dhid, dW1, db1, dW2, db2, ws = p
+    rows, h, f = 1000, 256, 1024
+    need = L.bpt_ffn_backward_workspace_bytes(rows, h, f, 384)
+    # chunk of 384 rows: bf16 copies of hid and dy, the intermediate and da
+    assert need == 2 * _up(384 * h * 2) + 2 * _up(384 * f * 2)
+    assert L.bpt_ffn_backward_workspace_bytes(rows, h, f, 0) == 2 * _up(1000 * h * 2) + 2 * _up(1000 * f * 2)
+    assert L.bpt_ffn_backward_workspace_bytes(rows, h, f, 100) == 2 * _up(128 * h * 2) + 2 * _up(128 * f * 2)
+    assert L.bpt_ffn_backward_workspace_bytes(rows, 100, f, 0) == 0
+
+    def call(**kw):
+        a = dict(hid=hid, W1=W1, b1=b1, W2=W2, dy=dy, rows=rows, h=h, f=f, chunk=384, dhid=dhid, dW1=dW1, db1=db1,
+                 dW2=dW2, db2=db2, ws=ws, nbytes=need)
+        a.update(kw)
+        return L.bpt_ffn_backward(a["hid"], a["W1"], a["b1"], a["W2"], a["dy"], a["rows"], a["h"], a["f"],
+                                  a["chunk"], a["dhid"], a["dW1"], a["db1"], a["dW2"], a["db2"], a["ws"],
+                                  a["nbytes"], None)
+
+    assert call(rows=0) == OK
+    assert call(h=100) == SHAPE and call(f=1000) == SHAPE and call(rows=-1) == SHAPE and call(chunk=-5) == SHAPE
+    assert call(W2=None) == NULL and call(ws=None) == NULL
+    assert call(dy=dy + 8) == ALIGN
+    assert call(nbytes=need - 1) == NOMEM
+    assert call(dW1=hid) == ALIAS  # an output over an input
+    assert call(db1=dW2 + 16) == ALIAS  # two outputs overlapping

@@ -29,6 +29,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_pair.cuh"
 #include "bpt.h"
 #include "ffn_chain.cuh"
 #include "gemm.cuh"
@@ -41,6 +42,15 @@
 // reads exceed what shared memory delivers per clock; a pair halves B's).
 #ifndef BPT_PAIR_GEMM
 #define BPT_PAIR_GEMM 1
+#endif
+// Attention with dh = 128 runs on SM pairs (attention_pair.cuh) when this is
+// 1, on single SMs (attention.cuh) when it is 0. The pair form passes the same
+// parity tests but measured 20-30% slower on B200 (b=1, s=32768, h=4096:
+// 10.8 ms against 8.7-9.0 ms): each of its MMA steps waits for the slower of
+// two CTAs' softmax, which costs more than the halved shared-memory traffic
+// of its S MMAs gains.
+#ifndef BPT_PAIR_ATTENTION
+#define BPT_PAIR_ATTENTION 0
 #endif
 
 namespace bpt {
@@ -125,12 +135,12 @@ bool map_rows(CUtensorMap* m, const void* base, long long rows, long long cols, 
   return make_map(m, base, 2, dims, strides, box);
 }
 
-// [b, s, cols] bf16 with `ld` elements between rows, [128 rows][64] boxes;
+// [b, s, cols] bf16 with `ld` elements between rows, [box_rows][64] boxes;
 // rows past s of a sequence read as zero.
-bool map_seq(CUtensorMap* m, const void* base, int b, int s, int cols, long long ld) {
+bool map_seq(CUtensorMap* m, const void* base, int b, int s, int cols, long long ld, uint32_t box_rows = 128) {
   const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)s, (uint64_t)b};
   const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)ld * 2 * (uint64_t)s};
-  const uint32_t box[3] = {64, 128, 1};
+  const uint32_t box[3] = {64, box_rows, 1};
   return make_map(m, base, 3, dims, strides, box);
 }
 
@@ -181,6 +191,8 @@ int check_device(int* sms) {
                                         GP_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(ffn_chain_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         GEMM_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_pair_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnPairCfg::SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         AttnCfg<64>::SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -189,11 +201,13 @@ int check_device(int* sms) {
       // the attention kernel splits its registers between warpgroups assuming
       // it was built with exactly ATT_REGS_LAUNCH per thread; any other build
       // is never launched (its register requests could not be met)
-      cudaFuncAttributes fa64{}, fa128{};
+      cudaFuncAttributes fa64{}, fa128{}, fap{};
       if (cudaFuncGetAttributes(&fa64, attention_fwd_tcgen05<64>) != cudaSuccess ||
-          cudaFuncGetAttributes(&fa128, attention_fwd_tcgen05<128>) != cudaSuccess)
+          cudaFuncGetAttributes(&fa128, attention_fwd_tcgen05<128>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fap, attention_pair_tcgen05) != cudaSuccess)
         return BPT_ERR_CUDA;
-      if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH) d.ok = false;
+      if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH || fap.numRegs != ATT_REGS_LAUNCH)
+        d.ok = false;
     }
     d.checked = true;
   }
@@ -637,6 +651,30 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
                      cudaStream_t st, int* status) {
   const int dh = h / heads;
   CUtensorMap tq, tk, tv;
+  if (BPT_PAIR_ATTENTION && dh == 128) {
+    // K halves are [64 keys][64 cols] boxes, Q and the V halves [128][64]
+    if (!map_seq(&tq, q, b, s, h, ldq, 128) || !map_seq(&tk, k, b, s, h, h, 64) || !map_seq(&tv, v, b, s, h, h, 128))
+      return BPT_ERR_CUDA;
+    AttnPairArgs a{};
+    a.s = s;
+    a.heads = heads;
+    a.causal = causal ? 1 : 0;
+    a.t_start = t_start;
+    a.t_len = t_len;
+    a.n_quads = (t_len + 4 * ATT_BM - 1) / (4 * ATT_BM);
+    a.ldo = ldo;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+    a.status = status;
+    for (int z0 = 0; z0 < n_seq; z0 += 65535) {
+      const int nz = std::min(65535, n_seq - z0);
+      a.beta0 = beta0 + z0;
+      a.o = o + (long long)z0 * t_len * ldo;
+      dim3 grid(2u * (unsigned)a.n_quads * (unsigned)heads, 1, nz);
+      LaunchScope ls("attention", st);
+      attention_pair_tcgen05<<<grid, ATT_THREADS, AttnPairCfg::SMEM_BYTES, st>>>(tq, tk, tv, a);
+    }
+    return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+  }
   if (!map_seq(&tq, q, b, s, h, ldq) || !map_seq(&tk, k, b, s, h, h) || !map_seq(&tv, v, b, s, h, h))
     return BPT_ERR_CUDA;
   AttnArgs a{};

@@ -25,6 +25,8 @@ EXPORTED = (
     "bpt_layer_forward_ws", "bpt_layer_forward_noalloc", "bpt_layer_workspace_bytes_ffn", "bpt_layer_forward_ffn",
     "bpt_layer_forward_host", "bpt_convert_f32_to_bf16",
     "bpt_qkv_projection", "bpt_attention", "bpt_ffn_backward_workspace_bytes", "bpt_ffn_backward",
+    "bpt_attention_lse", "bpt_attention_backward_workspace_bytes", "bpt_attention_backward",
+    "bpt_layer_backward_workspace_bytes", "bpt_layer_backward",
     "bpt_stream_status", "bpt_device_status", "bpt_wait_flag",
     "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
 )
@@ -79,6 +81,16 @@ def lib() -> ctypes.CDLL:
     L.bpt_ffn_backward_workspace_bytes.argtypes = [i] * 4
     L.bpt_ffn_backward.restype = i
     L.bpt_ffn_backward.argtypes = [vp] * 5 + [i] * 4 + [vp] * 6 + [sz, vp]
+    L.bpt_attention_lse.restype = i
+    L.bpt_attention_lse.argtypes = [vp] * 3 + [i] * 5 + [vp, vp, vp]
+    L.bpt_attention_backward_workspace_bytes.restype = sz
+    L.bpt_attention_backward_workspace_bytes.argtypes = [i] * 4
+    L.bpt_attention_backward.restype = i
+    L.bpt_attention_backward.argtypes = [vp] * 6 + [i] * 5 + [vp] * 4 + [sz, vp]
+    L.bpt_layer_backward_workspace_bytes.restype = sz
+    L.bpt_layer_backward_workspace_bytes.argtypes = [i] * 5
+    L.bpt_layer_backward.restype = i
+    L.bpt_layer_backward.argtypes = [vp] * 10 + [i] * 6 + [vp] * 10 + [sz, vp]
     L.bpt_stream_status.restype = i
     L.bpt_stream_status.argtypes = [vp]
     L.bpt_device_status.restype = i
@@ -273,6 +285,73 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int, q_b
                             _ptr(o), _stream(stream))
     _check(r, "bpt_attention")
     return o
+
+
+def attention_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int, causal: bool,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Attention (as `attention`) and each row's log-sum-exp of the scaled
+    scores in log2 units (bpt_attention_lse): returns (O bf16 [b, s, h], lse2
+    fp32 [b, heads, s])."""
+    b, s, h = q.shape
+    o = torch.empty((b, s, h), dtype=torch.bfloat16, device=q.device)
+    lse2 = torch.empty((b, heads, s), dtype=torch.float32, device=q.device)
+    r = lib().bpt_attention_lse(_ptr(q), _ptr(k), _ptr(v), b, s, h, heads, int(bool(causal)), _ptr(o), _ptr(lse2),
+                                _stream(stream))
+    _check(r, "bpt_attention_lse")
+    return o, lse2
+
+
+def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
+                       lse2: torch.Tensor, heads: int, causal: bool,
+                       stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """dQ, dK, dV (bf16 [b, s, h]) of the attention for dO = dL/dO, from the
+    forward's o and lse2 (bpt_attention_backward). Returns {"dq", "dk", "dv"}."""
+    b, s, h = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO)):
+        if t.dtype != torch.bfloat16 or t.shape != q.shape:
+            raise ValueError(f"{name} must be bf16 of shape {tuple(q.shape)}")
+    if lse2.dtype != torch.float32 or tuple(lse2.shape) != (b, heads, s):
+        raise ValueError(f"lse2 must be fp32 of shape {(b, heads, s)}")
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(q), "dv": torch.empty_like(q)}
+    nbytes = int(lib().bpt_attention_backward_workspace_bytes(b, s, h, heads))
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    r = lib().bpt_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse2), b, s, h, heads,
+                                     int(bool(causal)), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(ws),
+                                     ws.numel(), _stream(stream))
+    _check(r, "bpt_attention_backward")
+    return g
+
+
+def layer_backward(x: torch.Tensor, params: dict, dy: torch.Tensor, heads: int, causal: bool,
+                   stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of the layer's output (bpt_layer_backward) for dy = dL/dout
+    (fp32 [b, s, h]): x bf16 [b, s, h] and params as for layer_forward (bf16,
+    FFN width from W1). Returns {"dx", "dWqkv", "dbqkv", "dWo", "dbo", "dW1",
+    "db1", "dW2", "db2"} (fp32)."""
+    b, s, h = x.shape
+    ffn = params["W1"].shape[-1]
+    if x.dtype != torch.bfloat16 or dy.dtype != torch.float32 or dy.shape != x.shape:
+        raise TypeError("x must be bf16 and dy fp32 of the same shape")
+    shapes = {"Wqkv": (h, 3 * h), "bqkv": (3 * h,), "Wo": (h, h), "bo": (h,), "W1": (h, ffn), "b1": (ffn,),
+              "W2": (ffn, h), "b2": (h,)}
+    for name, shape in shapes.items():
+        t = params[name]
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be bf16 of shape {shape}")
+    dev = x.device
+    g = {"dx": torch.empty((b, s, h), dtype=torch.float32, device=dev)}
+    for name, shape in shapes.items():
+        g["d" + name] = torch.empty(shape, dtype=torch.float32, device=dev)
+    nbytes = int(lib().bpt_layer_backward_workspace_bytes(b, s, h, heads, ffn))
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    p = params
+    r = lib().bpt_layer_backward(_ptr(x), _ptr(p["Wqkv"]), _ptr(p["bqkv"]), _ptr(p["Wo"]), _ptr(p["bo"]),
+                                 _ptr(p["W1"]), _ptr(p["b1"]), _ptr(p["W2"]), _ptr(p["b2"]), _ptr(dy), b, s, h, heads,
+                                 ffn, int(bool(causal)), _ptr(g["dx"]), _ptr(g["dWqkv"]), _ptr(g["dbqkv"]),
+                                 _ptr(g["dWo"]), _ptr(g["dbo"]), _ptr(g["dW1"]), _ptr(g["db1"]), _ptr(g["dW2"]),
+                                 _ptr(g["db2"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check(r, "bpt_layer_backward")
+    return g
 
 
 def ffn_backward(hid: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, W2: torch.Tensor, dy: torch.Tensor,

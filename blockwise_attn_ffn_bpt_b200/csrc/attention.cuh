@@ -75,6 +75,7 @@ struct AttnArgs {
   long long ldo;
   float scale_log2; // log2(e) / sqrt(dh)
   int* status;      // status word of the launching stream
+  float* lse2;      // [n_seq][heads][t_len]: m + log2(l) of each row (log2 units); written by the LSE build only
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]: bf16 A read from tensor memory (K-major).
@@ -88,7 +89,9 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-template <int DH>
+// LSE: also write each row's log-sum-exp (args.lse2), for the backward; a
+// separate build so that the forward alone carries nothing for it.
+template <int DH, bool LSE = false>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_fwd_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
@@ -351,6 +354,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const bool row_ok = r < rows_valid[q];
+      // the row's log-sum-exp of the scaled scores, in log2 units: the
+      // (possibly stale) max m plus log2 of the sum l taken against it
+      if constexpr (LSE) {
+        if (row_ok)
+          args.lse2[((long long)(beta - args.beta0) * args.heads + head) * args.t_len + (t - args.t_start)] =
+              m + log2f(l);
+      }
       __nv_bfloat16* orow =
           args.o + ((long long)(beta - args.beta0) * args.t_len + (t - args.t_start)) * args.ldo + head * DH;
 #pragma unroll 1

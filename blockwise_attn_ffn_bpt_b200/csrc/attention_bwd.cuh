@@ -1,0 +1,360 @@
+// Attention backward: gradients dQ, dK, dV of O = softmax(Q K^T / sqrt(dh)) V
+// for one head, blockwise, from the forward's per-row log-sum-exp.
+//
+// Follows the blockwise backward of the BPT paper review (section 3: the
+// blockwise computation is rematerialised for training; Eq. 3 and Algorithm 1
+// give the forward it inverts). One CTA owns one key/value tile of 128 keys of
+// one head of one sequence and visits every query tile that sees it (causal:
+// from the diagonal on). Per query tile i it recomputes
+//     S^T  = K_j Q_i^T                 (scores, keys x queries)
+//     P^T  = 2^(S^T * scale_log2 - lse2_i)   (0 where masked)
+//     dP^T = V_j dO_i^T
+//     dS^T = P^T (dP^T - D_i),  D_i = rowsum(dO_i O_i)
+// and accumulates dV_j += P^T dO_i and dK_j += dS^T Q_i in tensor memory; the
+// query gradient dQ_i += dS K_j (x scale) is added to an fp32 accumulator in
+// global memory. At the end dK_j (x scale) and dV_j are written as bf16.
+//
+// Roles (256 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
+// tile (two-stage ring) with TMA; one thread of warp 1 issues the MMAs; warps
+// 4-7 (one row per thread = one tensor-memory lane) form P and dS, then read the
+// dQ partial and add it to global memory, and finally write dK and dV.
+// Tensor memory: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T over its first
+// 64 columns, then the dQ partial over all 128), dP^T [384, 512) (dS^T over its
+// first 64 columns).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace bpt {
+
+constexpr int AB_BM = 128;  // query rows per tile
+constexpr int AB_BN = 128;  // keys per CTA
+constexpr int AB_THREADS = 256;
+constexpr int AB_T_DV = 0, AB_T_DK = 128, AB_T_ST = 256, AB_T_DP = 384;
+
+template <int DH>
+struct AttnBwdCfg {
+  static_assert(DH == 64 || DH == 128, "dh must be 64 or 128");
+  static constexpr int ATOM = 128 * 128;            // [128 rows][64 bf16] swizzled box
+  static constexpr int TILE = 128 * DH * 2;         // one K, V, Q or dO tile
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_QDO = OFF_V + TILE;      // [2 stages][Q, dO]
+  static constexpr int OFF_DS = OFF_QDO + 4 * TILE;  // dS^T [128 keys][128 queries] bf16, two atoms
+  static constexpr int OFF_LD = OFF_DS + 2 * ATOM;   // lse2 and D of the query tile, 2 x 128 fp32
+  static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
+  static constexpr int USED = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM_BYTES = USED;
+  static_assert(USED <= 232448, "shared memory budget");
+};
+
+struct AttnBwdArgs {
+  int s, heads, causal;
+  int beta0;                // first sequence of this launch
+  int n_kv;                 // key/value tiles per (sequence, head)
+  const float* lse2;        // [b][heads][s]: max + log2(sum) of the forward, in log2 units
+  const float* dsum;        // [b][heads][s]: D = rowsum(dO O)
+  float* dq;                // [b][s][h] fp32 accumulator (zeroed by the caller)
+  __nv_bfloat16* dk;        // rows (beta * s + t), ld_kv elements apart, head columns
+  __nv_bfloat16* dv;
+  long long ld_kv;
+  int h;
+  float scale;              // 1 / sqrt(dh)
+  float scale_log2;         // log2(e) / sqrt(dh)
+  int* status;
+};
+
+__device__ __forceinline__ void ab_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void ab_named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void ab_red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <int DH>
+__global__ void __launch_bounds__(AB_THREADS, 1)
+    attention_bwd_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                          const AttnBwdArgs args) {
+  using C = AttnBwdCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  const uint32_t kv_full = smem_addr(bars + 0);
+  const uint32_t qdo_full0 = smem_addr(bars + 1);   // [2]
+  const uint32_t qdo_empty0 = smem_addr(bars + 3);  // [2]
+  const uint32_t s_ready = smem_addr(bars + 5);
+  const uint32_t p_ready = smem_addr(bars + 6);
+  const uint32_t dq_ready = smem_addr(bars + 7);
+  const uint32_t dq_free = smem_addr(bars + 8);
+  const uint32_t kv_done = smem_addr(bars + 9);
+  const uint32_t mma_done = smem_addr(bars + 10);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  const Abort abort_flag{reinterpret_cast<volatile int*>(bars + 12), args.status};
+  float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LD);
+  float* s_dsum = s_lse + 128;
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const uint32_t sbase = smem_addr(smem);
+
+  // grid: x = (head, key tile), heaviest key tiles first when causal; z = sequence
+  const int head = (int)blockIdx.x % args.heads;
+  const int rank = (int)blockIdx.x / args.heads;
+  const int jt = rank;  // key tile 0 sees the most query tiles
+  const int beta = args.beta0 + blockIdx.z;
+  const int j0 = jt * AB_BN;
+  const int n_q = (args.s + AB_BM - 1) / AB_BM;
+  const int i_first = args.causal ? jt : 0;  // query tiles before the key tile's diagonal see none of its keys
+  const int n_it = n_q - i_first;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(qdo_full0 + 8 * i, 1);
+      mbar_init(qdo_empty0 + 8 * i, 1);
+    }
+    mbar_init(s_ready, 1);
+    mbar_init(p_ready, 4);
+    mbar_init(dq_ready, 1);
+    mbar_init(dq_free, 4);
+    mbar_init(kv_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag.flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmdO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && n_it > 0) {
+      // ------------------------------------------------------------ TMA producer
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+#pragma unroll
+      for (int a = 0; a < DH / 64; ++a) {
+        tma_load_3d(sbase + C::OFF_K + a * C::ATOM, &tmK, kv_full, head * DH + a * 64, j0, beta);
+        tma_load_3d(sbase + C::OFF_V + a * C::ATOM, &tmV, kv_full, head * DH + a * 64, j0, beta);
+      }
+      uint32_t issued = 0, par = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(qdo_empty0 + 8 * st, ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(qdo_full0 + 8 * st, 2 * C::TILE);
+        const int i0 = (i_first + it) * AB_BM;
+        const uint32_t q_s = sbase + C::OFF_QDO + st * 2 * C::TILE;
+#pragma unroll
+        for (int a = 0; a < DH / 64; ++a) {
+          tma_load_3d(q_s + a * C::ATOM, &tmQ, qdo_full0 + 8 * st, head * DH + a * 64, i0, beta);
+          tma_load_3d(q_s + C::TILE + a * C::ATOM, &tmdO, qdo_full0 + 8 * st, head * DH + a * 64, i0, beta);
+        }
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (ph << st);
+      }
+      volatile int dummy = 0;
+      const Abort drain{&dummy, args.status};
+      mbar_wait(kv_full, 0, drain);
+      for (int i = 0; i < 2; ++i)
+        if (issued & (1u << i)) mbar_wait(qdo_full0 + 8 * i, (par >> i) & 1u, drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_it > 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t id_kmaj = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both operands K-major (dh)
+      const uint32_t id_bmn = idesc_bf16_f32(128, DH, 0, 1);    // dV, dK: A from tensor memory, B MN-major
+      const uint32_t id_amn = idesc_bf16_f32(128, DH, 1, 1);    // dQ: dS and K both MN-major
+      const uint32_t k_s = sbase + C::OFF_K, v_s = sbase + C::OFF_V, ds_s = sbase + C::OFF_DS;
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it & 1;
+        ok = mbar_wait(qdo_full0 + 8 * st, (uint32_t)(it >> 1) & 1u, abort_flag);
+        // the previous tile's dQ partial must be read out before S^T overwrites it
+        if (ok && it > 0) ok = mbar_wait(dq_free, (uint32_t)(it - 1) & 1u, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t q_s = sbase + C::OFF_QDO + st * 2 * C::TILE, do_s = q_s + C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+          mma_bf16_ss(tmem_base + AB_T_ST, smem_desc_sw128(k_s + off, 16, 1024), smem_desc_sw128(q_s + off, 16, 1024),
+                      id_kmaj, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+          mma_bf16_ss(tmem_base + AB_T_DP, smem_desc_sw128(v_s + off, 16, 1024),
+                      smem_desc_sw128(do_s + off, 16, 1024), id_kmaj, kk > 0);
+        }
+        mma_commit(s_ready);
+        if (!mbar_wait(p_ready, (uint32_t)it & 1u, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q (A from tensor memory: 16 queries = 8 columns per step)
+#pragma unroll
+        for (int kk = 0; kk < AB_BM / 16; ++kk)
+          ab_mma_ts(tmem_base + AB_T_DV, tmem_base + AB_T_ST + kk * 8,
+                    smem_desc_sw128(do_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
+#pragma unroll
+        for (int kk = 0; kk < AB_BM / 16; ++kk)
+          ab_mma_ts(tmem_base + AB_T_DK, tmem_base + AB_T_DP + kk * 8,
+                    smem_desc_sw128(q_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
+        // dQ partial = dS K over this key tile (16 keys per step), into the S^T columns
+#pragma unroll
+        for (int kk = 0; kk < AB_BN / 16; ++kk)
+          mma_bf16_ss(tmem_base + AB_T_ST, smem_desc_sw128(ds_s + kk * 16 * 128, C::ATOM, 1024),
+                      smem_desc_sw128(k_s + kk * 16 * 128, C::ATOM, 1024), id_amn, kk > 0);
+        mma_commit(dq_ready);
+        mma_commit(qdo_empty0 + 8 * st);
+      }
+      mma_commit(kv_done);
+      mma_commit(mma_done);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ P, dS, dQ, epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // tensor-memory lane: a key (P, dS) or a query (dQ)
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int key = j0 + r;
+    const float sl2 = args.scale_log2;
+    const long long bh = (long long)beta * args.heads + head;
+    // Every warp runs every iteration and both named barriers of it; a wait that
+    // gives up only switches the work off (the waits are bounded, and the
+    // barriers never see a warp missing).
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = (i_first + it) * AB_BM;
+      // the query tile's statistics, once per tile (the previous tile's readers are done)
+      ab_named_sync(1, 128);
+      {
+        const int t = i0 + r;
+        s_lse[r] = t < args.s ? args.lse2[bh * args.s + t] : 0.0f;
+        s_dsum[r] = t < args.s ? args.dsum[bh * args.s + t] : 0.0f;
+      }
+      ab_named_sync(1, 128);
+      ok = ok && warp_wait(s_ready, (uint32_t)it & 1u, abort_flag);
+      if (!ok) continue;
+      tc_fence_after();
+      // a query column q is used when it is a real row and (causal) not before this key
+      const bool key_ok = key < args.s;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dp[32];
+        tmem_load32x2(tmem_base + AB_T_ST + c * 32 + lane_base, tmem_base + AB_T_DP + c * 32 + lane_base, sv, dp);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int qc = c * 32 + 2 * x + e;
+            const int q = i0 + qc;
+            const bool use = key_ok && q < args.s && (!args.causal || key <= q);
+            const float p = use ? ex2_approx(__uint_as_float(sv[2 * x + e]) * sl2 - s_lse[qc]) : 0.0f;
+            p2[e] = p;
+            d2[e] = use ? p * (__uint_as_float(dp[2 * x + e]) - s_dsum[qc]) : 0.0f;
+          }
+          pk[x] = pack_bf16x2(p2[0], p2[1]);
+          dk[x] = pack_bf16x2(d2[0], d2[1]);
+        }
+        // P^T and dS^T (bf16 pairs) over the first 64 columns of their regions; the
+        // columns written here were loaded in this or an earlier chunk
+        tmem_store16(tmem_base + AB_T_ST + c * 16 + lane_base, pk);
+        tmem_store16(tmem_base + AB_T_DP + c * 16 + lane_base, dk);
+        // dS^T row of this key into the 128B-swizzled [keys][queries] layout of the dQ operand
+        const uint32_t row = sbase + C::OFF_DS + (c >> 1) * C::ATOM + r * 128;
+#pragma unroll
+        for (int t4 = 0; t4 < 4; ++t4) {
+          const int chunk = (c & 1) * 4 + t4;
+          st_shared_v4(row + (uint32_t)((chunk ^ (r & 7)) * 16), dk[4 * t4], dk[4 * t4 + 1], dk[4 * t4 + 2],
+                       dk[4 * t4 + 3]);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready);
+      // dQ partial of this query tile: lane = query row
+      ok = warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
+      if (!ok) continue;
+      tc_fence_after();
+      {
+        const int q = i0 + r;
+        float* dst = args.dq + ((long long)beta * args.s + q) * args.h + head * DH;
+#pragma unroll 1
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t o[32];
+          tmem_load32(tmem_base + AB_T_ST + c * 32 + lane_base, o);
+          if (q < args.s) {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              ab_red_add_v4(dst + c * 32 + 4 * x, __uint_as_float(o[4 * x]) * args.scale,
+                            __uint_as_float(o[4 * x + 1]) * args.scale, __uint_as_float(o[4 * x + 2]) * args.scale,
+                            __uint_as_float(o[4 * x + 3]) * args.scale);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+    }
+    // dK (x scale) and dV of this key tile: lane = key
+    if (ok && n_it > 0 && warp_wait(kv_done, 0, abort_flag)) {
+      tc_fence_after();
+      // the loads are warp-collective: every lane loads, only real keys store
+      const bool key_row = key < args.s;
+      __nv_bfloat16* dkr = args.dk + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
+      __nv_bfloat16* dvr = args.dv + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t a[32], b[32];
+        tmem_load32x2(tmem_base + AB_T_DK + c * 32 + lane_base, tmem_base + AB_T_DV + c * 32 + lane_base, a, b);
+        if (key_row) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float* fa = reinterpret_cast<const float*>(a) + 8 * x;
+            const float* fb = reinterpret_cast<const float*>(b) + 8 * x;
+            const float sc = args.scale;
+            st_global_v4(dkr + c * 32 + 8 * x, pack_bf16x2(fa[0] * sc, fa[1] * sc), pack_bf16x2(fa[2] * sc, fa[3] * sc),
+                         pack_bf16x2(fa[4] * sc, fa[5] * sc), pack_bf16x2(fa[6] * sc, fa[7] * sc));
+            st_global_v4(dvr + c * 32 + 8 * x, pack_bf16x2(fb[0], fb[1]), pack_bf16x2(fb[2], fb[3]),
+                         pack_bf16x2(fb[4], fb[5]), pack_bf16x2(fb[6], fb[7]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && n_it > 0) {
+      volatile int dummy = 0;
+      mbar_wait(mma_done, 0, Abort{&dummy, args.status});
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace bpt

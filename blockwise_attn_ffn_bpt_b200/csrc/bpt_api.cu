@@ -29,6 +29,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_bwd.cuh"
 #include "attention_pair.cuh"
 #include "bpt.h"
 #include "ffn_chain.cuh"
@@ -196,17 +197,28 @@ int check_device(int* sms) {
                    cudaFuncSetAttribute(attention_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         AttnCfg<64>::SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        AttnCfg<128>::SMEM_BYTES) == cudaSuccess;
+                                        AttnCfg<128>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_fwd_tcgen05<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnCfg<64>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_fwd_tcgen05<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnCfg<128>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_bwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnBwdCfg<64>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(attention_bwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        AttnBwdCfg<128>::SMEM_BYTES) == cudaSuccess;
       if (!attrs) return BPT_ERR_CUDA;
       // the attention kernel splits its registers between warpgroups assuming
       // it was built with exactly ATT_REGS_LAUNCH per thread; any other build
       // is never launched (its register requests could not be met)
-      cudaFuncAttributes fa64{}, fa128{}, fap{};
+      cudaFuncAttributes fa64{}, fa128{}, fl64{}, fl128{}, fap{};
       if (cudaFuncGetAttributes(&fa64, attention_fwd_tcgen05<64>) != cudaSuccess ||
           cudaFuncGetAttributes(&fa128, attention_fwd_tcgen05<128>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fl64, attention_fwd_tcgen05<64, true>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fl128, attention_fwd_tcgen05<128, true>) != cudaSuccess ||
           cudaFuncGetAttributes(&fap, attention_pair_tcgen05) != cudaSuccess)
         return BPT_ERR_CUDA;
-      if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH || fap.numRegs != ATT_REGS_LAUNCH)
+      if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH || fl64.numRegs != ATT_REGS_LAUNCH ||
+          fl128.numRegs != ATT_REGS_LAUNCH || fap.numRegs != ATT_REGS_LAUNCH)
         d.ok = false;
     }
     d.checked = true;
@@ -648,10 +660,10 @@ int launch_colsum(const T* src, long long rows, int cols, long long ld, float* o
 // beta0 .. beta0 + n_seq - 1; q rows have `ldq` elements between them.
 int launch_attention(const void* q, long long ldq, const void* k, const void* v, int b, int s, int h, int heads,
                      int causal, int beta0, int n_seq, int t_start, int t_len, __nv_bfloat16* o, long long ldo,
-                     cudaStream_t st, int* status) {
+                     cudaStream_t st, int* status, float* lse2 = nullptr) {
   const int dh = h / heads;
   CUtensorMap tq, tk, tv;
-  if (BPT_PAIR_ATTENTION && dh == 128) {
+  if (BPT_PAIR_ATTENTION && dh == 128 && lse2 == nullptr) {
     // K halves are [64 keys][64 cols] boxes, Q and the V halves [128][64]
     if (!map_seq(&tq, q, b, s, h, ldq, 128) || !map_seq(&tk, k, b, s, h, h, 64) || !map_seq(&tv, v, b, s, h, h, 128))
       return BPT_ERR_CUDA;
@@ -691,13 +703,123 @@ int launch_attention(const void* q, long long ldq, const void* k, const void* v,
     const int nz = std::min(65535, n_seq - z0);
     a.beta0 = beta0 + z0;
     a.o = o + (long long)z0 * t_len * ldo;
+    a.lse2 = lse2 ? lse2 + (long long)z0 * heads * t_len : nullptr;
     dim3 grid((unsigned)a.n_pairs * (unsigned)heads, 1, nz);
     LaunchScope ls("attention", st);
-    if (dh == 64)
+    if (lse2 != nullptr) {
+      if (dh == 64)
+        attention_fwd_tcgen05<64, true><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+      else
+        attention_fwd_tcgen05<128, true><<<grid, ATT_THREADS, AttnCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+    } else if (dh == 64) {
       attention_fwd_tcgen05<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, a);
-    else
+    } else {
       attention_fwd_tcgen05<128><<<grid, ATT_THREADS, AttnCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, a);
+    }
   }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+// D = rowsum(dO O) of every (row, head): dsum[(beta * heads + head) * s + t],
+// fp32 sums of the bf16 products, one thread per (row, head).
+__global__ void attn_dsum_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                                 long long ld, long long rows, int s, int heads, int dh, float* __restrict__ dsum) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * heads) return;
+  const int head = (int)(i % heads);
+  const long long row = i / heads;
+  const __nv_bfloat16* po = o + row * ld + (long long)head * dh;
+  const __nv_bfloat16* pd = dO + row * ld + (long long)head * dh;
+  float acc = 0.0f;
+  for (int c = 0; c < dh; c += 8) {
+    const uint4 a = *reinterpret_cast<const uint4*>(po + c);
+    const uint4 d = *reinterpret_cast<const uint4*>(pd + c);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 fa = __bfloat1622float2(a2[k]), fd = __bfloat1622float2(d2[k]);
+      acc = fmaf(fa.x, fd.x, acc);
+      acc = fmaf(fa.y, fd.y, acc);
+    }
+  }
+  const long long beta = row / s, t = row - beta * s;
+  dsum[(beta * heads + head) * s + t] = acc;
+}
+
+// dst[r * ld_dst + c] = bf16(src[r * cols + c]) for c < cols (cols a multiple of 8).
+__global__ void rows_f32_to_bf16_kernel(const float* __restrict__ src, long long rows, int cols,
+                                        __nv_bfloat16* __restrict__ dst, long long ld_dst) {
+  const long long per_row = cols / 8;
+  const long long n = rows * per_row;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / per_row, c = (i - r * per_row) * 8;
+    const float4 a = *reinterpret_cast<const float4*>(src + r * cols + c);
+    const float4 b = *reinterpret_cast<const float4*>(src + r * cols + c + 4);
+    st_global_v4(dst + r * ld_dst + c, pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                 pack_bf16x2(b.z, b.w));
+  }
+}
+
+// Gradients of the attention of b sequences: dK, dV (bf16, ld_kv apart) and
+// the fp32 dQ accumulator (rows h apart, zero on entry) from Q, K, V (ld_in
+// apart), dO (ld_do apart), the forward's lse2 and D = rowsum(dO O).
+int launch_attention_bwd(const void* q, const void* k, const void* v, long long ld_in, const void* dO,
+                         long long ld_do, const float* lse2, const float* dsum, float* dq, __nv_bfloat16* dk,
+                         __nv_bfloat16* dv, long long ld_kv, int b, int s, int h, int heads, int causal,
+                         cudaStream_t st, int* status) {
+  if ((long long)b * s == 0) return BPT_OK;
+  const int dh = h / heads;
+  CUtensorMap tq, tk, tv, td;
+  if (!map_seq(&tq, q, b, s, h, ld_in) || !map_seq(&tk, k, b, s, h, ld_in) || !map_seq(&tv, v, b, s, h, ld_in) ||
+      !map_seq(&td, dO, b, s, h, ld_do))
+    return BPT_ERR_CUDA;
+  AttnBwdArgs a{};
+  a.s = s;
+  a.heads = heads;
+  a.causal = causal ? 1 : 0;
+  a.n_kv = (s + AB_BN - 1) / AB_BN;
+  a.lse2 = lse2;
+  a.dsum = dsum;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ld_kv = ld_kv;
+  a.h = h;
+  a.scale = (float)(1.0 / std::sqrt((double)dh));
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  a.status = status;
+  for (int z0 = 0; z0 < b; z0 += 65535) {
+    a.beta0 = z0;
+    dim3 grid((unsigned)a.n_kv * (unsigned)heads, 1, std::min(65535, b - z0));
+    LaunchScope ls("attention_bwd", st);
+    if (dh == 64)
+      attention_bwd_tcgen05<64><<<grid, AB_THREADS, AttnBwdCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, td, a);
+    else
+      attention_bwd_tcgen05<128><<<grid, AB_THREADS, AttnBwdCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, td, a);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+int launch_dsum(const void* o, const void* dO, long long ld, long long rows, int s, int heads, int dh, float* dsum,
+                cudaStream_t st) {
+  const long long n = rows * heads;
+  if (n <= 0) return BPT_OK;
+  LaunchScope ls("attention_dsum", st);
+  attn_dsum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(o),
+                                                                 reinterpret_cast<const __nv_bfloat16*>(dO), ld, rows,
+                                                                 s, heads, dh, dsum);
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
+int launch_rows_to_bf16(const float* src, long long rows, int cols, void* dst, long long ld_dst, int sms,
+                        cudaStream_t st) {
+  if (rows <= 0) return BPT_OK;
+  const long long n = rows * (cols / 8);
+  const long long blocks = std::min<long long>((n + 255) / 256, (long long)sms * 8);
+  LaunchScope ls("f32_to_bf16", st);
+  rows_f32_to_bf16_kernel<<<(int)blocks, 256, 0, st>>>(src, rows, cols, reinterpret_cast<__nv_bfloat16*>(dst),
+                                                       ld_dst);
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
@@ -1259,42 +1381,11 @@ int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stre
   return launch_convert(src, dst, n, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t bpt_ffn_backward_workspace_bytes(int rows, int h, int ffn, int chunk_rows) {
-  if (rows <= 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return 0;
-  const long long R = ffn_bwd_chunk(rows, chunk_rows);
-  return 2 * align_up((size_t)R * h * 2, 1024) + 2 * align_up((size_t)R * ffn * 2, 1024);
-}
-
-int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy, int rows,
-                     int h, int ffn, int chunk_rows, float* dhid, float* dW1, float* db1, float* dW2, float* db2,
-                     void* workspace, size_t ws_bytes, void* stream) {
-  if (rows < 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return BPT_ERR_SHAPE;
-  if ((long long)h * ffn > 0x7fffffffLL || (long long)rows * std::max(h, ffn) > (1LL << 40)) return BPT_ERR_SHAPE;
-  if (rows == 0) return BPT_OK;
-  const void* ptrs[12] = {hid, W1, b1, W2, dy, dhid, dW1, db1, dW2, db2, workspace, nullptr};
-  for (int i = 0; i < 11; ++i)
-    if (!ptrs[i]) return BPT_ERR_NULL;
-  for (int i = 0; i < 11; ++i)
-    if (!aligned16(ptrs[i])) return BPT_ERR_ALIGN;
-  const long long R = ffn_bwd_chunk(rows, chunk_rows);
-  const size_t need = bpt_ffn_backward_workspace_bytes(rows, h, ffn, chunk_rows);
-  if (ws_bytes < need) return BPT_ERR_NOMEM;
-  // outputs must not overlap the inputs or one another
-  const Range in[5] = {rng(hid, (size_t)rows * h * 4), rng(W1, (size_t)h * ffn * 2), rng(b1, (size_t)ffn * 2),
-                       rng(W2, (size_t)ffn * h * 2), rng(dy, (size_t)rows * h * 4)};
-  const Range outs[6] = {rng(dhid, (size_t)rows * h * 4), rng(dW1, (size_t)h * ffn * 4), rng(db1, (size_t)ffn * 4),
-                         rng(dW2, (size_t)ffn * h * 4), rng(db2, (size_t)h * 4), rng(workspace, need)};
-  for (int i = 0; i < 6; ++i) {
-    for (const Range& r : in)
-      if (overlap(outs[i], r)) return BPT_ERR_ALIAS;
-    for (int j = i + 1; j < 6; ++j)
-      if (overlap(outs[i], outs[j])) return BPT_ERR_ALIAS;
-  }
-  int sms = 0;
-  BPT_TRY(check_device(&sms));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int* status = nullptr;
-  BPT_TRY(stream_status_word(st, &status));
+// The FFN block's backward over `rows` rows in chunks of R rows (workspace as
+// bpt_ffn_backward_workspace_bytes sizes it for R).
+int ffn_backward_impl(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy,
+                      long long rows, int h, int ffn, long long R, float* dhid, float* dW1, float* db1, float* dW2,
+                      float* db2, void* workspace, int sms, cudaStream_t st, int* status) {
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(ws + align_up((size_t)R * h * 2, 1024));
@@ -1337,6 +1428,262 @@ int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const voi
     BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(U, ffn, dyb, h, ffn, h, n, a, sms, st, status, "bwd_dW2")));
     BPT_TRY(launch_colsum(da, n, ffn, ffn, db1, acc, st));
     BPT_TRY(launch_colsum(dy + r0 * h, n, h, h, db2, acc, st));
+  }
+  return BPT_OK;
+}
+
+
+size_t bpt_ffn_backward_workspace_bytes(int rows, int h, int ffn, int chunk_rows) {
+  if (rows <= 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return 0;
+  const long long R = ffn_bwd_chunk(rows, chunk_rows);
+  return 2 * align_up((size_t)R * h * 2, 1024) + 2 * align_up((size_t)R * ffn * 2, 1024);
+}
+
+int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy, int rows,
+                     int h, int ffn, int chunk_rows, float* dhid, float* dW1, float* db1, float* dW2, float* db2,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (rows < 0 || h <= 0 || h % 64 || ffn <= 0 || ffn % 64 || chunk_rows < 0) return BPT_ERR_SHAPE;
+  if ((long long)h * ffn > 0x7fffffffLL || (long long)rows * std::max(h, ffn) > (1LL << 40)) return BPT_ERR_SHAPE;
+  if (rows == 0) return BPT_OK;
+  const void* ptrs[12] = {hid, W1, b1, W2, dy, dhid, dW1, db1, dW2, db2, workspace, nullptr};
+  for (int i = 0; i < 11; ++i)
+    if (!ptrs[i]) return BPT_ERR_NULL;
+  for (int i = 0; i < 11; ++i)
+    if (!aligned16(ptrs[i])) return BPT_ERR_ALIGN;
+  const long long R = ffn_bwd_chunk(rows, chunk_rows);
+  const size_t need = bpt_ffn_backward_workspace_bytes(rows, h, ffn, chunk_rows);
+  if (ws_bytes < need) return BPT_ERR_NOMEM;
+  // outputs must not overlap the inputs or one another
+  const Range in[5] = {rng(hid, (size_t)rows * h * 4), rng(W1, (size_t)h * ffn * 2), rng(b1, (size_t)ffn * 2),
+                       rng(W2, (size_t)ffn * h * 2), rng(dy, (size_t)rows * h * 4)};
+  const Range outs[6] = {rng(dhid, (size_t)rows * h * 4), rng(dW1, (size_t)h * ffn * 4), rng(db1, (size_t)ffn * 4),
+                         rng(dW2, (size_t)ffn * h * 4), rng(db2, (size_t)h * 4), rng(workspace, need)};
+  for (int i = 0; i < 6; ++i) {
+    for (const Range& r : in)
+      if (overlap(outs[i], r)) return BPT_ERR_ALIAS;
+    for (int j = i + 1; j < 6; ++j)
+      if (overlap(outs[i], outs[j])) return BPT_ERR_ALIAS;
+  }
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  return ffn_backward_impl(hid, W1, b1, W2, dy, rows, h, ffn, R, dhid, dW1, db1, dW2, db2, workspace, sms, st,
+                           status);
+}
+
+int bpt_attention_lse(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int causal,
+                      void* o, float* lse2, void* stream) {
+  BPT_TRY(check_shape(b, s, h, heads));
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[5] = {q, k, v, o, lse2};
+  for (const void* p : ptrs)
+    if (!p) return BPT_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return BPT_ERR_ALIGN;
+  const size_t act = (size_t)b * s * h * 2;
+  if (overlap(rng(lse2, (size_t)b * heads * s * 4), rng(o, act))) return BPT_ERR_ALIAS;
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  return launch_attention(q, h, k, v, b, s, h, heads, causal, 0, b, 0, s, reinterpret_cast<__nv_bfloat16*>(o), h,
+                          st, status, lse2);
+}
+
+size_t bpt_attention_backward_workspace_bytes(int b, int s, int h, int heads) {
+  if (check_shape(b, s, h, heads) != BPT_OK) return 0;
+  return align_up((size_t)b * heads * s * 4, 1024) + align_up((size_t)b * s * h * 4, 1024);
+}
+
+int bpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                           const float* lse2, int b, int s, int h, int heads, int causal, void* dq, void* dk,
+                           void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  BPT_TRY(check_shape(b, s, h, heads));
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[10] = {q, k, v, o, dO, lse2, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!p) return BPT_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return BPT_ERR_ALIGN;
+  const size_t need = bpt_attention_backward_workspace_bytes(b, s, h, heads);
+  if (ws_bytes < need) return BPT_ERR_NOMEM;
+  const size_t act = (size_t)b * s * h * 2;
+  const Range in[6] = {rng(q, act), rng(k, act), rng(v, act), rng(o, act), rng(dO, act),
+                       rng(lse2, (size_t)b * heads * s * 4)};
+  const Range outs[4] = {rng(dq, act), rng(dk, act), rng(dv, act), rng(workspace, need)};
+  for (int i = 0; i < 4; ++i) {
+    for (const Range& r : in)
+      if (overlap(outs[i], r)) return BPT_ERR_ALIAS;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], outs[j])) return BPT_ERR_ALIAS;
+  }
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  float* dsum = reinterpret_cast<float*>(ws);
+  float* dq32 = reinterpret_cast<float*>(ws + align_up((size_t)b * heads * s * 4, 1024));
+  const long long rows = (long long)b * s;
+  if (cudaMemsetAsync(dq32, 0, (size_t)rows * h * 4, st) != cudaSuccess) return BPT_ERR_CUDA;
+  BPT_TRY(launch_dsum(o, dO, h, rows, s, heads, h / heads, dsum, st));
+  BPT_TRY(launch_attention_bwd(q, k, v, h, dO, h, lse2, dsum, dq32, reinterpret_cast<__nv_bfloat16*>(dk),
+                               reinterpret_cast<__nv_bfloat16*>(dv), h, b, s, h, heads, causal, st, status));
+  return launch_rows_to_bf16(dq32, rows, h, dq, h, sms, st);
+}
+
+// Workspace of the layer backward: the recomputed forward (Q, K, V, O, the
+// log-sum-exp, hid and its bf16 copy), the gradients on the way (dhid and its
+// bf16 copy, dO, D, the fp32 dQ accumulator, [dQ | dK | dV]) and the FFN
+// backward's chunk buffers.
+struct LayerBwdLayout {
+  size_t q, k, v, o, lse, hid, hb, dhid, dhb, dO, dsum, dq32, dqkv, ffn, total;
+  long long R;
+};
+
+LayerBwdLayout layer_bwd_layout(int b, int s, int h, int heads, int ffn) {
+  LayerBwdLayout L{};
+  const size_t rows = (size_t)b * s;
+  const size_t act = align_up(rows * h * 2, 1024), act32 = align_up(rows * h * 4, 1024);
+  const size_t stat = align_up((size_t)b * heads * s * 4, 1024);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += bytes;
+    return o;
+  };
+  L.q = take(act);
+  L.k = take(act);
+  L.v = take(act);
+  L.o = take(act);
+  L.lse = take(stat);
+  L.hid = take(act32);  // later the fp32 dQ accumulator (hid is dead once dhid is known)
+  L.dq32 = L.hid;
+  L.hb = take(act);
+  L.dhid = take(act32);
+  L.dhb = take(act);
+  L.dO = take(act);
+  L.dsum = take(stat);
+  L.dqkv = take(align_up(rows * 3 * h * 2, 1024));
+  L.R = ffn_bwd_chunk((int)std::min<size_t>(rows, 0x7fffffff), 0);
+  L.ffn = take(bpt_ffn_backward_workspace_bytes((int)std::min<size_t>(rows, 0x7fffffff), h, ffn, 0));
+  L.total = off;
+  return L;
+}
+
+size_t bpt_layer_backward_workspace_bytes(int b, int s, int h, int heads, int ffn) {
+  if (check_shape(b, s, h, heads) != BPT_OK || ffn <= 0 || ffn % 64 || (long long)b * s == 0) return 0;
+  return layer_bwd_layout(b, s, h, heads, ffn).total;
+}
+
+int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                       const void* W1, const void* b1, const void* W2, const void* b2, const float* dy, int b, int s,
+                       int h, int heads, int ffn, int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo,
+                       float* dbo, float* dW1, float* db1, float* dW2, float* db2, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  BPT_TRY(check_shape(b, s, h, heads));
+  if (ffn <= 0 || ffn % 64 || (long long)h * ffn > 0x7fffffffLL) return BPT_ERR_SHAPE;
+  if ((long long)b * s == 0) return BPT_OK;
+  const void* ptrs[20] = {x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, dx, dWqkv, dbqkv, dWo, dbo, dW1, db1, dW2, db2,
+                          workspace};
+  for (const void* p : ptrs)
+    if (!p) return BPT_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return BPT_ERR_ALIGN;
+  const LayerBwdLayout L = layer_bwd_layout(b, s, h, heads, ffn);
+  if (ws_bytes < L.total) return BPT_ERR_NOMEM;
+  const long long rows = (long long)b * s;
+  const Range in[10] = {rng(x, (size_t)rows * h * 2),     rng(Wqkv, (size_t)h * 3 * h * 2), rng(bqkv, (size_t)3 * h * 2),
+                        rng(Wo, (size_t)h * h * 2),       rng(bo, (size_t)h * 2),           rng(W1, (size_t)h * ffn * 2),
+                        rng(b1, (size_t)ffn * 2),         rng(W2, (size_t)ffn * h * 2),     rng(b2, (size_t)h * 2),
+                        rng(dy, (size_t)rows * h * 4)};
+  const Range outs[10] = {rng(dx, (size_t)rows * h * 4), rng(dWqkv, (size_t)h * 3 * h * 4), rng(dbqkv, (size_t)3 * h * 4),
+                          rng(dWo, (size_t)h * h * 4),   rng(dbo, (size_t)h * 4),           rng(dW1, (size_t)h * ffn * 4),
+                          rng(db1, (size_t)ffn * 4),     rng(dW2, (size_t)ffn * h * 4),     rng(db2, (size_t)h * 4),
+                          rng(workspace, L.total)};
+  for (int i = 0; i < 10; ++i) {
+    for (const Range& r : in)
+      if (overlap(outs[i], r)) return BPT_ERR_ALIAS;
+    for (int j = i + 1; j < 10; ++j)
+      if (overlap(outs[i], outs[j])) return BPT_ERR_ALIAS;
+  }
+  int sms = 0;
+  BPT_TRY(check_device(&sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  BPT_TRY(stream_status_word(st, &status));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  const int dh = h / heads;
+
+  // the forward again (rematerialised): Q, K, V; O and each row's log-sum-exp; hid
+  {
+    GemmArgs a{};
+    a.bias = bqkv;
+    a.q = bf(L.q);
+    a.ldq = h;
+    a.k = bf(L.k);
+    a.v = bf(L.v);
+    a.ldkv = h;
+    a.h = h;
+    BPT_TRY(launch_gemm<EPI_QKV>(x, rows, h, h, Wqkv, 3LL * h, a, sms, st, status, "bwd_qkv"));
+  }
+  BPT_TRY(launch_attention(bf(L.q), h, bf(L.k), bf(L.v), b, s, h, heads, causal, 0, b, 0, s, bf(L.o), h, st, status,
+                           f32(L.lse)));
+  {
+    GemmArgs a{};
+    a.resid = x;
+    a.ld_resid = h;
+    a.hid = f32(L.hid);
+    a.ld_hid = h;
+    a.bias = bo;
+    a.dst = bf(L.hb);
+    a.ld_dst = h;
+    BPT_TRY(launch_gemm<EPI_OUTPROJ>(bf(L.o), rows, h, h, Wo, h, a, sms, st, status, "bwd_outproj"));
+  }
+  // FFN block: dhid, dW1, db1, dW2, db2
+  BPT_TRY(ffn_backward_impl(f32(L.hid), W1, b1, W2, dy, rows, h, ffn, L.R, f32(L.dhid), dW1, db1, dW2, db2,
+                            ws + L.ffn, sms, st, status));
+  // out-projection: dbo = sum dhid, dWo = O^T dhid, dO = dhid Wo^T
+  BPT_TRY(launch_colsum(f32(L.dhid), rows, h, h, dbo, 0, st));
+  BPT_TRY(launch_convert(f32(L.dhid), bf(L.dhb), rows * h, sms, st));
+  {
+    GemmArgs a{};
+    a.out = dWo;
+    a.ld_out = h;
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(bf(L.o), h, bf(L.dhb), h, h, h, rows, a, sms, st, status, "bwd_dWo")));
+    a = GemmArgs{};
+    a.dst = bf(L.dO);
+    a.ld_dst = h;
+    BPT_TRY((launch_gemm_t<EPI_BWD_DA, 0, 0>(bf(L.dhb), h, Wo, h, rows, h, h, a, sms, st, status, "bwd_dO")));
+  }
+  // attention: dQ, dK, dV into [dQ | dK | dV]
+  float* dq32 = f32(L.dq32);
+  __nv_bfloat16* dqkv = bf(L.dqkv);
+  if (cudaMemsetAsync(dq32, 0, (size_t)rows * h * 4, st) != cudaSuccess) return BPT_ERR_CUDA;
+  BPT_TRY(launch_dsum(bf(L.o), bf(L.dO), h, rows, s, heads, dh, f32(L.dsum), st));
+  BPT_TRY(launch_attention_bwd(bf(L.q), bf(L.k), bf(L.v), h, bf(L.dO), h, f32(L.lse), f32(L.dsum), dq32, dqkv + h,
+                               dqkv + 2 * h, 3LL * h, b, s, h, heads, causal, st, status));
+  BPT_TRY(launch_rows_to_bf16(dq32, rows, h, dqkv, 3LL * h, sms, st));
+  // projection: dbqkv = sum dqkv, dWqkv = x^T dqkv, dx = dhid + dqkv Wqkv^T
+  BPT_TRY(launch_colsum(dqkv, rows, 3 * h, 3LL * h, dbqkv, 0, st));
+  {
+    GemmArgs a{};
+    a.out = dWqkv;
+    a.ld_out = 3LL * h;
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(x, h, dqkv, 3LL * h, h, 3LL * h, rows, a, sms, st, status, "bwd_dWqkv")));
+    a = GemmArgs{};
+    a.dy = f32(L.dhid);
+    a.ld_dy = h;
+    a.out = dx;
+    a.ld_out = h;
+    BPT_TRY((launch_gemm_t<EPI_BWD_DHID, 0, 0>(dqkv, 3LL * h, Wqkv, 3LL * h, rows, h, 3LL * h, a, sms, st, status,
+                                               "bwd_dx")));
   }
   return BPT_OK;
 }

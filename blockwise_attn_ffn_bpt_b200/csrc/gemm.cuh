@@ -35,7 +35,7 @@ enum EpiMode {
   EPI_OUTPROJ = 1,   // + bo + x (first residual) -> fp32 hid and its bf16 copy (wave scratch)
   EPI_FFN_UP = 2,    // + b1, ReLU -> bf16 U
   EPI_FFN_DOWN = 3,  // + b2 + hid (second residual) -> fp32 out
-  EPI_BWD_DA = 4,    // (dy W2^T) masked by U > 0 (the ReLU's derivative) -> bf16 da
+  EPI_BWD_DA = 4,    // (dy W2^T) masked by U > 0 (the ReLU's derivative; no mask without U) -> bf16 da
   EPI_BWD_DHID = 5,  // + dy (the residual's gradient) -> fp32 dhid
   EPI_GRAD = 6,      // -> fp32 weight gradient, added to what is there when accumulate is set
 };
@@ -164,10 +164,12 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int co
     float* o = a.out + (a.row0 + row) * a.ld_out + col;
     store32_f32(o, v);
   } else if constexpr (MODE == EPI_BWD_DA) {
-    float u[32];
-    load32(a.mask_u, 0, (long long)row * a.ld_mask + col, u);
+    if (a.mask_u != nullptr) {
+      float u[32];
+      load32(a.mask_u, 0, (long long)row * a.ld_mask + col, u);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = u[i] > 0.0f ? v[i] : 0.0f;
+      for (int i = 0; i < 32; ++i) v[i] = u[i] > 0.0f ? v[i] : 0.0f;
+    }
     store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);
   } else if constexpr (MODE == EPI_BWD_DHID) {
     float dy[32];

@@ -317,6 +317,77 @@ int bpt_ffn_backward(const float* hid, const void* W1, const void* b1, const voi
                      int h, int ffn, int chunk_rows, float* dhid, float* dW1, float* db1, float* dW2, float* db2,
                      void* workspace, size_t ws_bytes, void* stream);
 
+/* Attention forward (as bpt_attention) that also writes each row's
+ * log-sum-exp of the scaled scores, the statistic the backward recomputes the
+ * attention weights from (Algorithm 1 records each query block's
+ * normalisation statistics, step 10; the backward of the paper review's
+ * section 3 rematerialises the blockwise computation from them).
+ * lse2: fp32 [b, heads, s] device memory, lse2[(beta * heads + k) * s + t] =
+ * log2(sum_u exp2(c S_tu)) for head k, with c = log2(e) / sqrt(dh) and S the
+ * scores Q K^T (masked keys left out); it must not overlap o. Other arguments,
+ * errors and stream semantics as for bpt_attention (no block sizes: the
+ * result does not depend on them). */
+int bpt_attention_lse(const void* q, const void* k, const void* v, int b, int s, int h, int heads, int causal,
+                      void* o, float* lse2, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Backward of the attention and of the whole layer.
+ * ------------------------------------------------------------------------ */
+
+/* Gradients of O = softmax(Q K^T / sqrt(dh)) V per head (Eq. 3 and Algorithm 1
+ * steps 4-10 of the paper review, inverted blockwise as its section 3
+ * rematerialises the blockwise computation for training): for dO = dL/dO,
+ *
+ *     P = 2^(c S - lse2) (0 where masked),  D = rowsum(dO O)
+ *     dV = P^T dO,  dS = P (dO V^T - D),  dQ = dS K / sqrt(dh),  dK = dS^T Q / sqrt(dh)
+ *
+ * computed per key/value tile of 128 keys over the query tiles that see it,
+ * with P recomputed from lse2 (from bpt_attention_lse) and never stored.
+ * q, k, v, o, dO: bf16 [b, s, h] device memory (o the forward's output);
+ * lse2 fp32 [b, heads, s]. Outputs dq, dk, dv: bf16 [b, s, h], written
+ * entirely. P and dS enter the products as bf16; dQ is summed over the key
+ * tiles in fp32. workspace: at least bpt_attention_backward_workspace_bytes
+ * bytes of device memory (D and the fp32 dQ sums). Errors: BPT_ERR_SHAPE
+ * (dh not 64 or 128, ...), BPT_ERR_NULL, BPT_ERR_ALIGN (16 bytes),
+ * BPT_ERR_NOMEM, BPT_ERR_ALIAS (an output or the workspace overlaps an input
+ * or another output); nothing launched then. Asynchronous on `stream`;
+ * device-side failures through bpt_stream_status. */
+size_t bpt_attention_backward_workspace_bytes(int b, int s, int h, int heads);
+int bpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                           const float* lse2, int b, int s, int h, int heads, int causal, void* dq, void* dk,
+                           void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Gradients of one BPT layer's output with respect to its input and every
+ * parameter (the layer of bpt_layer_forward_ffn, FFN width ffn), for the
+ * upstream gradient dy = dL/dout: the chain rule through the forward of
+ * Algorithm 1 and Eq. 3 of the paper review,
+ *
+ *     qkv = x Wqkv + bqkv;  O = attention(Q, K, V);  hid = x + O Wo + bo
+ *     out = hid + max(0, hid W1 + b1) W2 + b2
+ *     FFN block as bpt_ffn_backward -> dhid, dW1, db1, dW2, db2
+ *     dbo = sum dhid;  dWo = O^T dhid;  dO = dhid Wo^T
+ *     attention as bpt_attention_backward -> dQ, dK, dV
+ *     dbqkv = sum [dQ|dK|dV];  dWqkv = x^T [dQ|dK|dV];  dx = dhid + [dQ|dK|dV] Wqkv^T
+ *
+ * The forward is rematerialised here (the pages' training recipe stores none
+ * of it): the projection, the attention with its per-row statistics, and the
+ * out-projection are recomputed, and the FFN intermediate chunk by chunk.
+ * x and the weights bf16 as for bpt_layer_forward_ffn; dy fp32 [b, s, h].
+ * Outputs fp32, written entirely: dx [b, s, h], dWqkv [h, 3h], dbqkv [3h],
+ * dWo [h, h], dbo [h], dW1 [h, ffn], db1 [ffn], dW2 [ffn, h], db2 [h]. Products
+ * take bf16 operands with fp32 accumulation. workspace: at least
+ * bpt_layer_backward_workspace_bytes bytes of device memory (about 20 bytes
+ * per element of [b, s, h] plus the FFN backward's chunk buffers). Causal
+ * masking as for the forward. Errors as for bpt_attention_backward, plus
+ * BPT_ERR_SHAPE for ffn not a positive multiple of 64; nothing launched then.
+ * Asynchronous on `stream`; device-side failures through bpt_stream_status. */
+size_t bpt_layer_backward_workspace_bytes(int b, int s, int h, int heads, int ffn);
+int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                       const void* W1, const void* b1, const void* W2, const void* b2, const float* dy, int b, int s,
+                       int h, int heads, int ffn, int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo,
+                       float* dbo, float* dW1, float* db1, float* dW2, float* db2, void* workspace,
+                       size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Status and measurement.
  * ------------------------------------------------------------------------ */

@@ -77,6 +77,25 @@ def _attention_probs(Q, K, dh, causal):
     return E / E.sum(axis=-1, keepdims=True)
 
 
+def attention_row_lse2(Q, K, heads: int, causal: bool) -> np.ndarray:
+    """Per query row and head, the log-sum-exp of the row's scaled scores over
+    its visible keys, in log2 units: log2 sum_u exp(S_tu) with S = Q K^T /
+    sqrt(dh). It is the normalisation statistic of Algorithm 1 (the running max
+    m and sum l of a row, taken together as m + log2 l, with m in log2 units),
+    from which the backward recomputes P = exp(S - lse). Returns [b, heads, s]."""
+    b, s, h = Q.shape
+    dh = h // heads
+    t = np.arange(s)
+    allowed = ob._key_allowed(t, t, causal)
+    out = np.zeros((b, heads, s))
+    for k in range(heads):
+        c = ob._head_cols(k, dh)
+        S = np.where(allowed, (Q[..., c] @ np.swapaxes(K[..., c], -1, -2)) * ob._softmax_scale(dh), -np.inf)
+        mx = S.max(axis=-1, keepdims=True)
+        out[:, k, :] = (mx[..., 0] + np.log(np.exp(S - mx).sum(axis=-1))) / np.log(2.0)
+    return out
+
+
 def attention_backward(Q, K, V, dO, heads: int, causal: bool):
     """dQ, dK, dV [b, s, h] of O = softmax(Q K^T / sqrt(dh)) V per head, by the plain definition."""
     h = Q.shape[-1]

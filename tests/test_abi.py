@@ -353,3 +353,38 @@ def test_ffn_backward_entry_validates_before_touching_memory():
     assert call(nbytes=need - 1) == NOMEM
     assert call(dW1=hid) == ALIAS  # an output over an input
     assert call(db1=dW2 + 16) == ALIAS  # two outputs overlapping
+
+
+def test_backward_entries_validate_and_size_their_workspaces():
+    L = bpt.lib()
+
+    def up(v):
+        return (v + 1023) // 1024 * 1024
+
+    b, s, h, heads, f = 2, 256, 256, 2, 512
+    rows = b * s
+    # attention backward: D and the fp32 dQ sums
+    assert L.bpt_attention_backward_workspace_bytes(b, s, h, heads) == up(b * heads * s * 4) + up(rows * h * 4)
+    assert L.bpt_attention_backward_workspace_bytes(b, s, 192, 2) == 0  # dh 96
+    p = fake_ptrs(10)
+    ws_att = L.bpt_attention_backward_workspace_bytes(b, s, h, heads)
+    assert L.bpt_attention_backward(*p[:6], b, s, 192, 2, 1, *p[6:9], p[9], ws_att, None) == SHAPE
+    assert L.bpt_attention_backward(*p[:6], b, s, h, heads, 1, *p[6:9], None, ws_att, None) == NULL
+    assert L.bpt_attention_backward(*p[:6], b, s, h, heads, 1, *p[6:9], p[9], ws_att - 1, None) == NOMEM
+    assert L.bpt_attention_backward(*p[:6], b, s, h, heads, 1, p[6] + 8, *p[7:9], p[9], ws_att, None) == ALIGN
+    assert L.bpt_attention_backward(*p[:6], b, s, h, heads, 1, p[0], *p[7:9], p[9], ws_att, None) == ALIAS
+    assert L.bpt_attention_backward(*p[:6], 0, s, h, heads, 1, *p[6:9], p[9], 0, None) == OK  # nothing to do
+    assert L.bpt_attention_lse(*p[:3], b, s, h, heads, 1, p[3], None, None) == NULL
+    assert L.bpt_attention_lse(*p[:3], b, s, h, heads, 1, p[3], p[3], None) == ALIAS
+    # layer backward: the recomputed forward, the gradients on the way, the FFN chunk buffers
+    need = L.bpt_layer_backward_workspace_bytes(b, s, h, heads, f)
+    act, act32, stat = up(rows * h * 2), up(rows * h * 4), up(b * heads * s * 4)
+    ffn_ws = L.bpt_ffn_backward_workspace_bytes(rows, h, f, 0)
+    assert need == 7 * act + 2 * act32 + 2 * stat + up(rows * 3 * h * 2) + ffn_ws  # Q K V O hb dhb dO
+    for bad in (0, 32, 100):
+        assert L.bpt_layer_backward_workspace_bytes(b, s, h, heads, bad) == 0
+    q = fake_ptrs(20)
+    assert L.bpt_layer_backward(*q[:10], b, s, h, heads, 100, 1, *q[10:19], q[19], need, None) == SHAPE
+    assert L.bpt_layer_backward(*q[:10], b, s, h, heads, f, 1, *q[10:19], q[19], need - 1, None) == NOMEM
+    assert L.bpt_layer_backward(*q[:9], None, b, s, h, heads, f, 1, *q[10:19], q[19], need, None) == NULL
+    assert L.bpt_layer_backward(*q[:10], b, s, h, heads, f, 1, q[0], *q[11:19], q[19], need, None) == ALIAS

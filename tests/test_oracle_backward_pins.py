@@ -166,3 +166,43 @@ def test_ffn_backward_matches_torch_autograd():
     g = obb.ffn_backward(*(t[k].detach().numpy() for k in ("hid", "W1", "b1", "W2")), dy)
     for k in ("hid", "W1", "b1", "W2", "b2"):
         np.testing.assert_allclose(g["d" + k], t[k].grad.numpy(), rtol=1e-10, atol=1e-10, err_msg=k)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_lse_of_zero_queries_is_the_log_of_the_key_count(causal):
+    # all scores 0: each row sums exp(0) once per visible key (closed form)
+    b, s, h, heads = 2, 7, 8, 2
+    rng = np.random.default_rng(5)
+    Q, K = np.zeros((b, s, h)), rng.standard_normal((b, s, h))
+    lse = obb.attention_row_lse2(Q, K, heads, causal)
+    count = np.arange(1, s + 1) if causal else np.full(s, s)
+    assert np.allclose(lse, np.broadcast_to(np.log2(count), (b, heads, s)), rtol=0, atol=1e-12)
+
+
+def test_row_lse_of_the_first_causal_row_is_its_own_score():
+    # causal row 0 sees key 0 alone: log2 exp(S_00) = S_00 log2(e)
+    b, s, h, heads = 1, 5, 8, 2
+    rng = np.random.default_rng(6)
+    Q, K = rng.standard_normal((b, s, h)), rng.standard_normal((b, s, h))
+    lse = obb.attention_row_lse2(Q, K, heads, True)
+    for k in range(heads):
+        c = slice(k * 4, (k + 1) * 4)
+        s00 = float(Q[0, 0, c] @ K[0, 0, c]) / 2.0
+        assert abs(lse[0, k, 0] - s00 / np.log(2.0)) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_lse_recovers_the_attention_weights_of_torch(causal):
+    # exp(S - lse) reproduces torch's own softmax of the masked scores, row by row
+    b, s, h, heads = 2, 6, 8, 2
+    rng = np.random.default_rng(7)
+    Q, K = rng.standard_normal((b, s, h)) * 2.0, rng.standard_normal((b, s, h))
+    lse = obb.attention_row_lse2(Q, K, heads, causal)
+    for k in range(heads):
+        c = slice(k * 4, (k + 1) * 4)
+        S = torch.tensor(Q[..., c]) @ torch.tensor(K[..., c]).transpose(-1, -2) / 2.0
+        if causal:
+            S = S.masked_fill(torch.triu(torch.ones(s, s, dtype=torch.bool), 1), float("-inf"))
+        P = torch.softmax(S, dim=-1).numpy()
+        P2 = np.where(np.isfinite(S.numpy()), np.exp2(S.numpy() / np.log(2.0) - lse[:, k, :, None]), 0.0)
+        assert np.allclose(P2, P, rtol=1e-12, atol=1e-15)

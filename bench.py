@@ -768,6 +768,85 @@ def ffn_backward_arm(args):
     return 0 if status == 0 else 1
 
 
+def layer_backward_flops(shape: bi.LayerShape) -> dict:
+    """Matmul flops of one layer backward (bpt_layer_backward) per kernel name:
+    the forward it recomputes (projection, attention, out-projection), the FFN
+    block's five products, the out-projection's two, the attention backward's
+    five s x s products (S, dP, dV, dK, dQ; causal counted as half) and the
+    projection's two."""
+    b, s, h, f = shape.b, shape.s, shape.h, shape.f
+    tok = b * s
+    half = 0.5 if shape.causal else 1.0
+    return {
+        "forward recompute": 2.0 * tok * h * 3 * h + 4.0 * b * s * s * h * half + 2.0 * tok * h * h,
+        "ffn backward": 5 * 2.0 * tok * h * f,
+        "out-projection backward": 2 * 2.0 * tok * h * h,
+        "attention_bwd": 5 * 2.0 * b * s * s * h * half,
+        "projection backward": 2 * 2.0 * tok * h * 3 * h,
+    }
+
+
+def layer_backward_arm(args):
+    """Throughput of the whole layer's backward (bpt_layer_backward) on one
+    workload: the recomputed forward, the FFN block, the out-projection, the
+    attention backward kernel and the projection, one call per step; then the
+    per-kernel split in a pass of its own. Seeded synthetic inputs drawn on the
+    device (x and dy N(0, 1), weights N(0, 1/fan_in), biases N(0, 0.02^2))."""
+    import torch
+    import blockwise_attn_ffn_bpt_b200 as bpt
+    shape = shape_of(args.workload)
+    b, s, h, f, heads = shape.b, shape.s, shape.h, shape.f, shape.heads
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    g = torch.Generator(device=device).manual_seed(0)
+    x = torch.randn((b, s, h), generator=g, device=device).to(torch.bfloat16)
+    dy = torch.randn((b, s, h), generator=g, device=device)
+    params = {}
+    for name, shp in bi.tensor_shapes(shape).items():
+        if name != "x":
+            params[name] = (torch.randn(shp, generator=g, device=device) * bi.tensor_std(name, shape)).to(
+                torch.bfloat16)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        bpt.layer_backward(x, params, dy, heads, shape.causal, stream=stream)
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(gpu_index(0)) as clocks:
+        for e0, e1 in evs:
+            e0.record(stream)
+            bpt.layer_backward(x, params, dy, heads, shape.causal, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    status = bpt.stream_status(stream)
+    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    fl = layer_backward_flops(shape)
+    total = sum(fl.values())
+    # per-kernel split, in a pass of its own with the launch log on
+    bpt.set_kernel_timing(True)
+    bpt.kernel_times()
+    for _ in range(args.steps):
+        bpt.layer_backward(x, params, dy, heads, shape.causal, stream=stream)
+    kt = bpt.kernel_times()
+    bpt.set_kernel_timing(False)
+    kernels = {}
+    split_total = sum(ms_ for _, ms_ in kt.values()) or 1.0
+    for name, (n_, ms_) in sorted(kt.items(), key=lambda kv: -kv[1][1]):
+        kernels[name] = {"launches": n_, "ms_per_step": ms_ / args.steps, "share": ms_ / split_total}
+    att = kt.get("attention_bwd")
+    att_tflops = fl["attention_bwd"] / (att[1] / args.steps / 1e3) / 1e12 if att else None
+    peaks, src = measured_peaks()
+    line = {"metric": "BPT layer backward (bpt_layer_backward) tokens/s and TFLOP/s on 1 B200",
+            "value": b * s / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "tflops": total / (ms / 1e3) / 1e12,
+            "frac_of_bf16_peak": total / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
+            "peak_source": f"{src} bf16_tflops (burst)", "steps": args.steps, "warmup": args.warmup,
+            "dtype": "bf16", "config": config_of(shape, args.workload),
+            "flops_per_step": fl, "attention_bwd_tflops": att_tflops, "kernels": kernels,
+            "device_status": status, "clocks": clocks.summary(),
+            "data": "synthetic (torch generator on the device)"}
+    print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -787,11 +866,15 @@ def main(argv=None):
                     help="FFN-side schedule: the library's default, one chained launch, or per-GEMM waves")
     ap.add_argument("--ffn-backward", action="store_true",
                     help="instead: throughput of the FFN block's backward at the 7B-class layer's shapes")
+    ap.add_argument("--layer-backward", action="store_true",
+                    help="instead: throughput of the whole layer's backward on --workload")
     args = ap.parse_args(argv)
     if args.max_context:
         return max_context_arm(args)
     if args.ffn_backward:
         return ffn_backward_arm(args)
+    if args.layer_backward:
+        return layer_backward_arm(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.all_configs:

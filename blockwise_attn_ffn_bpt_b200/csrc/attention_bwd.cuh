@@ -12,12 +12,13 @@
 //     dS^T = P^T (dP^T - D_i),  D_i = rowsum(dO_i O_i)
 // and accumulates dV_j += P^T dO_i and dK_j += dS^T Q_i in tensor memory; the
 // query gradient dQ_i += dS K_j (x scale) is added to an fp32 accumulator in
-// global memory. At the end dK_j (x scale) and dV_j are written as bf16.
+// global memory by the TMA engine (bulk reduce-add of whole boxes). At the end
+// dK_j (x scale) and dV_j are written as bf16.
 //
 // Roles (256 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
 // tile (two-stage ring) with TMA; one thread of warp 1 issues the MMAs; warps
-// 4-7 (one row per thread = one tensor-memory lane) form P and dS, then read the
-// dQ partial and add it to global memory, and finally write dK and dV.
+// 4-7 (one row per thread = one tensor-memory lane) form P and dS, then stage
+// the dQ partial for the TMA reduce-add, and finally write dK and dV.
 // Tensor memory: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T over its first
 // 64 columns, then the dQ partial over all 128), dP^T [384, 512) (dS^T over its
 // first 64 columns).
@@ -54,7 +55,7 @@ struct AttnBwdArgs {
   int n_kv;                 // key/value tiles per (sequence, head)
   const float* lse2;        // [b][heads][s]: max + log2(sum) of the forward, in log2 units
   const float* dsum;        // [b][heads][s]: D = rowsum(dO O)
-  float* dq;                // [b][s][h] fp32 accumulator (zeroed by the caller)
+  float* dq;                // [b][s][h] fp32 accumulator (zeroed by the caller; reached through its tensor map)
   __nv_bfloat16* dk;        // rows (beta * s + t), ld_kv elements apart, head columns
   __nv_bfloat16* dv;
   long long ld_kv;
@@ -78,15 +79,26 @@ __device__ __forceinline__ void ab_named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-__device__ __forceinline__ void ab_red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+// Bulk reduce-add of a shared-memory box into global memory by the TMA engine
+// (the tensor map gives the global layout, here fp32 with 128B swizzle).
+__device__ __forceinline__ void ab_tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
+__device__ __forceinline__ void ab_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed bulk group have been read
+__device__ __forceinline__ void ab_bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed bulk group has completed
+__device__ __forceinline__ void ab_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int DH>
 __global__ void __launch_bounds__(AB_THREADS, 1)
     attention_bwd_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                          const AttnBwdArgs args) {
+                          const __grid_constant__ CUtensorMap tmdQ, const AttnBwdArgs args) {
   using C = AttnBwdCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,6 +149,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
+    tma_prefetch_desc(&tmdQ);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), 512);
@@ -237,8 +250,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const int key = j0 + r;
     const float sl2 = args.scale_log2;
     const long long bh = (long long)beta * args.heads + head;
-    // Every warp runs every iteration and both named barriers of it; a wait that
-    // gives up only switches the work off (the waits are bounded, and the
+    // Every warp runs every iteration and every named barrier of it; a wait
+    // that gives up only switches the work off (the waits are bounded, and the
     // barriers never see a warp missing).
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       }
       ab_named_sync(1, 128);
       ok = ok && warp_wait(s_ready, (uint32_t)it & 1u, abort_flag);
-      if (!ok) continue;
+      if (ok) {
       tc_fence_after();
       // a query column q is used when it is a real row and (causal) not before this key
       const bool key_ok = key < args.s;
@@ -293,30 +306,50 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_ready);
-      // dQ partial of this query tile: lane = query row
-      ok = warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
-      if (!ok) continue;
-      tc_fence_after();
-      {
-        const int q = i0 + r;
-        float* dst = args.dq + ((long long)beta * args.s + q) * args.h + head * DH;
+      }
+      // dQ partial of this query tile (lane = query row), x scale, added to the
+      // fp32 accumulator by the TMA engine: staged through the dS buffer (free
+      // once the dQ product has read it) 64 columns at a time, as two 128B-
+      // swizzled [128 rows][32 fp32] boxes. Rows past the sequence are clipped
+      // by the tensor map (and hold zeros: their dS is zero).
+      const bool got = ok && warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
+      ok = got;
+      if (got) tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < DH / 32; ++c) {
-          uint32_t o[32];
-          tmem_load32(tmem_base + AB_T_ST + c * 32 + lane_base, o);
-          if (q < args.s) {
+      for (int round = 0; round < DH / 64; ++round) {
+        if (got) {
+#pragma unroll 1
+          for (int bx = 0; bx < 2; ++bx) {
+            uint32_t o[32];
+            tmem_load32(tmem_base + AB_T_ST + round * 64 + bx * 32 + lane_base, o);
+            const uint32_t row = sbase + C::OFF_DS + bx * (128 * 128) + r * 128;
 #pragma unroll
             for (int x = 0; x < 8; ++x)
-              ab_red_add_v4(dst + c * 32 + 4 * x, __uint_as_float(o[4 * x]) * args.scale,
-                            __uint_as_float(o[4 * x + 1]) * args.scale, __uint_as_float(o[4 * x + 2]) * args.scale,
-                            __uint_as_float(o[4 * x + 3]) * args.scale);
+              st_shared_v4(row + (uint32_t)((x ^ (r & 7)) * 16), __float_as_uint(__uint_as_float(o[4 * x]) * args.scale),
+                           __float_as_uint(__uint_as_float(o[4 * x + 1]) * args.scale),
+                           __float_as_uint(__uint_as_float(o[4 * x + 2]) * args.scale),
+                           __float_as_uint(__uint_as_float(o[4 * x + 3]) * args.scale));
           }
         }
+        fence_async_smem();
+        ab_named_sync(1, 128);
+        if (warp == 4 && lane == 0 && got && !*abort_flag.flag) {
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+            ab_tma_reduce_add_3d(&tmdQ, sbase + C::OFF_DS + bx * (128 * 128), head * DH + round * 64 + bx * 32, i0,
+                                 beta);
+          ab_bulk_commit();
+          ab_bulk_wait_read();
+        }
+        ab_named_sync(1, 128);  // the boxes have been read: the buffer is free again
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
+      if (got) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+      }
     }
+    if (warp == 4 && lane == 0) ab_bulk_wait_all();  // the last reduce-adds have landed
     // dK (x scale) and dV of this key tile: lane = key
     if (ok && n_it > 0 && warp_wait(kv_done, 0, abort_flag)) {
       tc_fence_after();

@@ -111,7 +111,7 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor map with 128-byte swizzle; dims/strides innermost first,
 // strides in bytes for dims 1.. (dim 0 is contiguous).
 bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box) {
+              const uint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t gd[3], gs[2];
@@ -121,7 +121,7 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims
     bx[i] = box[i];
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides[i];
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = enc(map, dtype, rank, const_cast<void*>(base), gd, gs, bx, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -143,6 +143,16 @@ bool map_seq(CUtensorMap* m, const void* base, int b, int s, int cols, long long
   const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)ld * 2 * (uint64_t)s};
   const uint32_t box[3] = {64, box_rows, 1};
   return make_map(m, base, 3, dims, strides, box);
+}
+
+// [b, s, cols] fp32 (rows `cols` apart) as [128 rows][32] boxes: the dQ
+// accumulator of the attention backward, which the TMA engine adds into (rows
+// past s of a sequence are clipped).
+bool map_seq_f32(CUtensorMap* m, float* base, int b, int s, int cols) {
+  const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)s, (uint64_t)b};
+  const uint64_t strides[2] = {(uint64_t)cols * 4, (uint64_t)cols * 4 * (uint64_t)s};
+  const uint32_t box[3] = {32, 128, 1};
+  return make_map(m, base, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
 }
 
 // ------------------------------------------------------------- device info
@@ -631,28 +641,41 @@ int launch_gemm_t(const void* A, long long lda, const void* B, long long ldb, lo
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
-// out[c] (+)= sum over rows r of src[r * ld + c], fp32 accumulation in row
-// order (deterministic): one thread per column.
+// out[c] (+)= sum over rows r of src[r * ld + c], fp32: one block of 32 warps
+// per 32 columns; lane l of warp w sums column c0 + l over the rows r = w, w + 32,
+// ... (each row read as one coalesced line by the warp), then the 32 partial sums
+// of a column are added in warp order. Same order every run (deterministic).
 template <typename T>
-__global__ void colsum_kernel(const T* __restrict__ src, long long rows, int cols, long long ld, float* out,
-                              int accumulate) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
+__global__ void __launch_bounds__(1024) colsum_kernel(const T* __restrict__ src, long long rows, int cols, long long ld,
+                                                      float* out, int accumulate) {
+  __shared__ float part[32][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
   float acc = 0.0f;
-  for (long long r = 0; r < rows; ++r) {
-    if constexpr (sizeof(T) == 2)
-      acc += __bfloat162float(src[r * ld + c]);
-    else
-      acc += src[r * ld + c];
+  if (c < cols) {
+    long long r = w;
+#pragma unroll 4
+    for (; r < rows; r += 32) {
+      if constexpr (sizeof(T) == 2)
+        acc += __bfloat162float(src[r * ld + c]);
+      else
+        acc += src[r * ld + c];
+    }
   }
-  out[c] = accumulate ? out[c] + acc : acc;
+  part[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && c < cols) {
+    float t = 0.0f;
+    for (int i = 0; i < 32; ++i) t += part[i][lane];
+    out[c] = accumulate ? out[c] + t : t;
+  }
 }
 
 template <typename T>
 int launch_colsum(const T* src, long long rows, int cols, long long ld, float* out, int accumulate, cudaStream_t st) {
   if (cols <= 0) return BPT_OK;
   LaunchScope ls("colsum", st);
-  colsum_kernel<T><<<(cols + 127) / 128, 128, 0, st>>>(src, rows, cols, ld, out, accumulate);
+  colsum_kernel<T><<<(cols + 31) / 32, 1024, 0, st>>>(src, rows, cols, ld, out, accumulate);
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
@@ -770,9 +793,9 @@ int launch_attention_bwd(const void* q, const void* k, const void* v, long long 
                          cudaStream_t st, int* status) {
   if ((long long)b * s == 0) return BPT_OK;
   const int dh = h / heads;
-  CUtensorMap tq, tk, tv, td;
+  CUtensorMap tq, tk, tv, td, tdq;
   if (!map_seq(&tq, q, b, s, h, ld_in) || !map_seq(&tk, k, b, s, h, ld_in) || !map_seq(&tv, v, b, s, h, ld_in) ||
-      !map_seq(&td, dO, b, s, h, ld_do))
+      !map_seq(&td, dO, b, s, h, ld_do) || !map_seq_f32(&tdq, dq, b, s, h))
     return BPT_ERR_CUDA;
   AttnBwdArgs a{};
   a.s = s;
@@ -794,9 +817,9 @@ int launch_attention_bwd(const void* q, const void* k, const void* v, long long 
     dim3 grid((unsigned)a.n_kv * (unsigned)heads, 1, std::min(65535, b - z0));
     LaunchScope ls("attention_bwd", st);
     if (dh == 64)
-      attention_bwd_tcgen05<64><<<grid, AB_THREADS, AttnBwdCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, td, a);
+      attention_bwd_tcgen05<64><<<grid, AB_THREADS, AttnBwdCfg<64>::SMEM_BYTES, st>>>(tq, tk, tv, td, tdq, a);
     else
-      attention_bwd_tcgen05<128><<<grid, AB_THREADS, AttnBwdCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, td, a);
+      attention_bwd_tcgen05<128><<<grid, AB_THREADS, AttnBwdCfg<128>::SMEM_BYTES, st>>>(tq, tk, tv, td, tdq, a);
   }
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }

@@ -12,16 +12,22 @@
 //     dS^T = P^T (dP^T - D_i),  D_i = rowsum(dO_i O_i)
 // and accumulates dV_j += P^T dO_i and dK_j += dS^T Q_i in tensor memory; the
 // query gradient dQ_i += dS K_j (x scale) is added to an fp32 accumulator in
-// global memory by the TMA engine (bulk reduce-add of whole boxes). At the end
-// dK_j (x scale) and dV_j are written as bf16.
+// global memory by the TMA engine (bulk reduce-add of whole boxes, staged in the
+// query tile's own ring stage once its products are done). At the end dK_j
+// (x scale) and dV_j are written as bf16.
 //
-// Roles (256 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
-// tile (two-stage ring) with TMA; one thread of warp 1 issues the MMAs; warps
-// 4-7 (one row per thread = one tensor-memory lane) form P and dS, then stage
-// the dQ partial for the TMA reduce-add, and finally write dK and dV.
-// Tensor memory: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T over its first
-// 64 columns, then the dQ partial over all 128), dP^T [384, 512) (dS^T over its
-// first 64 columns).
+// Roles (384 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
+// tile (two-stage ring) with TMA; one thread of warp 1 issues the MMAs; one
+// thread of warp 2 issues the dQ reduce-adds and returns each ring stage to the
+// copies once they have read it; two warpgroups (warps 4-7 and 8-11, one row per
+// thread = one tensor-memory lane) form P and dS for the query columns [0, 64)
+// and [64, 128) of the tile, then stage the dQ partial, and finally write dK and
+// dV, each warpgroup half of the columns.
+// Tensor memory: dV [0, 128), dK [128, 256), S^T [256, 384), dP^T [384, 512).
+// Each warpgroup writes its P^T (bf16 pairs) over the first 32 of its own 64 S^T
+// columns and its dS^T likewise in dP^T, so that neither overwrites scores the
+// other has not loaded yet; the dQ partial then goes over dP^T, so that the next
+// tile's S^T product need not wait for it to be read out.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,7 +36,7 @@ namespace bpt {
 
 constexpr int AB_BM = 128;  // query rows per tile
 constexpr int AB_BN = 128;  // keys per CTA
-constexpr int AB_THREADS = 256;
+constexpr int AB_THREADS = 384;
 constexpr int AB_T_DV = 0, AB_T_DK = 128, AB_T_ST = 256, AB_T_DP = 384;
 
 template <int DH>
@@ -75,6 +81,22 @@ __device__ __forceinline__ void ab_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Two 16-column stores of this thread's lane behind one completion wait.
+__device__ __forceinline__ void ab_tmem_store16x2(uint32_t ta, const uint32_t (&a)[16], uint32_t tb,
+                                                  const uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], "
+      "{%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(ta),
+      "r"(tb), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]),
+      "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(b[0]), "r"(b[1]),
+      "r"(b[2]), "r"(b[3]), "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7]), "r"(b[8]), "r"(b[9]), "r"(b[10]),
+      "r"(b[11]), "r"(b[12]), "r"(b[13]), "r"(b[14]), "r"(b[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void ab_named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -114,6 +136,10 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
   const uint32_t mma_done = smem_addr(bars + 10);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   const Abort abort_flag{reinterpret_cast<volatile int*>(bars + 12), args.status};
+  // [2] per ring stage: the dQ boxes of the stage's tile are in place (the next
+  // arrival on a stage's barrier needs that stage refilled, which warp 2 allows only
+  // after its wait, so a wait can never fall a phase behind)
+  const uint32_t dq_staged0 = smem_addr(bars + 13);
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LD);
   float* s_dsum = s_lse + 128;
 
@@ -138,11 +164,13 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       mbar_init(qdo_empty0 + 8 * i, 1);
     }
     mbar_init(s_ready, 1);
-    mbar_init(p_ready, 4);
+    mbar_init(p_ready, 8);
     mbar_init(dq_ready, 1);
-    mbar_init(dq_free, 4);
+    mbar_init(dq_free, 8);
     mbar_init(kv_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(dq_staged0, 8);
+    mbar_init(dq_staged0 + 8, 8);
     *abort_flag.flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -202,17 +230,19 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it & 1;
         ok = mbar_wait(qdo_full0 + 8 * st, (uint32_t)(it >> 1) & 1u, abort_flag);
-        // the previous tile's dQ partial must be read out before S^T overwrites it
-        if (ok && it > 0) ok = mbar_wait(dq_free, (uint32_t)(it - 1) & 1u, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t q_s = sbase + C::OFF_QDO + st * 2 * C::TILE, do_s = q_s + C::TILE;
+        // S^T may overwrite the previous tile's P^T at once (its dV product was issued earlier)
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
           mma_bf16_ss(tmem_base + AB_T_ST, smem_desc_sw128(k_s + off, 16, 1024), smem_desc_sw128(q_s + off, 16, 1024),
                       id_kmaj, kk > 0);
         }
+        // the previous tile's dQ partial (in the dP^T columns) must be read out first
+        if (it > 0 && !mbar_wait(dq_free, (uint32_t)(it - 1) & 1u, abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
@@ -222,135 +252,169 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         mma_commit(s_ready);
         if (!mbar_wait(p_ready, (uint32_t)it & 1u, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q (A from tensor memory: 16 queries = 8 columns per step)
+        // dV += P^T dO, dK += dS^T Q (A from tensor memory: 16 queries = 8 columns per
+        // step; queries 0..63 in the first warpgroup's columns, 64..127 in the second's)
 #pragma unroll
         for (int kk = 0; kk < AB_BM / 16; ++kk)
-          ab_mma_ts(tmem_base + AB_T_DV, tmem_base + AB_T_ST + kk * 8,
+          ab_mma_ts(tmem_base + AB_T_DV, tmem_base + AB_T_ST + (kk >> 2) * 64 + (kk & 3) * 8,
                     smem_desc_sw128(do_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
 #pragma unroll
         for (int kk = 0; kk < AB_BM / 16; ++kk)
-          ab_mma_ts(tmem_base + AB_T_DK, tmem_base + AB_T_DP + kk * 8,
+          ab_mma_ts(tmem_base + AB_T_DK, tmem_base + AB_T_DP + (kk >> 2) * 64 + (kk & 3) * 8,
                     smem_desc_sw128(q_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
-        // dQ partial = dS K over this key tile (16 keys per step), into the S^T columns
+        // dQ partial = dS K over this key tile (16 keys per step), into the dP^T columns
+        // (after the dK product, which reads dS^T there)
 #pragma unroll
         for (int kk = 0; kk < AB_BN / 16; ++kk)
-          mma_bf16_ss(tmem_base + AB_T_ST, smem_desc_sw128(ds_s + kk * 16 * 128, C::ATOM, 1024),
+          mma_bf16_ss(tmem_base + AB_T_DP, smem_desc_sw128(ds_s + kk * 16 * 128, C::ATOM, 1024),
                       smem_desc_sw128(k_s + kk * 16 * 128, C::ATOM, 1024), id_amn, kk > 0);
         mma_commit(dq_ready);
-        mma_commit(qdo_empty0 + 8 * st);
       }
       mma_commit(kv_done);
       mma_commit(mma_done);
     }
+  } else if (warp == 2) {
+    if (lane == 0 && n_it > 0) {
+      // ------------------------------------------------------------ dQ reduce-adds
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait(dq_staged0 + 8 * st, (uint32_t)(it >> 1) & 1u, abort_flag)) break;
+        const uint32_t q_s = sbase + C::OFF_QDO + st * 2 * C::TILE;
+        const int i0 = (i_first + it) * AB_BM;
+#pragma unroll
+        for (int bx = 0; bx < DH / 32; ++bx)
+          ab_tma_reduce_add_3d(&tmdQ, q_s + bx * (128 * 128), head * DH + 32 * bx, i0, beta);
+        ab_bulk_commit();
+        ab_bulk_wait_read();
+        mbar_arrive(qdo_empty0 + 8 * st);  // the stage may take the next copies
+      }
+      ab_bulk_wait_all();  // the last reduce-adds have landed
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P, dS, dQ, epilogue
+    const int g = (warp - 4) >> 2;  // warpgroup: query columns [64g, 64g + 64) of the tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tensor-memory lane: a key (P, dS) or a query (dQ)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int key = j0 + r;
     const float sl2 = args.scale_log2;
     const long long bh = (long long)beta * args.heads + head;
+    constexpr int NBOX = DH / 32;  // dQ boxes of 32 columns per query tile, half of them per warpgroup
     // Every warp runs every iteration and every named barrier of it; a wait
     // that gives up only switches the work off (the waits are bounded, and the
     // barriers never see a warp missing).
+    // the query tile's statistics: row r of the first warpgroup holds -lse2, of the
+    // second D; loaded one tile ahead into a register (its latency hides behind the
+    // previous tile's dQ work) and staged in shared memory at the top of each tile
+    auto stat_of = [&](int i0_) {
+      const int t = i0_ + r;
+      if (t >= args.s) return 0.0f;
+      return g == 0 ? -args.lse2[bh * args.s + t] : args.dsum[bh * args.s + t];
+    };
+    float stat_next = n_it > 0 ? stat_of(i_first * AB_BM) : 0.0f;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i0 = (i_first + it) * AB_BM;
-      // the query tile's statistics, once per tile (the previous tile's readers are done)
-      ab_named_sync(1, 128);
-      {
-        const int t = i0 + r;
-        s_lse[r] = t < args.s ? args.lse2[bh * args.s + t] : 0.0f;
-        s_dsum[r] = t < args.s ? args.dsum[bh * args.s + t] : 0.0f;
-      }
-      ab_named_sync(1, 128);
+      ab_named_sync(1, 256);  // the previous tile's readers of the statistics are done
+      if (g == 0)
+        s_lse[r] = stat_next;
+      else
+        s_dsum[r] = stat_next;
       ok = ok && warp_wait(s_ready, (uint32_t)it & 1u, abort_flag);
+      ab_named_sync(1, 256);  // the statistics are in place
+      if (it + 1 < n_it) stat_next = stat_of(i0 + AB_BM);
       if (ok) {
-      tc_fence_after();
-      // a query column q is used when it is a real row and (causal) not before this key
-      const bool key_ok = key < args.s;
+        tc_fence_after();
+        // a query column q is used when it is a real row and (causal) not before this
+        // key; in most tiles every column of every row is, and no test is needed
+        const bool key_ok = key < args.s;
+        const bool all_used = key_ok && i0 + AB_BM <= args.s && (!args.causal || j0 + AB_BN - 1 <= i0);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], dp[32];
-        tmem_load32x2(tmem_base + AB_T_ST + c * 32 + lane_base, tmem_base + AB_T_DP + c * 32 + lane_base, sv, dp);
-        uint32_t pk[16], dk[16];
+        for (int c = 2 * g; c < 2 * g + 2; ++c) {
+          uint32_t sv[32], dp[32];
+          tmem_load32x2(tmem_base + AB_T_ST + c * 32 + lane_base, tmem_base + AB_T_DP + c * 32 + lane_base, sv, dp);
+          uint32_t pk[16], dk[16];
+          const float4* nl4 = reinterpret_cast<const float4*>(s_lse + c * 32);
+          const float4* d4 = reinterpret_cast<const float4*>(s_dsum + c * 32);
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          float p2[2], d2[2];
+          for (int x4 = 0; x4 < 8; ++x4) {
+            const float4 nl = nl4[x4], dd = d4[x4];
+            const float nlv[4] = {nl.x, nl.y, nl.z, nl.w}, ddv[4] = {dd.x, dd.y, dd.z, dd.w};
+            float p4[4], g4[4];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qc = c * 32 + 2 * x + e;
-            const int q = i0 + qc;
-            const bool use = key_ok && q < args.s && (!args.causal || key <= q);
-            const float p = use ? ex2_approx(__uint_as_float(sv[2 * x + e]) * sl2 - s_lse[qc]) : 0.0f;
-            p2[e] = p;
-            d2[e] = use ? p * (__uint_as_float(dp[2 * x + e]) - s_dsum[qc]) : 0.0f;
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * x4 + e;
+              const float p = ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, nlv[e]));
+              p4[e] = p;
+              g4[e] = p * (__uint_as_float(dp[i]) - ddv[e]);
+            }
+            if (!all_used) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int q = i0 + c * 32 + 4 * x4 + e;
+                const bool use = key_ok && q < args.s && (!args.causal || key <= q);
+                p4[e] = use ? p4[e] : 0.0f;
+                g4[e] = use ? g4[e] : 0.0f;
+              }
+            }
+            pk[2 * x4] = pack_bf16x2(p4[0], p4[1]);
+            pk[2 * x4 + 1] = pack_bf16x2(p4[2], p4[3]);
+            dk[2 * x4] = pack_bf16x2(g4[0], g4[1]);
+            dk[2 * x4 + 1] = pack_bf16x2(g4[2], g4[3]);
           }
-          pk[x] = pack_bf16x2(p2[0], p2[1]);
-          dk[x] = pack_bf16x2(d2[0], d2[1]);
-        }
-        // P^T and dS^T (bf16 pairs) over the first 64 columns of their regions; the
-        // columns written here were loaded in this or an earlier chunk
-        tmem_store16(tmem_base + AB_T_ST + c * 16 + lane_base, pk);
-        tmem_store16(tmem_base + AB_T_DP + c * 16 + lane_base, dk);
-        // dS^T row of this key into the 128B-swizzled [keys][queries] layout of the dQ operand
-        const uint32_t row = sbase + C::OFF_DS + (c >> 1) * C::ATOM + r * 128;
+          // P^T and dS^T (bf16 pairs) over the first 32 of this warpgroup's 64
+          // columns: columns this warpgroup has already loaded
+          const uint32_t pcol = (uint32_t)(g * 64 + (c & 1) * 16);
+          ab_tmem_store16x2(tmem_base + AB_T_ST + pcol + lane_base, pk, tmem_base + AB_T_DP + pcol + lane_base, dk);
+          // dS^T row of this key into the 128B-swizzled [keys][queries] layout of the dQ operand
+          const uint32_t row = sbase + C::OFF_DS + (c >> 1) * C::ATOM + r * 128;
 #pragma unroll
-        for (int t4 = 0; t4 < 4; ++t4) {
-          const int chunk = (c & 1) * 4 + t4;
-          st_shared_v4(row + (uint32_t)((chunk ^ (r & 7)) * 16), dk[4 * t4], dk[4 * t4 + 1], dk[4 * t4 + 2],
-                       dk[4 * t4 + 3]);
-        }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
-      }
-      // dQ partial of this query tile (lane = query row), x scale, added to the
-      // fp32 accumulator by the TMA engine: staged through the dS buffer (free
-      // once the dQ product has read it) 64 columns at a time, as two 128B-
-      // swizzled [128 rows][32 fp32] boxes. Rows past the sequence are clipped
-      // by the tensor map (and hold zeros: their dS is zero).
-      const bool got = ok && warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
-      ok = got;
-      if (got) tc_fence_after();
-#pragma unroll 1
-      for (int round = 0; round < DH / 64; ++round) {
-        if (got) {
-#pragma unroll 1
-          for (int bx = 0; bx < 2; ++bx) {
-            uint32_t o[32];
-            tmem_load32(tmem_base + AB_T_ST + round * 64 + bx * 32 + lane_base, o);
-            const uint32_t row = sbase + C::OFF_DS + bx * (128 * 128) + r * 128;
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-              st_shared_v4(row + (uint32_t)((x ^ (r & 7)) * 16), __float_as_uint(__uint_as_float(o[4 * x]) * args.scale),
-                           __float_as_uint(__uint_as_float(o[4 * x + 1]) * args.scale),
-                           __float_as_uint(__uint_as_float(o[4 * x + 2]) * args.scale),
-                           __float_as_uint(__uint_as_float(o[4 * x + 3]) * args.scale));
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const int chunk = (c & 1) * 4 + t4;
+            st_shared_v4(row + (uint32_t)((chunk ^ (r & 7)) * 16), dk[4 * t4], dk[4 * t4 + 1], dk[4 * t4 + 2],
+                         dk[4 * t4 + 3]);
           }
         }
         fence_async_smem();
-        ab_named_sync(1, 128);
-        if (warp == 4 && lane == 0 && got && !*abort_flag.flag) {
-#pragma unroll
-          for (int bx = 0; bx < 2; ++bx)
-            ab_tma_reduce_add_3d(&tmdQ, sbase + C::OFF_DS + bx * (128 * 128), head * DH + round * 64 + bx * 32, i0,
-                                 beta);
-          ab_bulk_commit();
-          ab_bulk_wait_read();
-        }
-        ab_named_sync(1, 128);  // the boxes have been read: the buffer is free again
-      }
-      if (got) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(dq_free);
+        if (lane == 0) mbar_arrive(p_ready);
+      }
+      // dQ partial of this query tile (lane = query row), x scale: each warpgroup
+      // stages its half of the columns as 128B-swizzled [128 rows][32 fp32] boxes in
+      // the tile's ring stage (its Q and dO have been read by every product once the
+      // dQ partial is complete), releasing the tensor memory after its last load;
+      // warp 2 then adds the boxes into the accumulator. Rows past the sequence are
+      // clipped by the tensor map (and hold zeros: their dS is zero).
+      const bool got = ok && warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
+      ok = got;
+      if (got) {
+        tc_fence_after();
+        const uint32_t stage = sbase + C::OFF_QDO + (it & 1) * 2 * C::TILE;
+#pragma unroll 1
+        for (int round = 0; round < NBOX / 2; ++round) {
+          const int box = g * (NBOX / 2) + round;
+          uint32_t o[32];
+          tmem_load32(tmem_base + AB_T_DP + box * 32 + lane_base, o);
+          if (round + 1 == NBOX / 2) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dq_free);
+          }
+          const uint32_t row = stage + box * (128 * 128) + r * 128;
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            st_shared_v4(row + (uint32_t)((x ^ (r & 7)) * 16), __float_as_uint(__uint_as_float(o[4 * x]) * args.scale),
+                         __float_as_uint(__uint_as_float(o[4 * x + 1]) * args.scale),
+                         __float_as_uint(__uint_as_float(o[4 * x + 2]) * args.scale),
+                         __float_as_uint(__uint_as_float(o[4 * x + 3]) * args.scale));
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_staged0 + 8 * (it & 1));
       }
     }
-    if (warp == 4 && lane == 0) ab_bulk_wait_all();  // the last reduce-adds have landed
-    // dK (x scale) and dV of this key tile: lane = key
+    // dK (x scale) and dV of this key tile: lane = key; each warpgroup half of the columns
     if (ok && n_it > 0 && warp_wait(kv_done, 0, abort_flag)) {
       tc_fence_after();
       // the loads are warp-collective: every lane loads, only real keys store
@@ -358,7 +422,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       __nv_bfloat16* dkr = args.dk + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
       __nv_bfloat16* dvr = args.dv + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
 #pragma unroll 1
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int c = g * (DH / 64); c < (g + 1) * (DH / 64); ++c) {
         uint32_t a[32], b[32];
         tmem_load32x2(tmem_base + AB_T_DK + c * 32 + lane_base, tmem_base + AB_T_DV + c * 32 + lane_base, a, b);
         if (key_row) {

@@ -16,17 +16,17 @@
 // query tile's own ring stage once its products are done). At the end dK_j
 // (x scale) and dV_j are written as bf16.
 //
-// Roles (384 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
+// Roles (640 threads): warp 0 copies K_j, V_j once and Q_i, dO_i per query
 // tile (two-stage ring) with TMA; one thread of warp 1 issues the MMAs; one
 // thread of warp 2 issues the dQ reduce-adds and returns each ring stage to the
-// copies once they have read it; two warpgroups (warps 4-7 and 8-11, one row per
-// thread = one tensor-memory lane) form P and dS for the query columns [0, 64)
-// and [64, 128) of the tile, then stage the dQ partial, and finally write dK and
-// dV, each warpgroup half of the columns.
+// copies once they have read it; four warpgroups (warps 4-19, one row per
+// thread = one tensor-memory lane) form P and dS for the query columns
+// [32g, 32g + 32) of the tile (warpgroup g), then stage the dQ partial, and
+// finally write dK and dV, one 32-column chunk per warpgroup.
 // Tensor memory: dV [0, 128), dK [128, 256), S^T [256, 384), dP^T [384, 512).
-// Each warpgroup writes its P^T (bf16 pairs) over the first 32 of its own 64 S^T
-// columns and its dS^T likewise in dP^T, so that neither overwrites scores the
-// other has not loaded yet; the dQ partial then goes over dP^T, so that the next
+// Each warpgroup writes its P^T (bf16 pairs) over the first 16 of its own 32 S^T
+// columns and its dS^T likewise in dP^T, so that none overwrites scores another
+// has not loaded yet; the dQ partial then goes over dP^T, so that the next
 // tile's S^T product need not wait for it to be read out.
 #pragma once
 
@@ -36,7 +36,8 @@ namespace bpt {
 
 constexpr int AB_BM = 128;  // query rows per tile
 constexpr int AB_BN = 128;  // keys per CTA
-constexpr int AB_THREADS = 384;
+constexpr int AB_THREADS = 640;
+constexpr int AB_EW_WARPS = 16;  // elementwise warps (four warpgroups)
 constexpr int AB_T_DV = 0, AB_T_DK = 128, AB_T_ST = 256, AB_T_DP = 384;
 
 template <int DH>
@@ -78,6 +79,34 @@ __device__ __forceinline__ void ab_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Two 16-column loads of this thread's lane behind one completion wait.
+__device__ __forceinline__ void ab_tmem_load16x2(uint32_t ta, uint32_t (&a)[16], uint32_t tb, uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+        "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// Two 8-column stores of this thread's lane behind one completion wait.
+__device__ __forceinline__ void ab_tmem_store8x2(uint32_t ta, const uint32_t (&a)[8], uint32_t tb,
+                                                 const uint32_t (&b)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%2, %3, %4, %5, %6, %7, %8, %9};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {%10, %11, %12, %13, %14, %15, %16, %17};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(ta),
+      "r"(tb), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(b[0]),
+      "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7])
       : "memory");
 }
 
@@ -164,13 +193,13 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       mbar_init(qdo_empty0 + 8 * i, 1);
     }
     mbar_init(s_ready, 1);
-    mbar_init(p_ready, 8);
+    mbar_init(p_ready, AB_EW_WARPS);
     mbar_init(dq_ready, 1);
-    mbar_init(dq_free, 8);
+    mbar_init(dq_free, AB_EW_WARPS);
     mbar_init(kv_done, 1);
     mbar_init(mma_done, 1);
-    mbar_init(dq_staged0, 8);
-    mbar_init(dq_staged0 + 8, 8);
+    mbar_init(dq_staged0, AB_EW_WARPS);
+    mbar_init(dq_staged0 + 8, AB_EW_WARPS);
     *abort_flag.flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -253,14 +282,14 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         if (!mbar_wait(p_ready, (uint32_t)it & 1u, abort_flag)) break;
         tc_fence_after();
         // dV += P^T dO, dK += dS^T Q (A from tensor memory: 16 queries = 8 columns per
-        // step; queries 0..63 in the first warpgroup's columns, 64..127 in the second's)
+        // step; queries [32g, 32g + 32) in warpgroup g's columns [32g, 32g + 16))
 #pragma unroll
         for (int kk = 0; kk < AB_BM / 16; ++kk)
-          ab_mma_ts(tmem_base + AB_T_DV, tmem_base + AB_T_ST + (kk >> 2) * 64 + (kk & 3) * 8,
+          ab_mma_ts(tmem_base + AB_T_DV, tmem_base + AB_T_ST + (kk >> 1) * 32 + (kk & 1) * 8,
                     smem_desc_sw128(do_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
 #pragma unroll
         for (int kk = 0; kk < AB_BM / 16; ++kk)
-          ab_mma_ts(tmem_base + AB_T_DK, tmem_base + AB_T_DP + (kk >> 2) * 64 + (kk & 3) * 8,
+          ab_mma_ts(tmem_base + AB_T_DK, tmem_base + AB_T_DP + (kk >> 1) * 32 + (kk & 1) * 8,
                     smem_desc_sw128(q_s + kk * 16 * 128, C::ATOM, 1024), id_bmn, (it | kk) != 0);
         // dQ partial = dS K over this key tile (16 keys per step), into the dP^T columns
         // (after the dK product, which reads dS^T there)
@@ -292,36 +321,36 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P, dS, dQ, epilogue
-    const int g = (warp - 4) >> 2;  // warpgroup: query columns [64g, 64g + 64) of the tile
+    const int g = (warp - 4) >> 2;  // warpgroup: query columns [32g, 32g + 32) of the tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tensor-memory lane: a key (P, dS) or a query (dQ)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int key = j0 + r;
     const float sl2 = args.scale_log2;
     const long long bh = (long long)beta * args.heads + head;
-    constexpr int NBOX = DH / 32;  // dQ boxes of 32 columns per query tile, half of them per warpgroup
+    constexpr int NBOX = DH / 32;  // dQ boxes of 32 columns per query tile, one per warpgroup g < NBOX
     // Every warp runs every iteration and every named barrier of it; a wait
     // that gives up only switches the work off (the waits are bounded, and the
     // barriers never see a warp missing).
-    // the query tile's statistics: row r of the first warpgroup holds -lse2, of the
-    // second D; loaded one tile ahead into a register (its latency hides behind the
+    // the query tile's statistics: row r of warpgroup 0 holds -lse2, of warpgroup 1
+    // D; loaded one tile ahead into a register (its latency hides behind the
     // previous tile's dQ work) and staged in shared memory at the top of each tile
     auto stat_of = [&](int i0_) {
       const int t = i0_ + r;
-      if (t >= args.s) return 0.0f;
+      if (t >= args.s || g > 1) return 0.0f;
       return g == 0 ? -args.lse2[bh * args.s + t] : args.dsum[bh * args.s + t];
     };
     float stat_next = n_it > 0 ? stat_of(i_first * AB_BM) : 0.0f;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i0 = (i_first + it) * AB_BM;
-      ab_named_sync(1, 256);  // the previous tile's readers of the statistics are done
+      ab_named_sync(1, 32 * AB_EW_WARPS);  // the previous tile's readers of the statistics are done
       if (g == 0)
         s_lse[r] = stat_next;
-      else
+      else if (g == 1)
         s_dsum[r] = stat_next;
       ok = ok && warp_wait(s_ready, (uint32_t)it & 1u, abort_flag);
-      ab_named_sync(1, 256);  // the statistics are in place
+      ab_named_sync(1, 32 * AB_EW_WARPS);  // the statistics are in place
       if (it + 1 < n_it) stat_next = stat_of(i0 + AB_BM);
       if (ok) {
         tc_fence_after();
@@ -330,14 +359,15 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         const bool key_ok = key < args.s;
         const bool all_used = key_ok && i0 + AB_BM <= args.s && (!args.causal || j0 + AB_BN - 1 <= i0);
 #pragma unroll 1
-        for (int c = 2 * g; c < 2 * g + 2; ++c) {
-          uint32_t sv[32], dp[32];
-          tmem_load32x2(tmem_base + AB_T_ST + c * 32 + lane_base, tmem_base + AB_T_DP + c * 32 + lane_base, sv, dp);
-          uint32_t pk[16], dk[16];
-          const float4* nl4 = reinterpret_cast<const float4*>(s_lse + c * 32);
-          const float4* d4 = reinterpret_cast<const float4*>(s_dsum + c * 32);
+        for (int sc = 0; sc < 2; ++sc) {
+          const int q0 = 32 * g + 16 * sc;  // this sub-chunk's first query column
+          uint32_t sv[16], dp[16];
+          ab_tmem_load16x2(tmem_base + AB_T_ST + q0 + lane_base, sv, tmem_base + AB_T_DP + q0 + lane_base, dp);
+          uint32_t pk[8], dk[8];
+          const float4* nl4 = reinterpret_cast<const float4*>(s_lse + q0);
+          const float4* d4 = reinterpret_cast<const float4*>(s_dsum + q0);
 #pragma unroll
-          for (int x4 = 0; x4 < 8; ++x4) {
+          for (int x4 = 0; x4 < 4; ++x4) {
             const float4 nl = nl4[x4], dd = d4[x4];
             const float nlv[4] = {nl.x, nl.y, nl.z, nl.w}, ddv[4] = {dd.x, dd.y, dd.z, dd.w};
             float p4[4], g4[4];
@@ -351,7 +381,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             if (!all_used) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int q = i0 + c * 32 + 4 * x4 + e;
+                const int q = i0 + q0 + 4 * x4 + e;
                 const bool use = key_ok && q < args.s && (!args.causal || key <= q);
                 p4[e] = use ? p4[e] : 0.0f;
                 g4[e] = use ? g4[e] : 0.0f;
@@ -362,17 +392,17 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             dk[2 * x4] = pack_bf16x2(g4[0], g4[1]);
             dk[2 * x4 + 1] = pack_bf16x2(g4[2], g4[3]);
           }
-          // P^T and dS^T (bf16 pairs) over the first 32 of this warpgroup's 64
+          // P^T and dS^T (bf16 pairs) over the first 16 of this warpgroup's 32
           // columns: columns this warpgroup has already loaded
-          const uint32_t pcol = (uint32_t)(g * 64 + (c & 1) * 16);
-          ab_tmem_store16x2(tmem_base + AB_T_ST + pcol + lane_base, pk, tmem_base + AB_T_DP + pcol + lane_base, dk);
+          const uint32_t pcol = (uint32_t)(32 * g + 8 * sc);
+          ab_tmem_store8x2(tmem_base + AB_T_ST + pcol + lane_base, pk, tmem_base + AB_T_DP + pcol + lane_base, dk);
           // dS^T row of this key into the 128B-swizzled [keys][queries] layout of the dQ operand
-          const uint32_t row = sbase + C::OFF_DS + (c >> 1) * C::ATOM + r * 128;
+          const uint32_t row = sbase + C::OFF_DS + (q0 >> 6) * C::ATOM + r * 128;
 #pragma unroll
-          for (int t4 = 0; t4 < 4; ++t4) {
-            const int chunk = (c & 1) * 4 + t4;
-            st_shared_v4(row + (uint32_t)((chunk ^ (r & 7)) * 16), dk[4 * t4], dk[4 * t4 + 1], dk[4 * t4 + 2],
-                         dk[4 * t4 + 3]);
+          for (int t2 = 0; t2 < 2; ++t2) {
+            const int chunk = ((q0 & 63) >> 3) + t2;
+            st_shared_v4(row + (uint32_t)((chunk ^ (r & 7)) * 16), dk[4 * t2], dk[4 * t2 + 1], dk[4 * t2 + 2],
+                         dk[4 * t2 + 3]);
           }
         }
         fence_async_smem();
@@ -380,41 +410,37 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready);
       }
-      // dQ partial of this query tile (lane = query row), x scale: each warpgroup
-      // stages its half of the columns as 128B-swizzled [128 rows][32 fp32] boxes in
+      // dQ partial of this query tile (lane = query row), x scale: warpgroup g <
+      // NBOX stages its 32 columns as a 128B-swizzled [128 rows][32 fp32] box in
       // the tile's ring stage (its Q and dO have been read by every product once the
-      // dQ partial is complete), releasing the tensor memory after its last load;
-      // warp 2 then adds the boxes into the accumulator. Rows past the sequence are
-      // clipped by the tensor map (and hold zeros: their dS is zero).
+      // dQ partial is complete), after releasing the tensor memory; warp 2 then
+      // adds the boxes into the accumulator. Rows past the sequence are clipped by
+      // the tensor map (and hold zeros: their dS is zero).
       const bool got = ok && warp_wait(dq_ready, (uint32_t)it & 1u, abort_flag);
       ok = got;
       if (got) {
         tc_fence_after();
-        const uint32_t stage = sbase + C::OFF_QDO + (it & 1) * 2 * C::TILE;
-#pragma unroll 1
-        for (int round = 0; round < NBOX / 2; ++round) {
-          const int box = g * (NBOX / 2) + round;
-          uint32_t o[32];
-          tmem_load32(tmem_base + AB_T_DP + box * 32 + lane_base, o);
-          if (round + 1 == NBOX / 2) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dq_free);
-          }
-          const uint32_t row = stage + box * (128 * 128) + r * 128;
+        uint32_t o[32];
+        if (g < NBOX) tmem_load32(tmem_base + AB_T_DP + g * 32 + lane_base, o);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+        if (g < NBOX) {
+          const uint32_t row = sbase + C::OFF_QDO + (it & 1) * 2 * C::TILE + g * (128 * 128) + r * 128;
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             st_shared_v4(row + (uint32_t)((x ^ (r & 7)) * 16), __float_as_uint(__uint_as_float(o[4 * x]) * args.scale),
                          __float_as_uint(__uint_as_float(o[4 * x + 1]) * args.scale),
                          __float_as_uint(__uint_as_float(o[4 * x + 2]) * args.scale),
                          __float_as_uint(__uint_as_float(o[4 * x + 3]) * args.scale));
+          fence_async_smem();
         }
-        fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_staged0 + 8 * (it & 1));
       }
     }
-    // dK (x scale) and dV of this key tile: lane = key; each warpgroup half of the columns
+    // dK (x scale) and dV of this key tile: lane = key; warpgroup g < DH / 32 the
+    // 32-column chunk g
     if (ok && n_it > 0 && warp_wait(kv_done, 0, abort_flag)) {
       tc_fence_after();
       // the loads are warp-collective: every lane loads, only real keys store
@@ -422,7 +448,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       __nv_bfloat16* dkr = args.dk + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
       __nv_bfloat16* dvr = args.dv + ((long long)beta * args.s + key) * args.ld_kv + head * DH;
 #pragma unroll 1
-      for (int c = g * (DH / 64); c < (g + 1) * (DH / 64); ++c) {
+      for (int c = g; c < g + 1 && c < DH / 32; ++c) {
         uint32_t a[32], b[32];
         tmem_load32x2(tmem_base + AB_T_DK + c * 32 + lane_base, tmem_base + AB_T_DV + c * 32 + lane_base, a, b);
         if (key_row) {

@@ -996,8 +996,15 @@ int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads
   return BPT_OK;
 }
 
+// Called after the launches that finish rows [row0, row0 + rows) of out (each
+// FFN wave's FFN-down), so that a caller can start copying them out.
+struct WaveHook {
+  int (*fn)(void* ctx, long long row0, long long rows) = nullptr;
+  void* ctx = nullptr;
+};
+
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
-              int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms) {
+              int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr) {
   int* status = nullptr;
   BPT_TRY(stream_status_word(st, &status));
   const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
@@ -1082,8 +1089,9 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     BPT_TRY(launch_gemm_split<EPI_FFN_UP>(HB, rows, h, h, w1, (long long)kf * h, ffn, sp, h / GEMM_BK, a, sms, st,
                                           status, "gemm_ffn_up"));
     a.bias = p.b2;
-    return launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
-                                           st, status, "gemm_ffn_down");
+    BPT_TRY(launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
+                                            st, status, "gemm_ffn_down"));
+    return hook ? hook->fn(hook->ctx, w.row0, rows) : BPT_OK;
   });
 }
 
@@ -1157,12 +1165,13 @@ struct HostPipe {
   static constexpr int kCopy = 2;  // streams per direction
   cudaStream_t h2d[kCopy] = {}, d2h[kCopy] = {};
   cudaEvent_t ready = nullptr, comp_done[2] = {}, h2d_done[2][kCopy] = {}, d2h_done[2][kCopy] = {};
+  cudaEvent_t wave_done = nullptr;  // re-recorded after each FFN wave (waits take its latest record)
   bool create() {
     for (int c = 0; c < kCopy; ++c)
       if (cudaStreamCreateWithFlags(&h2d[c], cudaStreamNonBlocking) != cudaSuccess ||
           cudaStreamCreateWithFlags(&d2h[c], cudaStreamNonBlocking) != cudaSuccess)
         return false;
-    cudaEvent_t* all[3] = {&ready, &comp_done[0], &comp_done[1]};
+    cudaEvent_t* all[4] = {&ready, &comp_done[0], &comp_done[1], &wave_done};
     for (cudaEvent_t* e : all)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
     for (int k = 0; k < 2; ++k)
@@ -1186,7 +1195,7 @@ struct HostPipe {
       if (h2d[c]) cudaStreamDestroy(h2d[c]);
       if (d2h[c]) cudaStreamDestroy(d2h[c]);
     }
-    cudaEvent_t all[3] = {ready, comp_done[0], comp_done[1]};
+    cudaEvent_t all[4] = {ready, comp_done[0], comp_done[1], wave_done};
     for (cudaEvent_t e : all)
       if (e) cudaEventDestroy(e);
     for (int k = 0; k < 2; ++k)
@@ -1194,6 +1203,32 @@ struct HostPipe {
         if (h2d_done[k][c]) cudaEventDestroy(h2d_done[k][c]);
         if (d2h_done[k][c]) cudaEventDestroy(d2h_done[k][c]);
       }
+  }
+};
+
+// Copies the rows of one finished FFN wave from device to host memory, half on
+// each copy stream, after the launches queued so far on the compute stream.
+struct WaveCopy {
+  HostPipe* pp;
+  cudaStream_t st;
+  const uint8_t* dev;  // result rows on the device
+  uint8_t* host;       // result rows in host memory
+  size_t row_bytes;
+  int waves;
+  static int on_wave(void* ctx, long long row0, long long rows) {
+    WaveCopy& c = *reinterpret_cast<WaveCopy*>(ctx);
+    ++c.waves;
+    if (cudaEventRecord(c.pp->wave_done, c.st) != cudaSuccess) return BPT_ERR_CUDA;
+    const long long half = rows / 2;
+    for (int k = 0; k < HostPipe::kCopy; ++k) {
+      const long long r0 = row0 + (k == 0 ? 0 : half), n = k == 0 ? half : rows - half;
+      if (n <= 0) continue;
+      const size_t off = (size_t)r0 * c.row_bytes, bytes = (size_t)n * c.row_bytes;
+      if (cudaStreamWaitEvent(c.pp->d2h[k], c.pp->wave_done, 0) != cudaSuccess ||
+          cudaMemcpyAsync(c.host + off, c.dev + off, bytes, cudaMemcpyDeviceToHost, c.pp->d2h[k]) != cudaSuccess)
+        return BPT_ERR_CUDA;
+    }
+    return BPT_OK;
   }
 };
 
@@ -1269,15 +1304,21 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
       if (!cu) break;
       LayerPtrs p = w;
       p.x = xdev[k];
-      r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms);
+      // each FFN wave's rows of the result are copied out as soon as they are final
+      // (split over the copy streams), overlapping the waves still to run
+      WaveCopy wc{&pp, st, reinterpret_cast<const uint8_t*>(odev[k]), oi, (size_t)h * 4, 0};
+      const WaveHook hook{&WaveCopy::on_wave, &wc};
+      r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms, &hook);
       if (r != BPT_OK) break;
       cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess;
       for (int c = 0; c < HostPipe::kCopy; ++c) {
+        // a schedule without waves (one FFN launch) copies the whole result here
         const size_t lo = c == 0 ? 0 : o_half, bytes = c == 0 ? o_half : ob - o_half;
-        cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.comp_done[k], 0) == cudaSuccess &&
-             (bytes == 0 || cudaMemcpyAsync(oi + lo, reinterpret_cast<uint8_t*>(odev[k]) + lo, bytes,
-                                            cudaMemcpyDeviceToHost, pp.d2h[c]) == cudaSuccess) &&
-             cudaEventRecord(pp.d2h_done[k][c], pp.d2h[c]) == cudaSuccess;
+        if (wc.waves == 0)
+          cu = cu && cudaStreamWaitEvent(pp.d2h[c], pp.comp_done[k], 0) == cudaSuccess &&
+               (bytes == 0 || cudaMemcpyAsync(oi + lo, reinterpret_cast<uint8_t*>(odev[k]) + lo, bytes,
+                                              cudaMemcpyDeviceToHost, pp.d2h[c]) == cudaSuccess);
+        cu = cu && cudaEventRecord(pp.d2h_done[k][c], pp.d2h[c]) == cudaSuccess;
       }
     }
     if (!cu && r == BPT_OK) r = BPT_ERR_CUDA;

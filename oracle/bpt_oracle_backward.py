@@ -167,6 +167,52 @@ def attention_backward_blockwise(Q, K, V, dO, heads: int, causal: bool, q_block:
     return dQ, dK, dV
 
 
+def attention_backward_rows(q, k, v, do, causal: bool, query_rows, key_rows, block: int = 1024):
+    """Selected rows of dQ, dK and dV of one head of one sequence, by the plain
+    definition, for sequences too long for the full s x s matrices.
+
+    q, k, v, do are [s, dh]. Returns (dQ[query_rows], dK[key_rows],
+    dV[key_rows]). The query rows are visited in blocks of `block` whole rows:
+    for each, the scaled and masked scores S = q k^T / sqrt(dh) of all keys, the
+    row softmax P (max and sum over the whole row), O = P v and D = rowsum(do O);
+    then, with dP = do v^T and dS = P (dP - D) (the softmax Jacobian applied per
+    row, D = rowsum(dP P) = rowsum(do O)):
+        dV[u] = sum_t P[t, u] do[t],   dK[u] = sum_t dS[t, u] q[t] / sqrt(dh)
+    over every query row t (the key rows u taken as columns of each block), and
+    dQ[t] = sum_u dS[t, u] k[u] / sqrt(dh) for the selected query rows t of the
+    block. Nothing is approximated: each row's softmax sees all of its keys.
+    """
+    s, dh = q.shape
+    scale = ob._softmax_scale(dh)
+    query_rows = np.asarray(query_rows, dtype=np.int64)
+    key_rows = np.asarray(key_rows, dtype=np.int64)
+    u_all = np.arange(s)
+    dQ = np.zeros((query_rows.size, dh))
+    dK = np.zeros((key_rows.size, dh))
+    dV = np.zeros((key_rows.size, dh))
+    vJ = v[key_rows]
+    for r0 in range(0, s, block):
+        t = np.arange(r0, min(s, r0 + block))
+        allowed = ob._key_allowed(t, u_all, causal)
+        S = np.where(allowed, (q[t] @ k.T) * scale, -np.inf)
+        E = np.where(allowed, np.exp(S - S.max(axis=1, keepdims=True)), 0.0)
+        P = E / E.sum(axis=1, keepdims=True)
+        del S, E
+        D = np.sum(do[t] * (P @ v), axis=1)
+        # key rows: columns key_rows of P and dS over these query rows
+        PJ = P[:, key_rows]
+        dSJ = PJ * (do[t] @ vJ.T - D[:, None])
+        dV += PJ.T @ do[t]
+        dK += (dSJ.T @ q[t]) * scale
+        # query rows inside this block: whole rows of dS
+        sel = np.nonzero((query_rows >= t[0]) & (query_rows <= t[-1]))[0]
+        if sel.size:
+            li = query_rows[sel] - r0
+            dSI = P[li] * (do[query_rows[sel]] @ v.T - D[li, None])
+            dQ[sel] = (dSI @ k) * scale
+    return dQ, dK, dV
+
+
 def ffn_backward(hid, W1, b1, W2, dy) -> dict:
     """Gradients of the FFN block with its residual, y = hid + max(0, hid W1 +
     b1) W2 + b2 (the standard FFN of the BPT paper review, section 3, with the

@@ -147,3 +147,27 @@ def torch_bf16_layer_grads(x, params, dy, heads, causal):
     y = hid + torch.relu(hid @ P["W1"] + P["b1"]) @ P["W2"] + P["b2"]
     y.backward(dy.to(torch.bfloat16))
     return {"dx": xx.grad, **{"d" + name: t.grad for name, t in P.items()}}
+
+
+def test_attention_backward_full_size_sampled_rows():
+    # The 7B-class shape of the layer benchmarks (b1 s32768 h4096, 32 heads of 128,
+    # causal: 256 key tiles, the dQ of a query tile summed from up to 256 partials,
+    # dK and dV of key tile 0 over 256 query tiles). Rows of one head against the
+    # row oracle, which takes every query row's softmax over all of its keys:
+    # first, last and tile-edge rows of both kinds and a few inside.
+    b, s, h, heads = 1, 32768, 4096, 32
+    bits = {name: bf16_normal(11, 70 + i, (b, s, h)) for i, name in enumerate(("q", "k", "v", "dO"))}
+    t = {k: bi.to_torch(v) for k, v in bits.items()}
+    o, lse2 = bpt.attention_lse(t["q"], t["k"], t["v"], heads, True)
+    g = bpt.attention_backward(t["q"], t["k"], t["v"], o, t["dO"], lse2, heads, True)
+    torch.cuda.synchronize()
+    assert bpt.stream_status() == 0
+    head = 13
+    c = slice(head * 128, (head + 1) * 128)
+    f = {k: bi.to_f64(v[0, :, c]) for k, v in bits.items()}
+    qr = [0, 1, 127, 128, 4095, 16383, 16384, 24577, 32766, 32767]
+    kr = [0, 1, 127, 128, 8191, 16384, 30000, 32640, 32767]
+    dQ, dK, dV = obb.attention_backward_rows(f["q"], f["k"], f["v"], f["dO"], True, qr, kr)
+    for name, got, ref in (("dq", g["dq"][0, qr, c], dQ), ("dk", g["dk"][0, kr, c], dK), ("dv", g["dv"][0, kr, c], dV)):
+        rl2, mx = rel_errors(got, ref)
+        assert rl2 <= 1.5e-2 and mx <= 4e-2, f"{name} (s {s}, head {head}): rel-L2 {rl2:.3e}, max {mx:.3e}"

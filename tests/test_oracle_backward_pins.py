@@ -206,3 +206,34 @@ def test_row_lse_recovers_the_attention_weights_of_torch(causal):
         P = torch.softmax(S, dim=-1).numpy()
         P2 = np.where(np.isfinite(S.numpy()), np.exp2(S.numpy() / np.log(2.0) - lse[:, k, :, None]), 0.0)
         assert np.allclose(P2, P, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("s,block", [(13, 4), (40, 16), (40, 40), (40, 64)])
+def test_sampled_gradient_rows_equal_the_plain_gradient(s, block, causal):
+    # the row-sampled gradient of one head (blocks of whole query rows, ragged
+    # last block) is the plain gradient's rows, every row of either kind
+    rng = np.random.default_rng(s + block)
+    dh = 8
+    Q, K, V, dO = (rng.standard_normal((1, s, dh)) for _ in range(4))
+    dQ, dK, dV = obb.attention_backward(Q, K, V, dO, heads=1, causal=causal)
+    rows = np.arange(s)[::-1]
+    gq, gk, gv = obb.attention_backward_rows(Q[0], K[0], V[0], dO[0], causal, rows, rows[:5], block=block)
+    np.testing.assert_allclose(gq, dQ[0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gk, dK[0, rows[:5]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gv, dV[0, rows[:5]], rtol=0, atol=1e-12)
+
+
+def test_sampled_gradient_rows_match_torch_autograd():
+    # against PyTorch's autograd of its own attention (fp64), causal
+    s, dh = 50, 16
+    rng = np.random.default_rng(3)
+    Q, K, V, dO = (rng.standard_normal((s, dh)) for _ in range(4))
+    q, k, v = (torch.tensor(a, requires_grad=True) for a in (Q, K, V))
+    o = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], is_causal=True)[0]
+    o.backward(torch.tensor(dO))
+    rows = [0, 7, 31, 49]
+    gq, gk, gv = obb.attention_backward_rows(Q, K, V, dO, True, rows, rows, block=16)
+    np.testing.assert_allclose(gq, q.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(gk, k.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(gv, v.grad.numpy()[rows], rtol=1e-10, atol=1e-12)

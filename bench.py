@@ -729,7 +729,7 @@ def max_context_arm(args):
 
 def ffn_backward_arm(args):
     """Throughput of the FFN block's backward (bpt_ffn_backward) at the 7B-class
-    layer's shapes (rows 32768, h 4096, ffn 16384; 4096-row chunks): five
+    layer's shapes (rows 32768, h 4096, ffn 16384; 16384-row chunks): five
     products of 2 rows h ffn flops each (the recomputed intermediate, da,
     dhid, dW1, dW2). Seeded synthetic inputs drawn on the device."""
     import torch
@@ -760,7 +760,7 @@ def ffn_backward_arm(args):
     peaks, src = measured_peaks()
     line = {"metric": "FFN block backward (bpt_ffn_backward) TFLOP/s on 1 B200", "value": flops / (ms / 1e3) / 1e12,
             "unit": "TFLOP/s", "ms": ms, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
-            "config": {"workload": "ffn_backward_rows32768_h4096_f16384", "chunk_rows": 4096},
+            "config": {"workload": "ffn_backward_rows32768_h4096_f16384", "chunk_rows": 16384},
             "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
             "peak_source": f"{src} bf16_tflops (burst)", "device_status": status, "clocks": clocks.summary(),
             "data": "synthetic (torch generator on the device)"}

@@ -304,7 +304,7 @@ int bpt_attention(const void* q, const void* k, const void* v, int b, int s, int
  * db2 [h]. The matrix products take bf16 operands (hid and dy rounded to
  * nearest even) with fp32 accumulation; the weight gradients sum the chunks
  * in fp32. chunk_rows: rows per chunk, rounded down to a multiple of 128 (0 =
- * 4096). workspace: device memory of at least
+ * 16384). workspace: device memory of at least
  * bpt_ffn_backward_workspace_bytes(...) bytes (bf16 copies of a chunk's hid
  * and dy, its recomputed intermediate and da). h and ffn must be multiples of
  * 64. Errors: BPT_ERR_SHAPE, BPT_ERR_NULL, BPT_ERR_ALIGN (16 bytes),

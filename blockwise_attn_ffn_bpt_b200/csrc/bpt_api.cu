@@ -1006,8 +1006,18 @@ struct WaveHook {
   void* ctx = nullptr;
 };
 
+// x arriving in row chunks (bf16 inputs): chunk c, rows [c rows, (c + 1) rows),
+// is in place once ev[c] has completed; the projection then runs chunk by
+// chunk, each launch after its chunk's event, instead of after all of x.
+struct XChunks {
+  int n = 0;
+  long long rows = 0;
+  const cudaEvent_t* ev = nullptr;
+};
+
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
-              int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr) {
+              int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr,
+              const XChunks* xc = nullptr) {
   int* status = nullptr;
   BPT_TRY(stream_status_word(st, &status));
   const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
@@ -1055,11 +1065,24 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.v = V;
     a.ldkv = h;
     a.h = h;
-    if (f32)
+    if (f32) {
       BPT_TRY(launch_gemm_split<EPI_QKV>(xa, tok, 2LL * h, 2LL * h, wqkv, 3LL * h, 3LL * h, 2, h / GEMM_BK, a, sms,
                                          st, status, "gemm_qkv"));
-    else
+    } else if (xc != nullptr && xc->n > 0) {
+      for (int c = 0; c < xc->n; ++c) {
+        const long long r0 = (long long)c * xc->rows, m = std::min(xc->rows, tok - r0);
+        if (m <= 0) break;
+        if (cudaStreamWaitEvent(st, xc->ev[c], 0) != cudaSuccess) return BPT_ERR_CUDA;
+        GemmArgs ac = a;
+        ac.q = QO + r0 * ldq;
+        ac.k = K + r0 * h;
+        ac.v = V + r0 * h;
+        BPT_TRY(launch_gemm<EPI_QKV>(reinterpret_cast<const __nv_bfloat16*>(xa) + r0 * h, m, h, h, wqkv, 3LL * h, ac,
+                                     sms, st, status, "gemm_qkv"));
+      }
+    } else {
       BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, status, "gemm_qkv"));
+    }
   }
 
   // steps 4-10 for every query block at once: each CTA overwrites the Q of its
@@ -1169,6 +1192,8 @@ struct HostPipe {
   cudaStream_t h2d[kCopy] = {}, d2h[kCopy] = {};
   cudaEvent_t ready = nullptr, comp_done[2] = {}, h2d_done[2][kCopy] = {}, d2h_done[2][kCopy] = {};
   cudaEvent_t wave_done = nullptr;  // re-recorded after each FFN wave (waits take its latest record)
+  static constexpr int kXChunks = 4;  // the first input arrives in this many row chunks
+  cudaEvent_t x_chunk[kXChunks] = {};
   bool create() {
     for (int c = 0; c < kCopy; ++c)
       if (cudaStreamCreateWithFlags(&h2d[c], cudaStreamNonBlocking) != cudaSuccess ||
@@ -1182,6 +1207,8 @@ struct HostPipe {
         if (cudaEventCreateWithFlags(&h2d_done[k][c], cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&d2h_done[k][c], cudaEventDisableTiming) != cudaSuccess)
           return false;
+    for (cudaEvent_t& e : x_chunk)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
     return true;
   }
   bool sync_copies() {
@@ -1206,6 +1233,8 @@ struct HostPipe {
         if (h2d_done[k][c]) cudaEventDestroy(h2d_done[k][c]);
         if (d2h_done[k][c]) cudaEventDestroy(d2h_done[k][c]);
       }
+    for (cudaEvent_t e : x_chunk)
+      if (e) cudaEventDestroy(e);
   }
 };
 
@@ -1292,14 +1321,37 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
       const int k = i & 1;
       const uint8_t* xi = reinterpret_cast<const uint8_t*>(x_host) + (size_t)x_stride * i;
       uint8_t* oi = reinterpret_cast<uint8_t*>(out_host) + (size_t)out_stride * i;
-      // x buffer k is free once input i - 2 has been computed
-      for (int c = 0; c < HostPipe::kCopy; ++c) {
-        const size_t lo = c == 0 ? 0 : x_half, bytes = c == 0 ? x_half : xb - x_half;
-        if (i >= 2) cu = cu && cudaStreamWaitEvent(pp.h2d[c], pp.comp_done[k], 0) == cudaSuccess;
-        cu = cu && (bytes == 0 || cudaMemcpyAsync(xdev[k] + lo, xi + lo, bytes, cudaMemcpyHostToDevice,
-                                                  pp.h2d[c]) == cudaSuccess) &&
-             cudaEventRecord(pp.h2d_done[k][c], pp.h2d[c]) == cudaSuccess;
-        cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k][c], 0) == cudaSuccess;
+      // The first input (bf16) comes in row chunks and the projection starts on each
+      // chunk as it lands, so that only the first chunk's copy is exposed; later
+      // inputs arrive while the previous one computes.
+      XChunks xc;
+      const long long xrows = ((long long)tok + HostPipe::kXChunks - 1) / HostPipe::kXChunks;
+      const long long crows = (xrows + 127) / 128 * 128;
+      if (i == 0 && dtype == BPT_DTYPE_BF16 && (long long)tok > crows) {
+        xc.n = (int)(((long long)tok + crows - 1) / crows);
+        xc.rows = crows;
+        xc.ev = pp.x_chunk;
+        for (int c = 0; cu && c < xc.n; ++c) {
+          const size_t lo = (size_t)(c * crows) * h * es;
+          const size_t bytes = (size_t)std::min<long long>(crows, (long long)tok - c * crows) * h * es;
+          // in order on one stream: the link's bandwidth is shared by every copy in
+          // flight in a direction, so chunk 0 lands soonest when it goes alone
+          cu = cudaMemcpyAsync(xdev[k] + lo, xi + lo, bytes, cudaMemcpyHostToDevice, pp.h2d[0]) == cudaSuccess &&
+               cudaEventRecord(pp.x_chunk[c], pp.h2d[0]) == cudaSuccess;
+        }
+        // the copy streams' completion events still mark the whole input
+        for (int c = 0; cu && c < HostPipe::kCopy; ++c)
+          cu = cudaEventRecord(pp.h2d_done[k][c], pp.h2d[c]) == cudaSuccess;
+      } else {
+        // x buffer k is free once input i - 2 has been computed
+        for (int c = 0; c < HostPipe::kCopy; ++c) {
+          const size_t lo = c == 0 ? 0 : x_half, bytes = c == 0 ? x_half : xb - x_half;
+          if (i >= 2) cu = cu && cudaStreamWaitEvent(pp.h2d[c], pp.comp_done[k], 0) == cudaSuccess;
+          cu = cu && (bytes == 0 || cudaMemcpyAsync(xdev[k] + lo, xi + lo, bytes, cudaMemcpyHostToDevice,
+                                                    pp.h2d[c]) == cudaSuccess) &&
+               cudaEventRecord(pp.h2d_done[k][c], pp.h2d[c]) == cudaSuccess;
+          cu = cu && cudaStreamWaitEvent(st, pp.h2d_done[k][c], 0) == cudaSuccess;
+        }
       }
       // out buffer k is free once result i - 2 has been copied out
       for (int c = 0; i >= 2 && c < HostPipe::kCopy; ++c)
@@ -1311,7 +1363,8 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
       // (split over the copy streams), overlapping the waves still to run
       WaveCopy wc{&pp, st, reinterpret_cast<const uint8_t*>(odev[k]), oi, (size_t)h * 4, 0};
       const WaveHook hook{&WaveCopy::on_wave, &wc};
-      r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms, &hook);
+      r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms, &hook,
+                    xc.n > 0 ? &xc : nullptr);
       if (r != BPT_OK) break;
       cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess;
       for (int c = 0; c < HostPipe::kCopy; ++c) {

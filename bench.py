@@ -34,7 +34,7 @@ import bpt_inputs as bi  # noqa: E402
 METRIC = "BPT layer fwd tokens/s and TFLOP/s (% BF16 peak) on 1 B200, vs fp64 oracle"
 DEFAULT_WORKLOAD = "gpt7b_s32768_h4096"
 # wave_rows values of the library's FFN-side schedules (BPT_WAVE_* in include/bpt.h)
-FFN_SCHEDULES = {"default": 0, "chained": -1, "waves": -2}
+FFN_SCHEDULES = {"default": 0, "chained": -1, "waves": -2, "mega": -3}
 L2_BYTES = 126 * 1024 * 1024
 
 

@@ -19,6 +19,11 @@ LIB_PATH = os.path.join(_HERE, "libbpt.so")
 
 BPT_DTYPE_BF16 = 0
 BPT_DTYPE_F32 = 1
+# FFN-side schedules (wave_rows): include/bpt.h
+BPT_WAVE_DEFAULT = 0
+BPT_WAVE_CHAINED = -1
+BPT_WAVE_DEFAULT_WAVES = -2
+BPT_WAVE_MEGA = -3
 
 EXPORTED = (
     "bpt_status_string", "bpt_layer_forward", "bpt_layer_forward_f32", "bpt_layer_workspace_bytes",

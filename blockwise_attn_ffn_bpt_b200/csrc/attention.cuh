@@ -76,6 +76,8 @@ struct AttnArgs {
   float scale_log2; // log2(e) / sqrt(dh)
   int* status;      // status word of the launching stream
   float* lse2;      // [n_seq][heads][t_len]: m + log2(l) of each row (log2 units); written by the LSE build only
+  unsigned* grp_cnt;  // one-launch layer only: per group of grp_rows output rows (flat over the sequences), one
+  int grp_rows;       // count per warp whose 32 rows of one head are stored (release order after the stores)
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]: bf16 A read from tensor memory (K-major).
@@ -89,12 +91,14 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// One CTA's work: query-tile pair `item` of sequence beta0 + zseq (the
+// attention kernel below), or, with MEGA (the one-launch layer), work item
+// `item` in row order with every warp's stored rows counted in args.grp_cnt.
 // LSE: also write each row's log-sum-exp (args.lse2), for the backward; a
 // separate build so that the forward alone carries nothing for it.
-template <int DH, bool LSE = false>
-__global__ void __launch_bounds__(ATT_THREADS, 1)
-    attention_fwd_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                          const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+template <int DH, bool LSE, bool MEGA>
+__device__ __forceinline__ void attention_fwd_body(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                                   const CUtensorMap& tmV, const AttnArgs& args, int item, int zseq) {
   using C = AttnCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -119,14 +123,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // the group's heads. CTAs resident together then touch a few heads, whose
   // K/V stay in L2, and the end of the grid holds the lightest pairs.
   // z = sequence.
-  const int per_group = ATT_HEAD_GROUP * args.n_pairs;
-  const int group = (int)blockIdx.x / per_group;
-  const int within = (int)blockIdx.x - group * per_group;
-  const int heads_in_group = min(ATT_HEAD_GROUP, args.heads - group * ATT_HEAD_GROUP);
-  const int pair_rank = within / heads_in_group;
-  const int head = group * ATT_HEAD_GROUP + (within - pair_rank * heads_in_group);
-  const int pair = args.causal ? (args.n_pairs - 1 - pair_rank) : pair_rank;
-  const int beta = args.beta0 + blockIdx.z;
+  // (MEGA: items in row order, every head of a pair before the next pair, so
+  // that the rows a later out-projection tile needs are finished early.)
+  int head, pair, beta;
+  if constexpr (MEGA) {
+    head = item % args.heads;
+    const int bp = item / args.heads;
+    pair = bp % args.n_pairs;
+    beta = args.beta0 + bp / args.n_pairs;
+  } else {
+    const int per_group = ATT_HEAD_GROUP * args.n_pairs;
+    const int group = item / per_group;
+    const int within = item - group * per_group;
+    const int heads_in_group = min(ATT_HEAD_GROUP, args.heads - group * ATT_HEAD_GROUP);
+    const int pair_rank = within / heads_in_group;
+    head = group * ATT_HEAD_GROUP + (within - pair_rank * heads_in_group);
+    pair = args.causal ? (args.n_pairs - 1 - pair_rank) : pair_rank;
+    beta = args.beta0 + zseq;
+  }
   const int t0 = args.t_start + pair * 2 * ATT_BM;  // first row of query tile 0
   const int t_end = args.t_start + args.t_len;
   int rows_valid[2], n_kv[2];
@@ -378,6 +392,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                          pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
         }
       }
+      if constexpr (MEGA) {
+        // publish this warp's 32 rows of this head (the rows of a 128-row tile lie
+        // in one group: groups are whole tiles)
+        __threadfence();
+        __syncwarp();
+        const long long frow = (long long)(beta - args.beta0) * args.t_len + (tq0 - args.t_start) + quarter * 32;
+        if (lane == 0) red_release_add(args.grp_cnt + frow / args.grp_rows, 1u);
+      }
     }
   }
 
@@ -392,6 +414,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, ATT_TMEM_COLS);
   }
+}
+
+template <int DH, bool LSE = false>
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attention_fwd_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+  attention_fwd_body<DH, LSE, false>(tmQ, tmK, tmV, args, (int)blockIdx.x, (int)blockIdx.z);
 }
 
 }  // namespace bpt

@@ -30,6 +30,7 @@
 
 #include "attention.cuh"
 #include "attention_bwd.cuh"
+#include "layer_mega.cuh"
 #include "attention_pair.cuh"
 #include "bpt.h"
 #include "ffn_chain.cuh"
@@ -159,6 +160,7 @@ bool map_seq_f32(CUtensorMap* m, float* base, int b, int s, int cols) {
 struct DeviceInfo {
   bool checked = false;
   bool ok = false;
+  bool mega_ok = false;  // the one-launch layer kernel was built with the attention's register count
   int sms = 0;
 };
 std::mutex g_dev_mu;
@@ -215,7 +217,11 @@ int check_device(int* sms) {
                    cudaFuncSetAttribute(attention_bwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         AttnBwdCfg<64>::SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_bwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        AttnBwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+                                        AttnBwdCfg<128>::SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(layer_mega_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        mega_smem_bytes<64>()) == cudaSuccess &&
+                   cudaFuncSetAttribute(layer_mega_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        mega_smem_bytes<128>()) == cudaSuccess;
       if (!attrs) return BPT_ERR_CUDA;
       // the attention kernel splits its registers between warpgroups assuming
       // it was built with exactly ATT_REGS_LAUNCH per thread; any other build
@@ -230,12 +236,25 @@ int check_device(int* sms) {
       if (fa64.numRegs != ATT_REGS_LAUNCH || fa128.numRegs != ATT_REGS_LAUNCH || fl64.numRegs != ATT_REGS_LAUNCH ||
           fl128.numRegs != ATT_REGS_LAUNCH || fap.numRegs != ATT_REGS_LAUNCH)
         d.ok = false;
+      cudaFuncAttributes fm64{}, fm128{};
+      if (cudaFuncGetAttributes(&fm64, layer_mega_tcgen05<64>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fm128, layer_mega_tcgen05<128>) != cudaSuccess)
+        return BPT_ERR_CUDA;
+      d.mega_ok = fm64.numRegs == ATT_REGS_LAUNCH && fm128.numRegs == ATT_REGS_LAUNCH;
     }
     d.checked = true;
   }
   if (!d.ok) return BPT_ERR_UNSUPPORTED;
   *sms = d.sms;
   return BPT_OK;
+}
+
+// Whether the one-launch layer kernel may run on the current device (after check_device).
+bool mega_available() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  return g_dev[dev].checked && g_dev[dev].mega_ok;
 }
 
 // ------------------------------------------------------------- stream status
@@ -511,6 +530,7 @@ struct Layout {
   size_t k, v, hid, hb, u, xb, wqkv, wo, w1, w2, cnt, total;
   int wave_rows;
   bool chain;
+  bool mega;  // attention and the chain in one launch: the chain's slots follow K/V instead of aliasing them
   ChainPlan cp;
 };
 
@@ -518,10 +538,16 @@ struct Layout {
 // launch (bf16 inputs), BPT_WAVE_DEFAULT_WAVES and any positive size in one
 // launch per GEMM and wave, and BPT_WAVE_DEFAULT (0) takes kChainByDefault.
 // fp32 inputs (split products) always run per wave.
+// BPT_WAVE_MEGA (bf16, s a multiple of 128) runs attention and the chain in
+// one launch; otherwise it runs as BPT_WAVE_CHAINED (bf16) or per wave (fp32).
 constexpr bool kChainByDefault = false;
+bool use_mega(int dtype, int s, int wave_rows) {
+  return dtype == BPT_DTYPE_BF16 && wave_rows == BPT_WAVE_MEGA && s % ATT_BM == 0;
+}
 bool use_chain(int dtype, int wave_rows) {
   if (dtype != BPT_DTYPE_BF16) return false;
-  return wave_rows == BPT_WAVE_CHAINED || (wave_rows == BPT_WAVE_DEFAULT && kChainByDefault);
+  return wave_rows == BPT_WAVE_CHAINED || wave_rows == BPT_WAVE_MEGA ||
+         (wave_rows == BPT_WAVE_DEFAULT && kChainByDefault);
 }
 
 Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave_rows) {
@@ -532,14 +558,19 @@ Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave
   size_t off;
   if (use_chain(dtype, wave_rows)) {
     L.chain = true;
+    L.mega = use_mega(dtype, s, wave_rows);
     L.cp = chain_plan(b, s, h, ffn);
     L.wave_rows = L.cp.gm * GEMM_BM;
-    L.hid = L.cp.hid;
-    L.hb = L.cp.hb;
-    L.u = L.cp.u;
-    off = std::max(kv_bytes(b, s, h), L.cp.bytes);
+    // the slots alias K/V (dead once attention has run), or follow them when
+    // attention runs in the same launch
+    const size_t base = L.mega ? align_up(kv_bytes(b, s, h), 1024) : 0;
+    L.hid = base + L.cp.hid;
+    L.hb = base + L.cp.hb;
+    L.u = base + L.cp.u;
+    off = L.mega ? base + L.cp.bytes : std::max(kv_bytes(b, s, h), L.cp.bytes);
     L.cnt = off;
-    off = align_up(off + 3 * (size_t)L.cp.groups * sizeof(unsigned), 1024);
+    // the chain's three counters per group; with mega, attention's per group and the ticket
+    off = align_up(off + (3 * (size_t)L.cp.groups + (L.mega ? (size_t)L.cp.groups + 1 : 0)) * sizeof(unsigned), 1024);
   } else {
     const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
     L.wave_rows = wr;
@@ -897,6 +928,89 @@ int launch_chain(const __nv_bfloat16* O, long long ldq, const LayerPtrs& p, long
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 
+// Attention and the chain in one launch (layer_mega.cuh): the same arguments
+// as launch_attention (every sequence, every row, O over Q) and launch_chain.
+int launch_mega(const __nv_bfloat16* QO, long long ldq, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int causal, const Layout& L, uint8_t* ws,
+                float* out, int sms, cudaStream_t st, int* status) {
+  const long long M = (long long)b * s;
+  if (M <= 0) return BPT_OK;
+  const int dh = h / heads;
+  const ChainPlan& cp = L.cp;
+  const long long rows = (long long)cp.gm * GEMM_BM;
+  // attention: every sequence in one grid, items in row order
+  CUtensorMap tq, tk, tv;
+  if (!map_seq(&tq, QO, b, s, h, ldq) || !map_seq(&tk, K, b, s, h, h) || !map_seq(&tv, V, b, s, h, h))
+    return BPT_ERR_CUDA;
+  unsigned* cnt = reinterpret_cast<unsigned*>(ws + L.cnt);
+  AttnArgs aa{};
+  aa.s = s;
+  aa.heads = heads;
+  aa.causal = causal ? 1 : 0;
+  aa.beta0 = 0;
+  aa.t_start = 0;
+  aa.t_len = s;
+  aa.n_pairs = (s + 2 * ATT_BM - 1) / (2 * ATT_BM);
+  aa.o = const_cast<__nv_bfloat16*>(QO);
+  aa.ldo = ldq;
+  aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  aa.status = status;
+  aa.grp_cnt = cnt + 3 * (size_t)cp.groups;
+  aa.grp_rows = (int)rows;
+  // the chain, waiting per group on attention's count
+  ChainArgs a{};
+  a.M = M;
+  a.h = h;
+  a.f = ffn;
+  a.m_tiles = cp.m_tiles;
+  a.gm = cp.gm;
+  a.groups = cp.groups;
+  a.hid_slots = cp.hs;
+  a.u_slots = cp.us;
+  a.n_op = (h + GEMM_BN - 1) / GEMM_BN;
+  a.n_up = (ffn + GEMM_BN - 1) / GEMM_BN;
+  a.n_dn = a.n_op;
+  a.x = reinterpret_cast<const __nv_bfloat16*>(p.x);
+  a.bo = reinterpret_cast<const __nv_bfloat16*>(p.bo);
+  a.b1 = reinterpret_cast<const __nv_bfloat16*>(p.b1);
+  a.b2 = reinterpret_cast<const __nv_bfloat16*>(p.b2);
+  a.hid = reinterpret_cast<float*>(ws + L.hid);
+  a.hb = reinterpret_cast<__nv_bfloat16*>(ws + L.hb);
+  a.u = reinterpret_cast<__nv_bfloat16*>(ws + L.u);
+  a.out = out;
+  a.op_cnt = cnt;
+  a.up_cnt = cnt + cp.groups;
+  a.dn_cnt = cnt + 2 * (size_t)cp.groups;
+  a.status = status;
+  a.att_cnt = aa.grp_cnt;
+  a.att_heads = heads;
+  CUtensorMap tO, tHb, tU, tWo, tW1, tW2;
+  if (!map_rows(&tO, QO, M, h, ldq, GEMM_BM) || !map_rows(&tHb, a.hb, cp.hs * rows, h, h, GEMM_BM) ||
+      !map_rows(&tU, a.u, cp.us * rows, ffn, ffn, GEMM_BM) || !map_rows(&tWo, p.Wo, h, h, h, 64) ||
+      !map_rows(&tW1, p.W1, h, ffn, ffn, 64) || !map_rows(&tW2, p.W2, ffn, h, h, 64))
+    return BPT_ERR_CUDA;
+  MegaArgs mg{};
+  mg.ticket = cnt + 4 * (size_t)cp.groups;
+  const long long n_att = (long long)b * aa.n_pairs * heads;
+  const long long tiles = (long long)cp.m_tiles * (a.n_op + a.n_up + a.n_dn);
+  const long long n_chain = std::min<long long>(tiles, sms);
+  if (n_att + n_chain > 0x7fffffffLL) return BPT_ERR_SHAPE;
+  mg.n_att = (int)n_att;
+  if (cudaMemsetAsync(cnt, 0, (4 * (size_t)cp.groups + 1) * sizeof(unsigned), st) != cudaSuccess)
+    return BPT_ERR_CUDA;
+  {
+    LaunchScope ls("layer_mega", st);
+    const unsigned grid = (unsigned)(n_att + n_chain);
+    if (dh == 64)
+      layer_mega_tcgen05<64><<<grid, ATT_THREADS, mega_smem_bytes<64>(), st>>>(tq, tk, tv, tO, tHb, tU, tWo, tW1,
+                                                                               tW2, aa, a, mg);
+    else
+      layer_mega_tcgen05<128><<<grid, ATT_THREADS, mega_smem_bytes<128>(), st>>>(tq, tk, tv, tO, tHb, tU, tWo, tW1,
+                                                                                 tW2, aa, a, mg);
+  }
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+}
+
 __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, long long n) {
   const long long n4 = n / 4;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
@@ -1086,7 +1200,10 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   }
 
   // steps 4-10 for every query block at once: each CTA overwrites the Q of its
-  // own rows and head with their attention output
+  // own rows and head with their attention output (or, in the one-launch
+  // schedule, attention and the whole FFN side together)
+  if (L.mega && mega_available())
+    return launch_mega(QO, ldq, K, V, p, b, s, h, heads, ffn, causal, L, ws, out, sms, st, status);
   BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st, status));
 
   // step 11 for every query block: out-projection, residuals and FFN

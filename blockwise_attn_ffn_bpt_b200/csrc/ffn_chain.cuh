@@ -68,6 +68,10 @@ struct ChainArgs {
   unsigned* up_cnt;        // [groups]
   unsigned* dn_cnt;        // [groups]
   int* status;
+  // one-launch layer only (else null): attention's count of stored warps per
+  // group, complete at 4 x (the group's M-tiles) x att_heads
+  const unsigned* att_cnt;
+  int att_heads;
 };
 
 struct ChainTile {
@@ -144,36 +148,6 @@ __host__ __device__ __forceinline__ long long chain_num_tiles(const ChainArgs& a
   return (long long)a.m_tiles * (a.n_op + a.n_up + a.n_dn);
 }
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Wait until *cnt >= target (bounded, like the mbarrier waits).
-__device__ __forceinline__ bool counter_wait(const unsigned* cnt, unsigned target, const Abort& ab) {
-  if (ld_acquire_u32(cnt) >= target) return true;
-  const unsigned long long t0 = global_timer_ns();
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire_u32(cnt) >= target) return true;
-    if (*ab.flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-      *ab.flag = 1;
-      atomicExch(ab.status, (int)BPT_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // 32 fp32 values read through L2 only (the line may have been written by
 // another SM since this SM last cached it).
 __device__ __forceinline__ void load32_f32_cg(const float* p, float (&v)[32]) {
@@ -185,11 +159,12 @@ __device__ __forceinline__ void load32_f32_cg(const float* p, float (&v)[32]) {
   }
 }
 
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    ffn_chain_tcgen05(const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmHb,
-                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmWo,
-                      const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
-                      const ChainArgs args) {
+// One CTA's share of the queue: CTA `cta` of `n_ctas` takes tiles cta,
+// cta + n_ctas, ... Warps 0-5 work (producer, MMA issuer, four epilogue warps);
+// any further warps of the block only pass the final barrier.
+__device__ __forceinline__ void ffn_chain_body(const CUtensorMap& tmO, const CUtensorMap& tmHb, const CUtensorMap& tmU,
+                                               const CUtensorMap& tmWo, const CUtensorMap& tmW1,
+                                               const CUtensorMap& tmW2, const ChainArgs& args, int cta, int n_ctas) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
@@ -244,20 +219,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t issued = 0, last_parity = 0;
       // latest group seen complete, per GEMM (groups complete in order of the
       // queue's steps, so "group g complete" covers the groups before it)
-      int done_op = -1, done_up = -1, done_dn = -1;
+      int done_op = -1, done_up = -1, done_dn = -1, done_att = -1;
       auto need = [&](int& done, const unsigned* cnt, int g, int n_tiles_per_mt) -> bool {
         if (g <= done) return true;
         if (!counter_wait(cnt + g, 4u * chain_group_mt(args, g) * n_tiles_per_mt, abort_flag)) return false;
         done = g;
         return true;
       };
-      for (long long t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (long long t = cta; t < num_tiles; t += n_ctas) {
         const ChainTile ct = chain_tile(args, t);
         // inputs of this tile, and the scratch slot it writes, are ready
-        const int d0 = done_op, d1 = done_up, d2 = done_dn;
+        const int d0 = done_op, d1 = done_up, d2 = done_dn, d3 = done_att;
         bool ok = true;
         if (ct.kind == CK_OP) {
-          if (ct.g >= args.hid_slots) ok = need(done_dn, args.dn_cnt, ct.g - args.hid_slots, args.n_dn);
+          if (args.att_cnt != nullptr) ok = need(done_att, args.att_cnt, ct.g, args.att_heads);
+          if (ok && ct.g >= args.hid_slots) ok = need(done_dn, args.dn_cnt, ct.g - args.hid_slots, args.n_dn);
         } else if (ct.kind == CK_UP) {
           ok = need(done_op, args.op_cnt, ct.g, args.n_op);
           if (ok && ct.g >= args.u_slots) ok = need(done_dn, args.dn_cnt, ct.g - args.u_slots, args.n_dn);
@@ -267,7 +243,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!ok) break;
         // another CTA's stores become visible to this thread's tensor-memory-
         // access loads once a counter has been acquired
-        if (d0 != done_op || d1 != done_up || d2 != done_dn) fence_proxy_async_global();
+        if (d0 != done_op || d1 != done_up || d2 != done_dn || d3 != done_att) fence_proxy_async_global();
         const CUtensorMap* ta = ct.kind == CK_OP ? &tmO : (ct.kind == CK_UP ? &tmHb : &tmU);
         const CUtensorMap* tb = ct.kind == CK_OP ? &tmWo : (ct.kind == CK_UP ? &tmW1 : &tmW2);
         const int a_row = ct.kind == CK_OP ? ct.g * group_rows + ct.mt * GEMM_BM
@@ -304,7 +280,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (long long t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      for (long long t = cta; t < num_tiles; t += n_ctas, ++it) {
         const ChainTile ct = chain_tile(args, t);
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
@@ -332,11 +308,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       mma_commit(mma_done);
     }
-  } else {
+  } else if (warp < 6) {
     // -------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
     int it = 0;
-    for (long long t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (long long t = cta; t < num_tiles; t += n_ctas, ++it) {
       const ChainTile ct = chain_tile(args, t);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -401,6 +377,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
   }
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    ffn_chain_tcgen05(const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmHb,
+                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmWo,
+                      const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
+                      const ChainArgs args) {
+  ffn_chain_body(tmO, tmHb, tmU, tmWo, tmW1, tmW2, args, (int)blockIdx.x, (int)gridDim.x);
 }
 
 }  // namespace bpt

@@ -104,6 +104,37 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const A
   return __all_sync(0xffffffffu, ok);
 }
 
+// ---------------------------------------------------------------- counters between CTAs
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *cnt >= target (bounded, like the mbarrier waits).
+__device__ __forceinline__ bool counter_wait(const unsigned* cnt, unsigned target, const Abort& ab) {
+  if (ld_acquire_u32(cnt) >= target) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_u32(cnt) >= target) return true;
+    if (*ab.flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *ab.flag = 1;
+      atomicExch(ab.status, (int)BPT_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

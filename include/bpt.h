@@ -91,6 +91,8 @@ typedef enum bpt_dtype {
 #define BPT_WAVE_DEFAULT 0         /* the library's choice (per-GEMM waves) */
 #define BPT_WAVE_CHAINED (-1)      /* every query block's FFN side in one launch (bf16 inputs) */
 #define BPT_WAVE_DEFAULT_WAVES (-2) /* one launch per GEMM and wave, waves of the library's default size */
+#define BPT_WAVE_MEGA (-3)         /* attention and the FFN side in one persistent launch (bf16, s % 128 == 0;
+                                      otherwise as BPT_WAVE_CHAINED, or per wave for fp32 inputs) */
 
 /* Human-readable name of a status code (static string, never NULL). A library
  * utility; the pages have no counterpart. */
@@ -155,7 +157,12 @@ int bpt_layer_forward_f32(const float* x, const float* Wqkv, const float* bqkv, 
  * sequences; otherwise the library picks the whole number of query
  * blocks (or of whole sequences) that its model of its GEMM tile
  * rounds finds fastest, with scratch of at most 1.5x the K/V bytes (or of
- * about 4096 rows). The fp32 entry adds bf16 copies of x and the weights. */
+ * about 4096 rows). BPT_WAVE_MEGA (bf16 inputs, s a multiple of 128) runs
+ * attention and the chained FFN side in one persistent launch whose
+ * out-projection tiles wait (bounded) for their rows' attention output; the
+ * chain's slots then follow the K/V region instead of aliasing it (K and V are
+ * still read while the FFN side of earlier rows runs). The fp32 entry adds
+ * bf16 copies of x and the weights. */
 size_t bpt_layer_workspace_bytes(int dtype, int b, int s, int h, int heads, int q_block, int kv_block,
                                  int wave_rows);
 

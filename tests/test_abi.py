@@ -128,6 +128,35 @@ def chain_workspace(b, s, h, f):
     return _up(max(kv, slots) + 3 * groups * 4), kv, slots
 
 
+def chain_groups(b, s, h, f):
+    """Row groups of the chained FFN side (the same choice as chain_workspace)."""
+    mt = -(-(b * s) // 128)
+    kv = 2 * _up(b * s * h * 2)
+    for gm in (16, 8, 4, 2, 1):
+        groups = -(-mt // gm)
+        hs, us, rows = min(3, groups), min(2, groups), gm * 128
+        if _up(hs * rows * h * 4) + _up(hs * rows * h * 2) + _up(us * rows * f * 2) <= max(kv // 2 * 3, 32 << 20):
+            return groups
+    return groups
+
+
+def test_one_launch_layer_workspace_puts_the_slots_after_the_keys_and_values():
+    # BPT_WAVE_MEGA: attention runs while the FFN side of earlier rows does, so
+    # the chain's slots follow the K/V region instead of aliasing it; then the
+    # counters (three per group for the chain, one per group for attention, one
+    # ticket)
+    for b, s, h, heads, qb, kvb in [(1, 32768, 4096, 32, 1024, 2048), (2, 4096, 256, 2, 128, 256),
+                                    (1, 8192, 2048, 16, 512, 512), (1, 1152, 256, 4, 128, 128)]:
+        _, kv, slots = chain_workspace(b, s, h, 4 * h)
+        groups = chain_groups(b, s, h, 4 * h)
+        assert bpt.workspace_bytes(0, b, s, h, heads, qb, kvb, -3) == _up(kv + slots + (4 * groups + 1) * 4)
+    # at the 32k-token 7B shape that is 2048-row groups: 285 MiB more than the K/V region
+    assert bpt.workspace_bytes(0, 1, 32768, 4096, 32, 1024, 2048, -3) - 2 * 32768 * 4096 * 2 < 300 << 20
+    # s not a multiple of 128: as the chained schedule; fp32 inputs: per wave, as by default
+    assert bpt.workspace_bytes(0, 3, 1000, 192, 3, 200, 125, -3) == chain_workspace(3, 1000, 192, 768)[0]
+    assert bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64, -3) == bpt.workspace_bytes(1, 1, 256, 256, 4, 64, 64)
+
+
 def test_workspace_bytes_follow_the_layout():
     def wave(b, s, h, wr):
         # explicit wave: K/V region, or one wave's fp32 hid, its bf16 copy and the bf16 U (wave rows x 4h)

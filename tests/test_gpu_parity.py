@@ -261,15 +261,39 @@ def test_layer_result_does_not_depend_on_the_wave(wave_rows):
     assert_parity(got, ref, f"wave_rows={wave_rows}")
 
 
-@pytest.mark.parametrize("schedule", [-1, -2], ids=["chained", "default-waves"])
+@pytest.mark.parametrize("schedule", [-1, -2, -3], ids=["chained", "default-waves", "one-launch"])
 def test_both_ffn_schedules_match_the_oracle(schedule):
     # the FFN side in one launch (BPT_WAVE_CHAINED: four 2048-row groups here,
-    # so both scratch slots are reused) and in one launch per GEMM and wave
-    # (BPT_WAVE_DEFAULT_WAVES) compute the same layer
+    # so both scratch slots are reused), in one launch per GEMM and wave
+    # (BPT_WAVE_DEFAULT_WAVES) and attention with the FFN side in one launch
+    # (BPT_WAVE_MEGA) compute the same layer
     shape = bi.LayerShape(2, 4096, 256, 2, 128, 256, True)
     inp = bi.make_inputs(shape, seed=9)
     got = run_layer(shape, inp, wave_rows=schedule, workspace=True)
     assert_parity(got, oracle_full(shape, inp), f"ffn schedule {schedule}")
+
+
+MEGA_SHAPES = [
+    bi.LayerShape(2, 4096, 256, 2, 128, 256, True),      # dh 128, row groups reusing the scratch slots
+    bi.LayerShape(1, 1152, 256, 4, 128, 128, False),     # dh 64, an odd number of query tiles
+    bi.WORKLOADS["gpt1b_s8192_h2048"],                   # the 1B-class workload
+]
+
+
+@pytest.mark.parametrize("shape", MEGA_SHAPES, ids=["b2_s4096", "s1152_dh64", "gpt1b"])
+def test_one_launch_layer_equals_the_chained_schedule(shape):
+    # attention and the FFN side in one persistent launch (BPT_WAVE_MEGA) run the
+    # same arithmetic as attention followed by the chained FFN side: equal bit for
+    # bit; and it is that kernel which ran
+    inp = bi.make_inputs(shape, seed=21)
+    chained = run_layer(shape, inp, wave_rows=-1, workspace=True)
+    bpt.set_kernel_timing(True)
+    bpt.kernel_times()
+    mega = run_layer(shape, inp, wave_rows=-3, workspace=True)
+    kinds = bpt.kernel_times()
+    bpt.set_kernel_timing(False)
+    assert "layer_mega" in kinds and "attention" not in kinds and "ffn_chain" not in kinds, kinds
+    assert np.array_equal(mega, chained)
 
 
 @pytest.mark.parametrize("q_scale,max_abs", [(2.0, MAX_ABS), (8.0, 0.1)])

@@ -202,6 +202,12 @@ int check_device(int* sms) {
                                         GP_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_FFN_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_BWD_DA, 0, 0>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_BWD_DHID, 0, 0>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GP_SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(gemm_pair_tcgen05<EPI_GRAD, 1, 1>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GP_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(ffn_chain_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         GEMM_SMEM_BYTES) == cudaSuccess &&
                    cudaFuncSetAttribute(attention_pair_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -657,14 +663,29 @@ template <int MODE, int A_MN, int B_MN>
 int launch_gemm_t(const void* A, long long lda, const void* B, long long ldb, long long M, long long N, long long K,
                   GemmArgs args, int sms, cudaStream_t st, int* status, const char* name) {
   if (M <= 0 || N <= 0) return BPT_OK;
-  CUtensorMap ta, tb;
-  const bool ok_a = A_MN ? map_rows(&ta, A, K, M, lda, 64) : map_rows(&ta, A, M, K, lda, GEMM_BM);
-  const bool ok_b = B_MN ? map_rows(&tb, B, K, N, ldb, 64) : map_rows(&tb, B, N, K, ldb, GEMM_BN);
-  if (!ok_a || !ok_b) return BPT_ERR_CUDA;
   args.status = status;
   args.M = (int)M;
   args.N = (int)N;
   args.K = (int)((K + GEMM_BK - 1) / GEMM_BK * GEMM_BK);
+  CUtensorMap ta, tb;
+  if (BPT_PAIR_GEMM) {
+    // 256 x 256 tiles on SM pairs: each CTA maps its own 128 rows of A and its
+    // 128-column half of B
+    const bool ok_a = A_MN ? map_rows(&ta, A, K, M, lda, 64) : map_rows(&ta, A, M, K, lda, 128);
+    const bool ok_b = B_MN ? map_rows(&tb, B, K, N, ldb, 64) : map_rows(&tb, B, N, K, ldb, 128);
+    if (!ok_a || !ok_b) return BPT_ERR_CUDA;
+    args.m_tiles = (int)((M + GP_BM - 1) / GP_BM);
+    args.n_tiles = (int)((N + GP_BN - 1) / GP_BN);
+    const int pairs = std::min(args.m_tiles * args.n_tiles, sms / 2);
+    {
+      LaunchScope ls(name, st);
+      gemm_pair_tcgen05<MODE, A_MN, B_MN><<<2 * pairs, GEMM_THREADS, GP_SMEM_BYTES, st>>>(ta, tb, args);
+    }
+    return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
+  }
+  const bool ok_a = A_MN ? map_rows(&ta, A, K, M, lda, 64) : map_rows(&ta, A, M, K, lda, GEMM_BM);
+  const bool ok_b = B_MN ? map_rows(&tb, B, K, N, ldb, 64) : map_rows(&tb, B, N, K, ldb, GEMM_BN);
+  if (!ok_a || !ok_b) return BPT_ERR_CUDA;
   args.m_tiles = (int)((M + GEMM_BM - 1) / GEMM_BM);
   args.n_tiles = (int)((N + GEMM_BN - 1) / GEMM_BN);
   const int grid = std::min(args.m_tiles * args.n_tiles, sms);

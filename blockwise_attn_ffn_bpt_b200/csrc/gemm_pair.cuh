@@ -98,7 +98,11 @@ __device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles
 }
 
 // args.m_tiles / n_tiles count 256 x 256 pair tiles; grid = 2 x pairs.
-template <int MODE>
+// Operand layouts as in gemm_bf16_tcgen05: A_MN = 1, A stored [K, M] (this
+// CTA's 128 rows as two [64 k][64 m] boxes), else [M, K] (one [128 m][64 k]
+// box); B_MN = 1, B stored [K, N] (this CTA's 128 columns as two [64 k][64 n]
+// boxes), else [N, K] (one [128 n][64 k] box).
+template <int MODE, int A_MN = 0, int B_MN = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmArgs args) {
@@ -165,10 +169,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * GP_STAGE_BYTES);
           const uint32_t fb = full_leader0 + 8 * stage;
           const uint32_t sa = smem_base + stage * GP_STAGE_BYTES;
-          tma_load_2d_pair(sa, &tmA, fb, kb * GEMM_BK, m0);
+          if constexpr (A_MN) {
 #pragma unroll
-          for (int j = 0; j < GP_BN / 2 / 64; ++j)
-            tma_load_2d_pair(sa + GP_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);
+            for (int j = 0; j < 128 / 64; ++j)
+              tma_load_2d_pair(sa + j * GEMM_B_BOX_BYTES, &tmA, fb, m0 + 64 * j, kb * GEMM_BK);
+          } else {
+            tma_load_2d_pair(sa, &tmA, fb, kb * GEMM_BK, m0);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int j = 0; j < GP_BN / 2 / 64; ++j)
+              tma_load_2d_pair(sa + GP_A_BYTES + j * GEMM_B_BOX_BYTES, &tmB, fb, n0 + 64 * j, kb * GEMM_BK);
+          } else {
+            tma_load_2d_pair(sa + GP_A_BYTES, &tmB, fb, kb * GEMM_BK, n0);
+          }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == GP_STAGES) { stage = 0; phase ^= 1; }
@@ -190,7 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     if (leader && lane == 0) {
       // ------------------------------------------------------------ MMA issuer (leader)
-      const uint32_t idesc = idesc_bf16_f32(GP_BM, GP_BN, 0, 1);
+      const uint32_t idesc = idesc_bf16_f32(GP_BM, GP_BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -208,8 +222,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sb = sa + GP_A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(sb + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024);
+            const uint64_t adesc = A_MN ? smem_desc_sw128(sa + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024)
+                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bdesc = B_MN ? smem_desc_sw128(sb + kk * 16 * 128, GEMM_B_BOX_BYTES, 1024)
+                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
             mma_bf16_ss_pair(d, adesc, bdesc, idesc, (kb | kk) != 0);
           }
           mma_commit_pair(empty0 + 8 * stage);

@@ -91,6 +91,22 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Work item `item` of the one-launch layer: query-tile pairs in row order, every
+// head of a pair before the next pair (host code, the schedule's tests, uses it too).
+__host__ __device__ __forceinline__ void mega_item_coords(const AttnArgs& a, int item, int& beta, int& head,
+                                                          int& pair) {
+  head = item % a.heads;
+  const int bp = item / a.heads;
+  pair = bp % a.n_pairs;
+  beta = a.beta0 + bp / a.n_pairs;
+}
+
+// The first of the output rows (flat over the call's sequences) that a warp of
+// a query tile stores, and so the group whose count it raises.
+__host__ __device__ __forceinline__ long long mega_warp_row(const AttnArgs& a, int beta, int tq0, int quarter) {
+  return (long long)(beta - a.beta0) * a.t_len + (tq0 - a.t_start) + quarter * 32;
+}
+
 // One CTA's work: query-tile pair `item` of sequence beta0 + zseq (the
 // attention kernel below), or, with MEGA (the one-launch layer), work item
 // `item` in row order with every warp's stored rows counted in args.grp_cnt.
@@ -127,10 +143,7 @@ __device__ __forceinline__ void attention_fwd_body(const CUtensorMap& tmQ, const
   // that the rows a later out-projection tile needs are finished early.)
   int head, pair, beta;
   if constexpr (MEGA) {
-    head = item % args.heads;
-    const int bp = item / args.heads;
-    pair = bp % args.n_pairs;
-    beta = args.beta0 + bp / args.n_pairs;
+    mega_item_coords(args, item, beta, head, pair);
   } else {
     const int per_group = ATT_HEAD_GROUP * args.n_pairs;
     const int group = item / per_group;
@@ -397,8 +410,7 @@ __device__ __forceinline__ void attention_fwd_body(const CUtensorMap& tmQ, const
         // in one group: groups are whole tiles)
         __threadfence();
         __syncwarp();
-        const long long frow = (long long)(beta - args.beta0) * args.t_len + (tq0 - args.t_start) + quarter * 32;
-        if (lane == 0) red_release_add(args.grp_cnt + frow / args.grp_rows, 1u);
+        if (lane == 0) red_release_add(args.grp_cnt + mega_warp_row(args, beta, tq0, quarter) / args.grp_rows, 1u);
       }
     }
   }

@@ -726,11 +726,84 @@ __global__ void __launch_bounds__(1024) colsum_kernel(const T* __restrict__ src,
   }
 }
 
+// The same column sums with 16-byte loads: a cluster of CS_SPLIT CTAs shares one
+// strip of 32 x (16 / sizeof(T)) columns, each CTA a contiguous eighth of the
+// rows; in a CTA, warp w takes rows w, w + CS_WARPS, ... and each lane one
+// 16-byte vector of a row (a warp reads 512 contiguous bytes per row). The sums
+// are taken in a fixed order (rows in order within a thread, then the warps in
+// order, then the CTAs of the cluster in rank order, read by rank 0 from the
+// others' shared memory), so results are the same on every run.
+constexpr int CS_SPLIT = 8;
+constexpr int CS_WARPS = 32;
+template <typename T>
+__global__ void __cluster_dims__(1, CS_SPLIT, 1) __launch_bounds__(CS_WARPS * 32)
+    colsum_vec_kernel(const T* __restrict__ src, long long rows, int cols, long long ld, float* out, int accumulate) {
+  constexpr int VEC = 16 / (int)sizeof(T);
+  constexpr int CW = 32 * VEC;  // columns of the strip
+  __shared__ float part[CS_WARPS][CW];  // [warp][i * 32 + lane]: column lane * VEC + i
+  __shared__ float csum[CW];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int rank = (int)blockIdx.y;  // the cluster spans grid.y (= CS_SPLIT)
+  const long long c0 = (long long)blockIdx.x * CW + lane * VEC;
+  const long long per = (rows + CS_SPLIT - 1) / CS_SPLIT;
+  const long long rb = rank * per, re = rows < rb + per ? rows : rb + per;
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.0f;
+  if (c0 < cols) {
+#pragma unroll 4
+    for (long long r = rb + w; r < re; r += CS_WARPS) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(src + r * ld + c0));
+      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += __uint_as_float(u[i] << 16);
+          acc[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += __uint_as_float(u[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) part[w][i * 32 + lane] = acc[i];
+  __syncthreads();
+  for (int t = threadIdx.x; t < CW; t += blockDim.x) {
+    float v = 0.0f;
+    for (int k = 0; k < CS_WARPS; ++k) v += part[k][t];
+    csum[t] = v;
+  }
+  cluster_sync_all();  // every CTA's strip sum is in its shared memory
+  if (rank == 0) {
+    for (int t = threadIdx.x; t < CW; t += blockDim.x) {
+      const long long col = (long long)blockIdx.x * CW + (t & 31) * VEC + (t >> 5);
+      float v = 0.0f;
+      for (int k = 0; k < CS_SPLIT; ++k) {
+        float x;
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(mapa_shared(smem_addr(csum + t), k)) : "memory");
+        v += x;
+      }
+      if (col < cols) out[col] = accumulate ? out[col] + v : v;
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while rank 0 may still read its shared memory
+}
+
+// Column sums (deterministic): the vector kernel when rows are 16-byte aligned
+// vectors, else one thread per column.
 template <typename T>
 int launch_colsum(const T* src, long long rows, int cols, long long ld, float* out, int accumulate, cudaStream_t st) {
   if (cols <= 0) return BPT_OK;
   LaunchScope ls("colsum", st);
-  colsum_kernel<T><<<(cols + 31) / 32, 1024, 0, st>>>(src, rows, cols, ld, out, accumulate);
+  constexpr int VEC = 16 / (int)sizeof(T);
+  if (cols % VEC == 0 && ld % VEC == 0 && aligned16(src)) {
+    const dim3 grid((unsigned)((cols + 32 * VEC - 1) / (32 * VEC)), CS_SPLIT);
+    colsum_vec_kernel<T><<<grid, CS_WARPS * 32, 0, st>>>(src, rows, cols, ld, out, accumulate);
+  } else {
+    colsum_kernel<T><<<(cols + 31) / 32, 1024, 0, st>>>(src, rows, cols, ld, out, accumulate);
+  }
   return cudaGetLastError() == cudaSuccess ? BPT_OK : BPT_ERR_CUDA;
 }
 

@@ -161,3 +161,35 @@ def test_roofline_frac_is_against_the_burst_peak():
     # without a clock key the fallback's clock is used
     assert bench.sustained_clock_mhz({"bf16_tflops": 1.0}) == bench.FALLBACK_PEAKS["bf16_tflops_sustained_sm_mhz"]
     assert bench.sustained_clock_mhz({"x": {"sustained_clock_mhz": 1234}}) == 1234.0
+
+
+def test_clock_sampler_reads_nvml_only_inside_the_timed_region(monkeypatch):
+    # a fake NVML: SM clock 1500 then 1900 MHz, the power-cap bit from the third read on
+    import sys
+    import time
+    import types
+    reads = {"n": 0}
+
+    def clock(handle, kind):
+        reads["n"] += 1
+        return 1500 if reads["n"] <= 2 else 1900
+
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None, nvmlShutdown=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, k: 1965,
+        nvmlDeviceGetClockInfo=clock,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 if reads["n"] >= 3 else 0x0)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    import bench
+    c = bench.ClockSampler(3)
+    assert reads["n"] == 0  # nothing read before the region starts
+    with c:
+        time.sleep(0.25)
+    n_in = reads["n"]
+    time.sleep(0.1)
+    assert reads["n"] == n_in  # and nothing after it ends
+    s = c.summary()
+    assert s["samples"] == n_in >= 5 and s["sm_max_mhz"] == 1965.0
+    assert s["sm_mhz"] == 1900.0 and s["reasons"] == ["sw_power_cap"]

@@ -241,6 +241,31 @@ def ffn_backward(hid, W1, b1, W2, dy) -> dict:
     return g
 
 
+def ffn_backward_samples(hid, W1, b1, W2, dy, rows, f_cols, h_cols) -> dict:
+    """Selected parts of ffn_backward's gradients, for problems whose [rows, ffn]
+    intermediate is too large to form (hid, dy: [R, h]): rows `rows` of dhid,
+    columns `f_cols` of dW1 and db1, the block dW2[f_cols, h_cols], and all of
+    db2; plus the pre-activations a = hid W1 + b1 they used (rows `rows`, and
+    columns `f_cols` over every row), so that a caller can see where a ReLU
+    decision lies within rounding of zero. Same definitions as ffn_backward:
+        da = (dy W2^T) [a > 0];  dhid = dy + da W1^T;  dW1 = hid^T da
+        db1 = sum da;  dW2 = u^T dy with u = max(0, a);  db2 = sum dy
+    taken only over the needed rows or columns of a, u and da.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    f_cols = np.asarray(f_cols, dtype=np.int64)
+    h_cols = np.asarray(h_cols, dtype=np.int64)
+    # rows of dhid need whole rows of da
+    a_rows = hid[rows] @ W1 + b1
+    da_rows = (dy[rows] @ W2.T) * _relu_grad(a_rows)
+    # columns of dW1, db1 and dW2 need whole columns of a (over every row)
+    a_cols = hid @ W1[:, f_cols] + b1[f_cols]
+    da_cols = (dy @ W2[f_cols].T) * _relu_grad(a_cols)
+    u_cols = ob._relu(a_cols)
+    return {"dhid": _dhid(dy[rows], da_rows, W1), "dW1": hid.T @ da_cols, "db1": da_cols.sum(axis=0),
+            "dW2": u_cols.T @ dy[:, h_cols], "db2": dy.sum(axis=0), "a_rows": a_rows, "a_cols": a_cols}
+
+
 def layer_backward(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, heads: int, causal: bool,
                    q_block: int | None = None, kv_block: int | None = None) -> dict:
     """Gradients of the layer output y with respect to x and every parameter,

@@ -88,3 +88,37 @@ def test_ffn_backward_does_not_depend_on_the_chunk():
     for k in ("dW1", "db1", "dW2", "db2"):
         d = (a[k] - b[k]).abs().max().item()
         assert d <= 1e-3 * a[k].abs().max().item(), k
+
+
+def test_ffn_backward_full_size_sampled():
+    # The 7B-class layer's FFN block (rows 32768, h 4096, ffn 16384: two 16384-row
+    # chunks, every product on SM pairs): rows of dhid, columns of dW1 and db1, a
+    # block of dW2 and all of db2 against the sampled oracle, which forms the
+    # pre-activations it needs in fp64 over every row; the first and last rows and
+    # columns, the chunk boundary and a few inside.
+    rows, h, f = 32768, 4096, 16384
+    shape = bi.LayerShape(1, rows, h, h // 128, 1, 1, False, "bf16", ffn=f)
+    inp = bi.make_inputs(shape, seed=2024)
+    hid64 = bi.to_f64(inp["x"].reshape(rows, h))
+    dy64 = bi.to_f64(bi.f32_to_bf16_bits(bi.normal_f64(2024, 40, rows * h).astype(np.float32)).reshape(rows, h))
+    W1, b1, W2 = (bi.to_torch(inp[k]) for k in ("W1", "b1", "W2"))
+    g = bpt.ffn_backward(torch.tensor(hid64, dtype=torch.float32, device="cuda"), W1, b1, W2,
+                         torch.tensor(dy64, dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    assert bpt.stream_status() == 0
+    W1_64, b1_64, W2_64 = bi.to_f64(inp["W1"]), bi.to_f64(inp["b1"]), bi.to_f64(inp["W2"])
+    rs = np.random.default_rng(5)
+    r_s = np.unique(np.concatenate([[0, 1, 16383, 16384, 32767], rs.integers(0, rows, 5)]))
+    f_s = np.unique(np.concatenate([[0, 255, 256, 16383], rs.integers(0, f, 3)]))
+    h_s = np.unique(np.concatenate([[0, 4095], rs.integers(0, h, 2)]))
+    ref = obb.ffn_backward_samples(hid64, W1_64, b1_64, W2_64, dy64, r_s, f_s, h_s)
+    # mask slack as in mask_slack(), over the sampled rows and columns
+    amb_rows = np.abs(ref["a_rows"]) < 1e-4
+    da_rows = np.abs(dy64[r_s] @ W2_64.T) * amb_rows
+    amb_cols = np.abs(ref["a_cols"]) < 1e-4
+    da_cols = np.abs(dy64 @ W2_64[f_s].T) * amb_cols
+    slack = {"dhid": da_rows @ np.abs(W1_64).T, "dW1": np.abs(hid64).T @ da_cols, "db1": da_cols.sum(axis=0)}
+    got = {"dhid": g["dhid"][r_s], "dW1": g["dW1"][:, f_s], "db1": g["db1"][f_s],
+           "dW2": g["dW2"][f_s][:, h_s], "db2": g["db2"]}
+    for k in ("dhid", "dW1", "db1", "dW2", "db2"):
+        check(got[k], ref[k], f"{k} (rows 32768, h 4096, ffn 16384, sampled)", slack.get(k, 0.0))

@@ -237,3 +237,20 @@ def test_sampled_gradient_rows_match_torch_autograd():
     np.testing.assert_allclose(gq, q.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(gk, k.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(gv, v.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
+
+
+def test_sampled_ffn_gradients_equal_the_whole_gradients():
+    # the row/column-sampled FFN gradients are the corresponding parts of ffn_backward's
+    rng = np.random.default_rng(11)
+    R, h, f = 37, 16, 24
+    hid, dy = rng.standard_normal((R, h)), rng.standard_normal((R, h))
+    W1, b1, W2 = rng.standard_normal((h, f)) / 4, rng.standard_normal(f) * 0.1, rng.standard_normal((f, h)) / 5
+    full = obb.ffn_backward(hid, W1, b1, W2, dy)
+    rows, fc, hc = [0, 5, 36], [1, 7, 23], [0, 15, 3]
+    got = obb.ffn_backward_samples(hid, W1, b1, W2, dy, rows, fc, hc)
+    np.testing.assert_allclose(got["dhid"], full["dhid"][rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["dW1"], full["dW1"][:, fc], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["db1"], full["db1"][fc], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["dW2"], full["dW2"][np.ix_(fc, hc)], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["db2"], full["db2"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["a_cols"], (hid @ W1 + b1)[:, fc], rtol=0, atol=1e-12)

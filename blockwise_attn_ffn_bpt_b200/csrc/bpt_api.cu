@@ -1713,10 +1713,13 @@ int bpt_convert_f32_to_bf16(const float* src, void* dst, long long n, void* stre
 }
 
 // The FFN block's backward over `rows` rows in chunks of R rows (workspace as
-// bpt_ffn_backward_workspace_bytes sizes it for R).
+// bpt_ffn_backward_workspace_bytes sizes it for R). hid_bf16, when given, is
+// hid already rounded to bf16 (every row, h apart), used instead of converting
+// each chunk; dhid_bf16, when given, receives dhid rounded to bf16 as well.
 int ffn_backward_impl(const float* hid, const void* W1, const void* b1, const void* W2, const float* dy,
                       long long rows, int h, int ffn, long long R, float* dhid, float* dW1, float* db1, float* dW2,
-                      float* db2, void* workspace, int sms, cudaStream_t st, int* status) {
+                      float* db2, void* workspace, int sms, cudaStream_t st, int* status,
+                      const __nv_bfloat16* hid_bf16 = nullptr, __nv_bfloat16* dhid_bf16 = nullptr) {
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(ws + align_up((size_t)R * h * 2, 1024));
@@ -1726,14 +1729,15 @@ int ffn_backward_impl(const float* hid, const void* W1, const void* b1, const vo
   for (long long r0 = 0; r0 < rows; r0 += R) {
     const long long n = std::min<long long>(R, rows - r0);
     const int acc = r0 > 0 ? 1 : 0;
-    BPT_TRY(launch_convert(hid + r0 * h, hb, n * h, sms, st));
+    const __nv_bfloat16* hbp = hid_bf16 != nullptr ? hid_bf16 + r0 * h : hb;
+    if (hid_bf16 == nullptr) BPT_TRY(launch_convert(hid + r0 * h, hb, n * h, sms, st));
     BPT_TRY(launch_convert(dy + r0 * h, dyb, n * h, sms, st));
     // the chunk's FFN intermediate again (rematerialised, not stored by the forward)
     GemmArgs a{};
     a.bias = b1;
     a.dst = U;
     a.ld_dst = ffn;
-    BPT_TRY((launch_gemm_t<EPI_FFN_UP, 0, 1>(hb, h, W1, ffn, n, ffn, h, a, sms, st, status, "bwd_ffn_up")));
+    BPT_TRY((launch_gemm_t<EPI_FFN_UP, 0, 1>(hbp, h, W1, ffn, n, ffn, h, a, sms, st, status, "bwd_ffn_up")));
     // da = (dy W2^T) [U > 0]
     a = GemmArgs{};
     a.mask_u = U;
@@ -1747,13 +1751,15 @@ int ffn_backward_impl(const float* hid, const void* W1, const void* b1, const vo
     a.ld_dy = h;
     a.out = dhid + r0 * h;
     a.ld_out = h;
+    a.dst = dhid_bf16 != nullptr ? dhid_bf16 + r0 * h : nullptr;
+    a.ld_dst = h;
     BPT_TRY((launch_gemm_t<EPI_BWD_DHID, 0, 0>(da, ffn, W1, ffn, n, h, ffn, a, sms, st, status, "bwd_dhid")));
     // dW1 (+)= hid^T da and dW2 (+)= U^T dy over the chunk's rows
     a = GemmArgs{};
     a.accumulate = acc;
     a.out = dW1;
     a.ld_out = ffn;
-    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(hb, h, da, ffn, h, ffn, n, a, sms, st, status, "bwd_dW1")));
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(hbp, h, da, ffn, h, ffn, n, a, sms, st, status, "bwd_dW1")));
     a.out = dW2;
     a.ld_out = h;
     BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(U, ffn, dyb, h, ffn, h, n, a, sms, st, status, "bwd_dW2")));
@@ -1978,11 +1984,11 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
     BPT_TRY(launch_gemm<EPI_OUTPROJ>(bf(L.o), rows, h, h, Wo, h, a, sms, st, status, "bwd_outproj"));
   }
   // FFN block: dhid, dW1, db1, dW2, db2
+  // (hid's bf16 copy is the out-projection's; dhid's bf16 copy comes from the dhid product's epilogue)
   BPT_TRY(ffn_backward_impl(f32(L.hid), W1, b1, W2, dy, rows, h, ffn, L.R, f32(L.dhid), dW1, db1, dW2, db2,
-                            ws + L.ffn, sms, st, status));
+                            ws + L.ffn, sms, st, status, bf(L.hb), bf(L.dhb)));
   // out-projection: dbo = sum dhid, dWo = O^T dhid, dO = dhid Wo^T
   BPT_TRY(launch_colsum(f32(L.dhid), rows, h, h, dbo, 0, st));
-  BPT_TRY(launch_convert(f32(L.dhid), bf(L.dhb), rows * h, sms, st));
   {
     GemmArgs a{};
     a.out = dWo;

@@ -177,6 +177,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int row, int co
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += dy[i];
     store32_f32(a.out + (long long)row * a.ld_out + col, v);
+    if (a.dst != nullptr) store32_bf16(a.dst + (long long)row * a.ld_dst + col, v);  // its bf16 copy, if asked
   } else {
     float* o = a.out + (long long)row * a.ld_out + col;
     if (a.accumulate) {

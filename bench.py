@@ -886,6 +886,24 @@ def layer_backward_arm(args):
         kernels[name] = {"launches": n_, "ms_per_step": ms_ / args.steps, "share": ms_ / split_total}
     att = kt.get("attention_bwd")
     att_tflops = fl["attention_bwd"] / (att[1] / args.steps / 1e3) / 1e12 if att else None
+    # the same backward from the forward's saved O and statistics (bpt_layer_forward_save once, untimed):
+    # no attention recomputation
+    _, o_sv, lse_sv = bpt.layer_forward_save(x, params, heads, shape.q_block, shape.kv_block, shape.causal,
+                                             stream=stream)
+    for _ in range(args.warmup):
+        bpt.layer_backward(x, params, dy, heads, shape.causal, stream=stream, saved=(o_sv, lse_sv))
+    torch.cuda.synchronize(device)
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs2:
+        e0.record(stream)
+        bpt.layer_backward(x, params, dy, heads, shape.causal, stream=stream, saved=(o_sv, lse_sv))
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    status = status or bpt.stream_status(stream)
+    ms_sv = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs2]))
+    total_sv = total - 4.0 * b * s * s * h * (0.5 if shape.causal else 1.0)
+    saved = {"ms_per_step": ms_sv, "tokens_per_s": b * s / (ms_sv / 1e3), "tflops": total_sv / (ms_sv / 1e3) / 1e12,
+             "api": "bpt_layer_forward_save, then bpt_layer_backward_saved (the attention is not recomputed)"}
     peaks, src = measured_peaks()
     line = {"metric": "BPT layer backward (bpt_layer_backward) tokens/s and TFLOP/s on 1 B200",
             "value": b * s / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "tflops": total / (ms / 1e3) / 1e12,
@@ -893,6 +911,7 @@ def layer_backward_arm(args):
             "peak_source": f"{src} bf16_tflops (burst)", "steps": args.steps, "warmup": args.warmup,
             "dtype": "bf16", "config": config_of(shape, args.workload),
             "flops_per_step": fl, "attention_bwd_tflops": att_tflops, "kernels": kernels,
+            "from_saved_forward": saved,
             "device_status": status, "clocks": clocks.summary(),
             "data": "synthetic (torch generator on the device)"}
     print(json.dumps(line))

@@ -31,7 +31,7 @@ EXPORTED = (
     "bpt_layer_forward_host", "bpt_convert_f32_to_bf16",
     "bpt_qkv_projection", "bpt_attention", "bpt_ffn_backward_workspace_bytes", "bpt_ffn_backward",
     "bpt_attention_lse", "bpt_attention_backward_workspace_bytes", "bpt_attention_backward",
-    "bpt_layer_backward_workspace_bytes", "bpt_layer_backward",
+    "bpt_layer_backward_workspace_bytes", "bpt_layer_backward", "bpt_layer_forward_save", "bpt_layer_backward_saved",
     "bpt_stream_status", "bpt_device_status", "bpt_wait_flag",
     "bpt_launch_count", "bpt_set_kernel_timing", "bpt_kernel_times",
 )
@@ -96,6 +96,10 @@ def lib() -> ctypes.CDLL:
     L.bpt_layer_backward_workspace_bytes.argtypes = [i] * 5
     L.bpt_layer_backward.restype = i
     L.bpt_layer_backward.argtypes = [vp] * 10 + [i] * 6 + [vp] * 10 + [sz, vp]
+    L.bpt_layer_forward_save.restype = i
+    L.bpt_layer_forward_save.argtypes = [vp] * 9 + [i] * 8 + [vp] * 4
+    L.bpt_layer_backward_saved.restype = i
+    L.bpt_layer_backward_saved.argtypes = [vp] * 12 + [i] * 6 + [vp] * 10 + [sz, vp]
     L.bpt_stream_status.restype = i
     L.bpt_stream_status.argtypes = [vp]
     L.bpt_device_status.restype = i
@@ -327,12 +331,35 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     return g
 
 
+def layer_forward_save(x: torch.Tensor, params: dict, heads: int, q_block: int, kv_block: int, causal: bool,
+                       stream: Optional[torch.cuda.Stream] = None):
+    """The layer forward that also keeps the attention output O and each row's
+    log-sum-exp for a later backward (bpt_layer_forward_save): bf16 x and
+    params as for layer_forward. Returns (out fp32 [b, s, h], o bf16 [b, s, h],
+    lse2 fp32 [b, heads, s]); pass (o, lse2) as layer_backward's `saved`."""
+    b, s, h = x.shape
+    ffn = int(params["W1"].shape[-1])
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bf16")
+    for k, shape in _param_shapes(h, ffn).items():
+        if params[k].dtype != torch.bfloat16 or tuple(params[k].shape) != shape:
+            raise ValueError(f"{k} must be bf16 of shape {shape}")
+    out = torch.empty((b, s, h), dtype=torch.float32, device=x.device)
+    o = torch.empty((b, s, h), dtype=torch.bfloat16, device=x.device)
+    lse2 = torch.empty((b, heads, s), dtype=torch.float32, device=x.device)
+    r = lib().bpt_layer_forward_save(_ptr(x), *[_ptr(params[k]) for k in PARAM_NAMES], b, s, h, heads, ffn, q_block,
+                                     kv_block, int(bool(causal)), _ptr(out), _ptr(o), _ptr(lse2), _stream(stream))
+    _check(r, "bpt_layer_forward_save")
+    return out, o, lse2
+
+
 def layer_backward(x: torch.Tensor, params: dict, dy: torch.Tensor, heads: int, causal: bool,
-                   stream: Optional[torch.cuda.Stream] = None) -> dict:
+                   stream: Optional[torch.cuda.Stream] = None, saved=None) -> dict:
     """Gradients of the layer's output (bpt_layer_backward) for dy = dL/dout
     (fp32 [b, s, h]): x bf16 [b, s, h] and params as for layer_forward (bf16,
     FFN width from W1). Returns {"dx", "dWqkv", "dbqkv", "dWo", "dbo", "dW1",
-    "db1", "dW2", "db2"} (fp32)."""
+    "db1", "dW2", "db2"} (fp32). saved = (o, lse2) from layer_forward_save skips
+    the attention's recomputation (bpt_layer_backward_saved)."""
     b, s, h = x.shape
     ffn = params["W1"].shape[-1]
     if x.dtype != torch.bfloat16 or dy.dtype != torch.float32 or dy.shape != x.shape:
@@ -350,12 +377,23 @@ def layer_backward(x: torch.Tensor, params: dict, dy: torch.Tensor, heads: int, 
     nbytes = int(lib().bpt_layer_backward_workspace_bytes(b, s, h, heads, ffn))
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     p = params
-    r = lib().bpt_layer_backward(_ptr(x), _ptr(p["Wqkv"]), _ptr(p["bqkv"]), _ptr(p["Wo"]), _ptr(p["bo"]),
-                                 _ptr(p["W1"]), _ptr(p["b1"]), _ptr(p["W2"]), _ptr(p["b2"]), _ptr(dy), b, s, h, heads,
-                                 ffn, int(bool(causal)), _ptr(g["dx"]), _ptr(g["dWqkv"]), _ptr(g["dbqkv"]),
-                                 _ptr(g["dWo"]), _ptr(g["dbo"]), _ptr(g["dW1"]), _ptr(g["db1"]), _ptr(g["dW2"]),
-                                 _ptr(g["db2"]), _ptr(ws), ws.numel(), _stream(stream))
-    _check(r, "bpt_layer_backward")
+    outs = [_ptr(g[k]) for k in ("dx", "dWqkv", "dbqkv", "dWo", "dbo", "dW1", "db1", "dW2", "db2")]
+    if saved is None:
+        r = lib().bpt_layer_backward(_ptr(x), _ptr(p["Wqkv"]), _ptr(p["bqkv"]), _ptr(p["Wo"]), _ptr(p["bo"]),
+                                     _ptr(p["W1"]), _ptr(p["b1"]), _ptr(p["W2"]), _ptr(p["b2"]), _ptr(dy), b, s, h,
+                                     heads, ffn, int(bool(causal)), *outs, _ptr(ws), ws.numel(), _stream(stream))
+        _check(r, "bpt_layer_backward")
+        return g
+    o, lse2 = saved
+    if o.dtype != torch.bfloat16 or tuple(o.shape) != (b, s, h):
+        raise ValueError("saved o must be bf16 [b, s, h]")
+    if lse2.dtype != torch.float32 or tuple(lse2.shape) != (b, heads, s):
+        raise ValueError("saved lse2 must be fp32 [b, heads, s]")
+    r = lib().bpt_layer_backward_saved(_ptr(x), _ptr(p["Wqkv"]), _ptr(p["bqkv"]), _ptr(p["Wo"]), _ptr(p["bo"]),
+                                       _ptr(p["W1"]), _ptr(p["b1"]), _ptr(p["W2"]), _ptr(p["b2"]), _ptr(o),
+                                       _ptr(lse2), _ptr(dy), b, s, h, heads, ffn, int(bool(causal)), *outs, _ptr(ws),
+                                       ws.numel(), _stream(stream))
+    _check(r, "bpt_layer_backward_saved")
     return g
 
 

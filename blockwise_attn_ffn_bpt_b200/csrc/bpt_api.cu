@@ -1225,7 +1225,7 @@ struct XChunks {
 
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
               int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr,
-              const XChunks* xc = nullptr) {
+              const XChunks* xc = nullptr, __nv_bfloat16* o_save = nullptr, float* lse2_save = nullptr) {
   int* status = nullptr;
   BPT_TRY(stream_status_word(st, &status));
   const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
@@ -1296,12 +1296,17 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   // steps 4-10 for every query block at once: each CTA overwrites the Q of its
   // own rows and head with their attention output (or, in the one-launch
   // schedule, attention and the whole FFN side together)
-  if (L.mega && mega_available())
+  // (With o_save, for a later backward: O goes to o_save, h apart, and each row's
+  // log-sum-exp to lse2_save; the FFN side then reads O from there.)
+  if (L.mega && mega_available() && o_save == nullptr)
     return launch_mega(QO, ldq, K, V, p, b, s, h, heads, ffn, causal, L, ws, out, sms, st, status);
-  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, QO, ldq, st, status));
+  const __nv_bfloat16* O = o_save != nullptr ? o_save : QO;
+  const long long ldo = o_save != nullptr ? (long long)h : ldq;
+  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, const_cast<__nv_bfloat16*>(O), ldo, st,
+                           status, lse2_save));
 
   // step 11 for every query block: out-projection, residuals and FFN
-  if (L.chain) return launch_chain(QO, ldq, p, tok, h, ffn, L, ws, out, sms, st, status);
+  if (L.chain) return launch_chain(O, ldo, p, tok, h, ffn, L, ws, out, sms, st, status);
   return for_each_wave(b, s, h, ffn, q_block, wave_rows, [&](const Wave& w) -> int {
     const long long rows = w.rows();
     GemmArgs a{};
@@ -1318,7 +1323,7 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     a.dst = HB;
     a.ld_dst = h;
     const int sp = f32 ? 1 : 0, kf = f32 ? 2 : 1;  // fp32 inputs: A against [W_hi; W_lo]
-    BPT_TRY(launch_gemm_split<EPI_OUTPROJ>(QO + w.row0 * ldq, rows, h, ldq, wo, (long long)kf * h, h, sp,
+    BPT_TRY(launch_gemm_split<EPI_OUTPROJ>(O + w.row0 * ldo, rows, h, ldo, wo, (long long)kf * h, h, sp,
                                            h / GEMM_BK, a, sms, st, status, "gemm_outproj"));
     a.bias = p.b1;
     a.dst = U;
@@ -1334,7 +1339,7 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
 
 int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int kv_block,
                 int causal, int wave_rows, void* workspace, size_t ws_bytes, bool caller_ws, float* out,
-                void* stream) {
+                void* stream, __nv_bfloat16* o_save = nullptr, float* lse2_save = nullptr) {
   BPT_TRY(validate_layer(dtype, p, b, s, h, heads, ffn, q_block, kv_block, out));
   if ((long long)b * s == 0) return BPT_OK;
   const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
@@ -1366,7 +1371,9 @@ int layer_entry(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, i
     }
     ws = reinterpret_cast<uint8_t*>(m);
   }
-  const int r = run_layer(dtype, p, b, s, h, heads, ffn, q_block, causal, wave_rows, ws, out, st, sms);
+  const int r =
+      run_layer(dtype, p, b, s, h, heads, ffn, q_block, causal, wave_rows, ws, out, st, sms, nullptr, nullptr, o_save,
+                lse2_save);
   if (!caller_ws) cudaFreeAsync(ws, st);
   return r;
 }
@@ -1675,6 +1682,28 @@ int bpt_layer_forward_ffn(int dtype, const void* x, const void* Wqkv, const void
                      caller_ws, out, stream);
 }
 
+int bpt_layer_forward_save(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                           const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                           int heads, int ffn, int q_block, int kv_block, int causal, float* out, void* o_save,
+                           float* lse2_save, void* stream) {
+  const LayerPtrs p{x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2};
+  BPT_TRY(validate_layer(BPT_DTYPE_BF16, p, b, s, h, heads, ffn, q_block, kv_block, out));
+  if ((long long)b * s == 0) return BPT_OK;
+  if (!o_save || !lse2_save) return BPT_ERR_NULL;
+  if (!aligned16(o_save) || !aligned16(lse2_save)) return BPT_ERR_ALIGN;
+  const size_t rows = (size_t)b * s;
+  const Range ro = rng(o_save, rows * h * 2), rl = rng(lse2_save, (size_t)b * heads * s * 4);
+  const Range others[10] = {rng(out, rows * h * 4), rng(x, rows * h * 2), rng(Wqkv, (size_t)3 * h * h * 2),
+                            rng(bqkv, (size_t)3 * h * 2), rng(Wo, (size_t)h * h * 2), rng(bo, (size_t)h * 2),
+                            rng(W1, (size_t)h * ffn * 2), rng(b1, (size_t)ffn * 2), rng(W2, (size_t)ffn * h * 2),
+                            rng(b2, (size_t)h * 2)};
+  if (overlap(ro, rl)) return BPT_ERR_ALIAS;
+  for (const Range& r : others)
+    if (overlap(ro, r) || overlap(rl, r)) return BPT_ERR_ALIAS;
+  return layer_entry(BPT_DTYPE_BF16, p, b, s, h, heads, ffn, q_block, kv_block, causal, BPT_WAVE_DEFAULT_WAVES,
+                     nullptr, 0, false, out, stream, reinterpret_cast<__nv_bfloat16*>(o_save), lse2_save);
+}
+
 int bpt_layer_forward_noalloc(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
                               const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
                               int heads, int q_block, int kv_block, int causal, float* out, void* stream) {
@@ -1917,11 +1946,14 @@ size_t bpt_layer_backward_workspace_bytes(int b, int s, int h, int heads, int ff
   return layer_bwd_layout(b, s, h, heads, ffn).total;
 }
 
-int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
-                       const void* W1, const void* b1, const void* W2, const void* b2, const float* dy, int b, int s,
-                       int h, int heads, int ffn, int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo,
-                       float* dbo, float* dW1, float* db1, float* dW2, float* db2, void* workspace,
-                       size_t ws_bytes, void* stream) {
+// The layer backward; with o_saved and lse2_saved (the forward's O and per-row
+// log-sum-exp, bpt_layer_forward_save) the attention is not recomputed.
+static int layer_backward_impl(const void* x, const void* Wqkv, const void* bqkv, const void* Wo,
+                               const void* bo, const void* W1, const void* b1, const void* W2, const void* b2,
+                               const float* dy, int b, int s, int h, int heads, int ffn, int causal, float* dx,
+                               float* dWqkv, float* dbqkv, float* dWo, float* dbo, float* dW1, float* db1, float* dW2,
+                               float* db2, void* workspace, size_t ws_bytes, void* stream, const void* o_saved,
+                               const float* lse2_saved) {
   BPT_TRY(check_shape(b, s, h, heads));
   if (ffn <= 0 || ffn % 64 || (long long)h * ffn > 0x7fffffffLL) return BPT_ERR_SHAPE;
   if ((long long)b * s == 0) return BPT_OK;
@@ -1934,10 +1966,16 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
   const LayerBwdLayout L = layer_bwd_layout(b, s, h, heads, ffn);
   if (ws_bytes < L.total) return BPT_ERR_NOMEM;
   const long long rows = (long long)b * s;
-  const Range in[10] = {rng(x, (size_t)rows * h * 2),     rng(Wqkv, (size_t)h * 3 * h * 2), rng(bqkv, (size_t)3 * h * 2),
+  const bool saved = o_saved != nullptr;
+  if (saved != (lse2_saved != nullptr)) return BPT_ERR_NULL;
+  if (saved && (!aligned16(o_saved) || !aligned16(lse2_saved))) return BPT_ERR_ALIGN;
+  // (without saved inputs the two extra ranges are empty)
+  const Range in[12] = {rng(x, (size_t)rows * h * 2),     rng(Wqkv, (size_t)h * 3 * h * 2), rng(bqkv, (size_t)3 * h * 2),
                         rng(Wo, (size_t)h * h * 2),       rng(bo, (size_t)h * 2),           rng(W1, (size_t)h * ffn * 2),
                         rng(b1, (size_t)ffn * 2),         rng(W2, (size_t)ffn * h * 2),     rng(b2, (size_t)h * 2),
-                        rng(dy, (size_t)rows * h * 4)};
+                        rng(dy, (size_t)rows * h * 4),
+                        rng(o_saved, saved ? (size_t)rows * h * 2 : 0),
+                        rng(lse2_saved, saved ? (size_t)b * heads * s * 4 : 0)};
   const Range outs[10] = {rng(dx, (size_t)rows * h * 4), rng(dWqkv, (size_t)h * 3 * h * 4), rng(dbqkv, (size_t)3 * h * 4),
                           rng(dWo, (size_t)h * h * 4),   rng(dbo, (size_t)h * 4),           rng(dW1, (size_t)h * ffn * 4),
                           rng(db1, (size_t)ffn * 4),     rng(dW2, (size_t)ffn * h * 4),     rng(db2, (size_t)h * 4),
@@ -1958,7 +1996,10 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
   const int dh = h / heads;
 
-  // the forward again (rematerialised): Q, K, V; O and each row's log-sum-exp; hid
+  // the forward again (rematerialised): Q, K, V; O and each row's log-sum-exp (or the
+  // forward's own, saved); hid
+  const __nv_bfloat16* Osrc = saved ? reinterpret_cast<const __nv_bfloat16*>(o_saved) : bf(L.o);
+  const float* lse = saved ? lse2_saved : f32(L.lse);
   {
     GemmArgs a{};
     a.bias = bqkv;
@@ -1970,8 +2011,9 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
     a.h = h;
     BPT_TRY(launch_gemm<EPI_QKV>(x, rows, h, h, Wqkv, 3LL * h, a, sms, st, status, "bwd_qkv"));
   }
-  BPT_TRY(launch_attention(bf(L.q), h, bf(L.k), bf(L.v), b, s, h, heads, causal, 0, b, 0, s, bf(L.o), h, st, status,
-                           f32(L.lse)));
+  if (!saved)
+    BPT_TRY(launch_attention(bf(L.q), h, bf(L.k), bf(L.v), b, s, h, heads, causal, 0, b, 0, s, bf(L.o), h, st,
+                             status, f32(L.lse)));
   {
     GemmArgs a{};
     a.resid = x;
@@ -1981,7 +2023,7 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
     a.bias = bo;
     a.dst = bf(L.hb);
     a.ld_dst = h;
-    BPT_TRY(launch_gemm<EPI_OUTPROJ>(bf(L.o), rows, h, h, Wo, h, a, sms, st, status, "bwd_outproj"));
+    BPT_TRY(launch_gemm<EPI_OUTPROJ>(Osrc, rows, h, h, Wo, h, a, sms, st, status, "bwd_outproj"));
   }
   // FFN block: dhid, dW1, db1, dW2, db2
   // (hid's bf16 copy is the out-projection's; dhid's bf16 copy comes from the dhid product's epilogue)
@@ -1993,7 +2035,7 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
     GemmArgs a{};
     a.out = dWo;
     a.ld_out = h;
-    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(bf(L.o), h, bf(L.dhb), h, h, h, rows, a, sms, st, status, "bwd_dWo")));
+    BPT_TRY((launch_gemm_t<EPI_GRAD, 1, 1>(Osrc, h, bf(L.dhb), h, h, h, rows, a, sms, st, status, "bwd_dWo")));
     a = GemmArgs{};
     a.dst = bf(L.dO);
     a.ld_dst = h;
@@ -2003,8 +2045,8 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
   float* dq32 = f32(L.dq32);
   __nv_bfloat16* dqkv = bf(L.dqkv);
   if (cudaMemsetAsync(dq32, 0, (size_t)rows * h * 4, st) != cudaSuccess) return BPT_ERR_CUDA;
-  BPT_TRY(launch_dsum(bf(L.o), bf(L.dO), h, rows, s, heads, dh, f32(L.dsum), st));
-  BPT_TRY(launch_attention_bwd(bf(L.q), bf(L.k), bf(L.v), h, bf(L.dO), h, f32(L.lse), f32(L.dsum), dq32, dqkv + h,
+  BPT_TRY(launch_dsum(Osrc, bf(L.dO), h, rows, s, heads, dh, f32(L.dsum), st));
+  BPT_TRY(launch_attention_bwd(bf(L.q), bf(L.k), bf(L.v), h, bf(L.dO), h, lse, f32(L.dsum), dq32, dqkv + h,
                                dqkv + 2 * h, 3LL * h, b, s, h, heads, causal, st, status));
   BPT_TRY(launch_rows_to_bf16(dq32, rows, h, dqkv, 3LL * h, sms, st));
   // projection: dbqkv = sum dqkv, dWqkv = x^T dqkv, dx = dhid + dqkv Wqkv^T
@@ -2023,6 +2065,25 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
                                                "bwd_dx")));
   }
   return BPT_OK;
+}
+
+int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                       const void* W1, const void* b1, const void* W2, const void* b2, const float* dy, int b, int s,
+                       int h, int heads, int ffn, int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo,
+                       float* dbo, float* dW1, float* db1, float* dW2, float* db2, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  return layer_backward_impl(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, b, s, h, heads, ffn, causal, dx, dWqkv, dbqkv,
+                             dWo, dbo, dW1, db1, dW2, db2, workspace, ws_bytes, stream, nullptr, nullptr);
+}
+
+int bpt_layer_backward_saved(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                             const void* W1, const void* b1, const void* W2, const void* b2, const void* o_saved,
+                             const float* lse2_saved, const float* dy, int b, int s, int h, int heads, int ffn,
+                             int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo, float* dbo, float* dW1,
+                             float* db1, float* dW2, float* db2, void* workspace, size_t ws_bytes, void* stream) {
+  if ((long long)b * s > 0 && (!o_saved || !lse2_saved)) return BPT_ERR_NULL;
+  return layer_backward_impl(x, Wqkv, bqkv, Wo, bo, W1, b1, W2, b2, dy, b, s, h, heads, ffn, causal, dx, dWqkv, dbqkv,
+                             dWo, dbo, dW1, db1, dW2, db2, workspace, ws_bytes, stream, o_saved, lse2_saved);
 }
 
 int bpt_qkv_projection(const void* x, const void* Wqkv, const void* bqkv, int b, int s, int h, void* q, void* k,

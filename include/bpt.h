@@ -395,6 +395,40 @@ int bpt_layer_backward(const void* x, const void* Wqkv, const void* bqkv, const 
                        float* dbo, float* dW1, float* db1, float* dW2, float* db2, void* workspace,
                        size_t ws_bytes, void* stream);
 
+/* The forward for a later backward: bpt_layer_forward_ffn (bf16 inputs, FFN
+ * width ffn, one launch per GEMM and FFN wave, workspace from the library's
+ * pool) that also keeps what the backward would otherwise recompute with a
+ * second attention pass -- the attention output O and, per row and head, the
+ * normalisation statistic that Algorithm 1 of the paper review records for
+ * each query block (the running max m and sum l, kept as m + log2 l in log2
+ * units, as bpt_attention_lse writes it). The pages rematerialise the
+ * blockwise FFN for training; attention's P is never stored either way, and O
+ * is the layer's own activation (the out-projection's input).
+ * o_save: bf16 [b, s, h] (head k in columns k*dh ..), lse2_save: fp32
+ * [b][heads][s]; both caller-owned device memory, written entirely. out as for
+ * bpt_layer_forward_ffn (the same values). Errors as for bpt_layer_forward_ffn,
+ * plus BPT_ERR_NULL / BPT_ERR_ALIGN (16 bytes) for o_save and lse2_save and
+ * BPT_ERR_ALIAS where they overlap each other, out or an input. */
+int bpt_layer_forward_save(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                           const void* W1, const void* b1, const void* W2, const void* b2, int b, int s, int h,
+                           int heads, int ffn, int q_block, int kv_block, int causal, float* out, void* o_save,
+                           float* lse2_save, void* stream);
+
+/* bpt_layer_backward from the forward's saved O and statistics
+ * (bpt_layer_forward_save) instead of recomputing the attention: the
+ * projection and the out-projection are still recomputed, and the FFN
+ * intermediate chunk by chunk. The same arguments, workspace and results as
+ * bpt_layer_backward (equal bit for bit when o_saved and lse2_saved come from
+ * bpt_layer_forward_save on the same x and weights), plus o_saved bf16 [b, s, h]
+ * and lse2_saved fp32 [b][heads][s], read only. Errors as for
+ * bpt_layer_backward, plus BPT_ERR_NULL / BPT_ERR_ALIGN for the saved inputs and
+ * BPT_ERR_ALIAS where an output or the workspace overlaps them. */
+int bpt_layer_backward_saved(const void* x, const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                             const void* W1, const void* b1, const void* W2, const void* b2, const void* o_saved,
+                             const float* lse2_saved, const float* dy, int b, int s, int h, int heads, int ffn,
+                             int causal, float* dx, float* dWqkv, float* dbqkv, float* dWo, float* dbo, float* dW1,
+                             float* db1, float* dW2, float* db2, void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Status and measurement.
  * ------------------------------------------------------------------------ */

@@ -417,3 +417,33 @@ def test_backward_entries_validate_and_size_their_workspaces():
     assert L.bpt_layer_backward(*q[:10], b, s, h, heads, f, 1, *q[10:19], q[19], need - 1, None) == NOMEM
     assert L.bpt_layer_backward(*q[:9], None, b, s, h, heads, f, 1, *q[10:19], q[19], need, None) == NULL
     assert L.bpt_layer_backward(*q[:10], b, s, h, heads, f, 1, q[0], *q[11:19], q[19], need, None) == ALIAS
+
+
+def test_saved_forward_and_backward_entries_validate_before_touching_memory():
+    L = bpt.lib()
+    b, s, h, heads, f = 2, 256, 256, 2, 512
+    rows = b * s
+    # forward with saved O and statistics: the layer's own checks, then the two extra buffers
+    p = fake_ptrs(13)  # x, 8 weights, out, o_save, lse2_save, (spare)
+    w = p[1:9]
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, 192, 2, f, 64, 64, 1, p[9], p[10], p[11], None) == SHAPE
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], None, p[11], None) == NULL
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], p[10], None, None) == NULL
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], p[10] + 8, p[11], None) == ALIGN
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], p[9], p[11], None) == ALIAS
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], p[10], p[10], None) == ALIAS
+    assert L.bpt_layer_forward_save(p[0], *w, b, s, h, heads, f, 64, 64, 1, p[9], p[10], p[0], None) == ALIAS
+    assert L.bpt_layer_forward_save(p[0], *w, 0, s, h, heads, f, 64, 64, 1, p[9], None, None, None) == OK
+    # backward from the saved inputs: the layer backward's checks plus the saved pair
+    need = L.bpt_layer_backward_workspace_bytes(b, s, h, heads, f)
+    q = fake_ptrs(22)  # x, 8 weights, o_saved, lse2_saved, dy, 9 gradients, workspace
+    x, ws_, o, lse, dy, outs, ws = q[0], q[1:9], q[9], q[10], q[11], q[12:21], q[21]
+    assert L.bpt_layer_backward_saved(x, *ws_, o, lse, dy, b, s, h, heads, f, 1, *outs, ws, need, None) != NULL
+    assert L.bpt_layer_backward_saved(x, *ws_, None, lse, dy, b, s, h, heads, f, 1, *outs, ws, need, None) == NULL
+    assert L.bpt_layer_backward_saved(x, *ws_, o, None, dy, b, s, h, heads, f, 1, *outs, ws, need, None) == NULL
+    assert L.bpt_layer_backward_saved(x, *ws_, o + 8, lse, dy, b, s, h, heads, f, 1, *outs, ws, need, None) == ALIGN
+    assert L.bpt_layer_backward_saved(x, *ws_, o, lse, dy, b, s, h, heads, f, 1, o, *outs[1:], ws, need,
+                                      None) == ALIAS  # dx over the saved O
+    assert L.bpt_layer_backward_saved(x, *ws_, o, lse, dy, b, s, h, heads, f, 1, *outs, lse, need,
+                                      None) == ALIAS  # the workspace over the saved statistics
+    assert L.bpt_layer_backward_saved(x, *ws_, o, lse, dy, b, s, h, heads, f, 1, *outs, ws, need - 1, None) == NOMEM

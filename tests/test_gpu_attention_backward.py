@@ -171,3 +171,25 @@ def test_attention_backward_full_size_sampled_rows():
     for name, got, ref in (("dq", g["dq"][0, qr, c], dQ), ("dk", g["dk"][0, kr, c], dK), ("dv", g["dv"][0, kr, c], dV)):
         rl2, mx = rel_errors(got, ref)
         assert rl2 <= 1.5e-2 and mx <= 4e-2, f"{name} (s {s}, head {head}): rel-L2 {rl2:.3e}, max {mx:.3e}"
+
+
+@pytest.mark.parametrize("b,s,h,heads,f,causal", LAYER_CASES + [(1, 1024, 256, 2, 1024, True)])
+def test_layer_backward_from_saved_inputs_equals_the_rematerialising_backward(b, s, h, heads, f, causal):
+    # the forward that keeps O and each row's log-sum-exp gives the same output
+    # as the plain forward; the backward from them gives the same gradients, bit
+    # for bit, as the backward that recomputes the attention (same kernels, same
+    # operands)
+    shape = bi.LayerShape(b, s, h, heads, s, s, causal, "bf16", ffn=f)
+    inp = bi.make_inputs(shape, seed=s + h + 1)
+    params = {k: bi.to_torch(inp[k]) for k in ("Wqkv", "bqkv", "Wo", "bo", "W1", "b1", "W2", "b2")}
+    x = bi.to_torch(inp["x"])
+    dy = torch.tensor(bi.to_f64(bf16_normal(s + h + 1, 41, (b, s, h))), dtype=torch.float32, device="cuda")
+    out_s, o, lse2 = bpt.layer_forward_save(x, params, heads, s, s, causal)
+    out = bpt.layer_forward(x, params, heads, s, s, causal)
+    g_re = bpt.layer_backward(x, params, dy, heads, causal)
+    g_sv = bpt.layer_backward(x, params, dy, heads, causal, saved=(o, lse2))
+    torch.cuda.synchronize()
+    assert bpt.stream_status() == 0
+    assert torch.equal(out_s, out)
+    for k in g_re:
+        assert torch.equal(g_sv[k], g_re[k]), k

@@ -556,7 +556,10 @@ bool use_chain(int dtype, int wave_rows) {
          (wave_rows == BPT_WAVE_DEFAULT && kChainByDefault);
 }
 
-Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave_rows) {
+// With ffn_after_kv (per-GEMM waves only), the wave scratch follows the K/V
+// copies instead of aliasing them, so that a wave's FFN side can run while
+// later rows still need K and V.
+Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave_rows, bool ffn_after_kv = false) {
   Layout L{};
   const size_t tok = (size_t)b * s;
   L.k = 0;
@@ -579,11 +582,12 @@ Layout layout_for(int dtype, int b, int s, int h, int ffn, int q_block, int wave
     off = align_up(off + (3 * (size_t)L.cp.groups + (L.mega ? (size_t)L.cp.groups + 1 : 0)) * sizeof(unsigned), 1024);
   } else {
     const int wr = wave_rows_for(b, s, h, ffn, q_block, wave_rows);
+    const size_t base = ffn_after_kv ? align_up(kv_bytes(b, s, h), 1024) : 0;
     L.wave_rows = wr;
-    L.hid = 0;
-    L.hb = align_up((size_t)wr * h * 4, 1024);
+    L.hid = base;
+    L.hb = base + align_up((size_t)wr * h * 4, 1024);
     L.u = L.hb + align_up((size_t)wr * h * 2, 1024);
-    off = std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h, ffn));
+    off = ffn_after_kv ? base + wave_scratch_bytes(wr, h, ffn) : std::max(kv_bytes(b, s, h), wave_scratch_bytes(wr, h, ffn));
   }
   auto take = [&](size_t bytes) {
     size_t at = off;
@@ -1208,10 +1212,13 @@ int validate_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads
 }
 
 // Called after the launches that finish rows [row0, row0 + rows) of out (each
-// FFN wave's FFN-down), so that a caller can start copying them out.
+// FFN wave's FFN-down), so that a caller can start copying them out. With
+// split_last, the last wave runs as two halves, each followed by the call, so
+// that only the second half's copy waits for the last launch.
 struct WaveHook {
   int (*fn)(void* ctx, long long row0, long long rows) = nullptr;
   void* ctx = nullptr;
+  bool split_last = false;
 };
 
 // x arriving in row chunks (bf16 inputs): chunk c, rows [c rows, (c + 1) rows),
@@ -1223,12 +1230,24 @@ struct XChunks {
   const cudaEvent_t* ev = nullptr;
 };
 
+// Whether a layer can run wave by wave (attention of a wave's rows, then its
+// FFN side): causal attention (a row needs only the keys at or before it)
+// and the per-GEMM wave schedule.
+bool interleavable(int dtype, int causal, int wave_rows) { return causal && !use_chain(dtype, wave_rows); }
+
+// interleave (callers that size the workspace with layout_for(...,
+// interleavable(dtype, causal, wave_rows))): attention runs wave by wave, each
+// wave's rows just before that wave's FFN side, and the first input's row
+// chunks (xc) are projected as the waves need them, so that results start to
+// come out early in the layer rather than after all of attention.
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
               int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr,
-              const XChunks* xc = nullptr, __nv_bfloat16* o_save = nullptr, float* lse2_save = nullptr) {
+              const XChunks* xc = nullptr, __nv_bfloat16* o_save = nullptr, float* lse2_save = nullptr,
+              bool interleave_req = false) {
   int* status = nullptr;
   BPT_TRY(stream_status_word(st, &status));
-  const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows);
+  const bool interleave = interleave_req && interleavable(dtype, causal, wave_rows) && o_save == nullptr;
+  const Layout L = layout_for(dtype, b, s, h, ffn, q_block, wave_rows, interleave);
   const long long tok = (long long)b * s;
   __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(ws + L.k);
   __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(ws + L.v);
@@ -1242,6 +1261,28 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
 
   const void *xa = p.x, *wqkv = p.Wqkv, *wo = p.Wo, *w1 = p.W1, *w2 = p.W2;
   const int f32 = dtype == BPT_DTYPE_F32 ? 1 : 0;
+  const bool mega = L.mega && mega_available() && o_save == nullptr;
+  const __nv_bfloat16* O = o_save != nullptr ? o_save : QO;
+  const long long ldo = o_save != nullptr ? (long long)h : ldq;
+  // Attention of the flat rows [r0, r0 + m), split at sequence boundaries into
+  // launches over whole sequences or one sequence's run of rows. Every row's
+  // arithmetic is the same as in one launch over all rows.
+  auto attend_rows = [&](long long r0, long long m) -> int {
+    for (long long r = r0, end = r0 + m; r < end;) {
+      const int beta = (int)(r / s), t = (int)(r - (long long)beta * s);
+      const bool whole = t == 0 && end - r >= s;
+      const int nb = whole ? (int)std::min<long long>((end - r) / s, b - beta) : 1;
+      const int tl = whole ? s : (int)std::min<long long>(s - t, end - r);
+      BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, beta, nb, t, tl,
+                               const_cast<__nv_bfloat16*>(O) + r * ldo, ldo, st, status));
+      r += (long long)nb * tl;
+    }
+    return BPT_OK;
+  };
+  // the first input's row chunks, projected in order up to a given row
+  const bool chunked = !f32 && xc != nullptr && xc->n > 0;
+  int next_chunk = 0;
+  long long projected = 0;
   if (f32) {
     // fp32 inputs: split bf16 products, so that neither x nor the weights
     // lose more than about 16 significant bits (x W = x_hi W_hi + x_hi W_lo +
@@ -1263,31 +1304,40 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   }
 
   // step 1: projection of the whole sequence
+  GemmArgs qa{};
+  qa.bias = p.bqkv;
+  qa.bias_f32 = f32;
+  qa.q = QO;
+  qa.ldq = ldq;
+  qa.k = K;
+  qa.v = V;
+  qa.ldkv = h;
+  qa.h = h;
+  auto project_to = [&](long long end) -> int {
+    for (; next_chunk < xc->n && projected < end; ++next_chunk) {
+      const long long r0 = (long long)next_chunk * xc->rows, m = std::min(xc->rows, tok - r0);
+      if (m <= 0) {
+        projected = tok;
+        break;
+      }
+      if (cudaStreamWaitEvent(st, xc->ev[next_chunk], 0) != cudaSuccess) return BPT_ERR_CUDA;
+      GemmArgs ac = qa;
+      ac.q = QO + r0 * ldq;
+      ac.k = K + r0 * h;
+      ac.v = V + r0 * h;
+      BPT_TRY(launch_gemm<EPI_QKV>(reinterpret_cast<const __nv_bfloat16*>(xa) + r0 * h, m, h, h, wqkv, 3LL * h, ac,
+                                   sms, st, status, "gemm_qkv"));
+      projected = r0 + m;
+    }
+    return BPT_OK;
+  };
   {
-    GemmArgs a{};
-    a.bias = p.bqkv;
-    a.bias_f32 = f32;
-    a.q = QO;
-    a.ldq = ldq;
-    a.k = K;
-    a.v = V;
-    a.ldkv = h;
-    a.h = h;
+    const GemmArgs& a = qa;
     if (f32) {
       BPT_TRY(launch_gemm_split<EPI_QKV>(xa, tok, 2LL * h, 2LL * h, wqkv, 3LL * h, 3LL * h, 2, h / GEMM_BK, a, sms,
                                          st, status, "gemm_qkv"));
-    } else if (xc != nullptr && xc->n > 0) {
-      for (int c = 0; c < xc->n; ++c) {
-        const long long r0 = (long long)c * xc->rows, m = std::min(xc->rows, tok - r0);
-        if (m <= 0) break;
-        if (cudaStreamWaitEvent(st, xc->ev[c], 0) != cudaSuccess) return BPT_ERR_CUDA;
-        GemmArgs ac = a;
-        ac.q = QO + r0 * ldq;
-        ac.k = K + r0 * h;
-        ac.v = V + r0 * h;
-        BPT_TRY(launch_gemm<EPI_QKV>(reinterpret_cast<const __nv_bfloat16*>(xa) + r0 * h, m, h, h, wqkv, 3LL * h, ac,
-                                     sms, st, status, "gemm_qkv"));
-      }
+    } else if (chunked) {
+      if (!interleave) BPT_TRY(project_to(tok));
     } else {
       BPT_TRY(launch_gemm<EPI_QKV>(xa, tok, h, h, wqkv, 3LL * h, a, sms, st, status, "gemm_qkv"));
     }
@@ -1298,16 +1348,14 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   // schedule, attention and the whole FFN side together)
   // (With o_save, for a later backward: O goes to o_save, h apart, and each row's
   // log-sum-exp to lse2_save; the FFN side then reads O from there.)
-  if (L.mega && mega_available() && o_save == nullptr)
-    return launch_mega(QO, ldq, K, V, p, b, s, h, heads, ffn, causal, L, ws, out, sms, st, status);
-  const __nv_bfloat16* O = o_save != nullptr ? o_save : QO;
-  const long long ldo = o_save != nullptr ? (long long)h : ldq;
-  BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, const_cast<__nv_bfloat16*>(O), ldo, st,
-                           status, lse2_save));
+  if (mega) return launch_mega(QO, ldq, K, V, p, b, s, h, heads, ffn, causal, L, ws, out, sms, st, status);
+  if (!interleave)
+    BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, 0, b, 0, s, const_cast<__nv_bfloat16*>(O), ldo,
+                             st, status, lse2_save));
 
   // step 11 for every query block: out-projection, residuals and FFN
   if (L.chain) return launch_chain(O, ldo, p, tok, h, ffn, L, ws, out, sms, st, status);
-  return for_each_wave(b, s, h, ffn, q_block, wave_rows, [&](const Wave& w) -> int {
+  auto ffn_side = [&](const Wave& w) -> int {
     const long long rows = w.rows();
     GemmArgs a{};
     a.resid = p.x;
@@ -1334,6 +1382,22 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
     BPT_TRY(launch_gemm_split<EPI_FFN_DOWN>(U, rows, ffn, ffn, w2, (long long)kf * ffn, h, sp, ffn / GEMM_BK, a, sms,
                                             st, status, "gemm_ffn_down"));
     return hook ? hook->fn(hook->ctx, w.row0, rows) : BPT_OK;
+  };
+  return for_each_wave(b, s, h, ffn, q_block, wave_rows, [&](const Wave& w) -> int {
+    // The last wave as two halves (hook->split_last): the first half's rows are
+    // copied out while the second half computes. Each row's arithmetic is the
+    // same either way.
+    const long long rows = w.rows();
+    if (interleave) {
+      if (chunked) BPT_TRY(project_to(w.row0 + rows));
+      BPT_TRY(attend_rows(w.row0, rows));
+    }
+    if (hook != nullptr && hook->split_last && w.n_seq == 1 && w.row0 + rows == tok && rows >= 2 * GEMM_BM) {
+      const int half = (int)((rows / 2 + GEMM_BM - 1) / GEMM_BM * GEMM_BM);
+      BPT_TRY(ffn_side(Wave{w.row0, w.beta0, 1, w.t_start, half}));
+      return ffn_side(Wave{w.row0 + half, w.beta0, 1, w.t_start + half, w.t_len - half});
+    }
+    return ffn_side(w);
   });
 }
 
@@ -1511,7 +1575,11 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
   if (overlap(xr, orr)) return BPT_ERR_ALIAS;
   int sms = 0;
   BPT_TRY(check_device(&sms));
-  const Layout L = layout_for(dtype, b, s, h, 4 * h, q_block, 0);
+  // causal: attention and the FFN side wave by wave for the first and last
+  // input (run_layer's interleave), with one wave's FFN scratch beside the K/V
+  // copies (the inputs between them use the same workspace with the scratch
+  // over K/V)
+  const Layout L = layout_for(dtype, b, s, h, 4 * h, q_block, 0, interleavable(dtype, causal, 0));
   const size_t xa = align_up(xb, 1024), oa = align_up(ob, 1024);
   const size_t total = 2 * xa + 2 * oa + L.total;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1580,9 +1648,14 @@ int host_entry(int dtype, const void* x_host, long long x_stride, const LayerPtr
       // each FFN wave's rows of the result are copied out as soon as they are final
       // (split over the copy streams), overlapping the waves still to run
       WaveCopy wc{&pp, st, reinterpret_cast<const uint8_t*>(odev[k]), oi, (size_t)h * 4, 0};
-      const WaveHook hook{&WaveCopy::on_wave, &wc};
+      // the last input's last wave in halves: its copy out is the call's tail
+      const WaveHook hook{&WaveCopy::on_wave, &wc, i == n - 1};
+      // wave by wave only where it shortens the call: the first input (whose
+      // copy in is not hidden) and the last (whose copy out is the call's tail);
+      // between them one attention launch per input leaves fewer launch tails,
+      // and the copies are hidden by the neighbouring inputs' compute
       r = run_layer(dtype, p, b, s, h, heads, 4 * h, q_block, causal, 0, ws, odev[k], st, sms, &hook,
-                    xc.n > 0 ? &xc : nullptr);
+                    xc.n > 0 ? &xc : nullptr, nullptr, nullptr, i == 0 || i == n - 1);
       if (r != BPT_OK) break;
       cu = cudaEventRecord(pp.comp_done[k], st) == cudaSuccess;
       for (int c = 0; c < HostPipe::kCopy; ++c) {

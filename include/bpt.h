@@ -212,8 +212,18 @@ int bpt_layer_forward_ws(int dtype, const void* x, const void* Wqkv, const void*
  * i + 1 computes (two device buffers each for x and out and one workspace,
  * from the library's pool; four internal copy streams, two each way, that
  * move every input and every result in two halves, ordered by events
- * against `stream`, which runs the layer). Returns after every result has
- * reached host memory. Errors as bpt_layer_forward; BPT_ERR_SHAPE also for
+ * against `stream`, which runs the layer). The first bf16 input arrives in
+ * four row chunks, each projected when the rows it holds are needed. With
+ * causal attention (a row needs only the keys at or before it) the first and
+ * the last input run wave by wave: the attention of an FFN wave's rows, then
+ * that wave's FFN side, whose scratch then lies beside the K/V copies instead
+ * of over them (one wave's, 14 h bytes a row, more device memory), so that the
+ * first input's compute starts with its first chunk and the last input's
+ * results start to come out early in the layer. Each wave's rows are copied out as soon as
+ * the wave is done, and the last input's last wave runs in two halves so that
+ * only the second half's copy follows the last launch. None of this changes a
+ * result: every row is computed as in bpt_layer_forward, bit for bit. Returns after every result has reached host memory. Errors as
+ * bpt_layer_forward; BPT_ERR_SHAPE also for
  * n_inputs < 0 or a nonzero stride smaller than one input (output); and
  * BPT_ERR_ALIAS if the input and output host ranges overlap. */
 int bpt_layer_forward_host(int dtype, const void* x_host, long long x_stride, const void* Wqkv, const void* bqkv,

@@ -213,6 +213,48 @@ def test_host_entry_equals_the_device_path(dtype):
     assert_parity(got[0].numpy(), oracle_full(shape, inps[0]), f"host entry {dtype}")
 
 
+@pytest.mark.parametrize("b,s,h,heads,q_block,kv_block,causal", [
+    (1, 4096, 256, 2, 512, 512, True),    # one sequence: attention wave by wave, last wave in halves
+    (3, 1000, 256, 2, 200, 125, True),    # waves and row chunks that straddle sequence boundaries
+    (1, 4096, 256, 2, 512, 512, False),   # not causal: one attention launch before the waves
+], ids=["causal_b1", "causal_b3_ragged", "full_b1"])
+def test_host_entry_pipelining_keeps_every_row_bit_equal(b, s, h, heads, q_block, kv_block, causal):
+    # With causal attention the host entry runs each FFN wave's attention just
+    # before the wave (launches split at sequence boundaries, the first input's
+    # row chunks projected as the waves need them) and the last input's last
+    # wave in two halves; the launch counts show that it did, and every row
+    # must still equal the device entry's bit for bit.
+    shape = bi.LayerShape(b, s, h, heads, q_block, kv_block, causal)
+    inp = bi.make_inputs(shape, seed=21)
+    params = device_params(inp)
+    x = bi.to_torch(inp["x"], device="cpu")
+    bpt.set_kernel_timing(True)
+    try:
+        bpt.kernel_times()
+        got = bpt.layer_forward_host(x.pin_memory(), params, heads, q_block, kv_block, causal)
+        torch.cuda.synchronize()
+        k_host = bpt.kernel_times()
+        ref = bpt.layer_forward(x.cuda(), params, heads, q_block, kv_block, causal)
+        torch.cuda.synchronize()
+        k_dev = bpt.kernel_times()
+    finally:
+        bpt.set_kernel_timing(False)
+    assert bpt.stream_status() == 0
+    assert torch.equal(got, ref.cpu())
+    n_att_host, n_att_dev = k_host["attention"][0], k_dev["attention"][0]
+    op_host, op_dev = k_host["gemm_outproj"][0], k_dev["gemm_outproj"][0]
+    assert n_att_dev == 1
+    if causal:
+        # at least one attention launch per wave (one per sequence piece of it)
+        assert n_att_host >= op_dev, (k_host, k_dev)
+    else:
+        assert n_att_host == 1, k_host
+    assert op_dev <= op_host <= op_dev + 1, (k_host, k_dev)
+    if b == 1:
+        assert op_host == op_dev + 1, (k_host, k_dev)
+    assert_parity(got.numpy(), oracle_full(shape, inp), f"host pipeline {shape}")
+
+
 def test_convert_rounds_to_nearest_even_like_torch():
     g = torch.Generator(device="cuda").manual_seed(7)
     src = torch.randn(1 << 20 | 3, generator=g, device="cuda") * 100.0

@@ -205,7 +205,9 @@ class ClockSampler:
         self.path = None
         self.nvml = None
         self.samples = []  # (sm MHz, reasons bitmask)
+        self.watts = []    # board power draw, where NVML reports it
         self.max_mhz = None
+        self.limit_w = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -214,6 +216,11 @@ class ClockSampler:
             self.nvml = pynvml
         except Exception:
             self.nvml = None
+        if self.nvml is not None:
+            try:  # read-only: the limit the power cap enforces, in mW
+                self.limit_w = float(self.nvml.nvmlDeviceGetEnforcedPowerLimit(self.handle)) / 1000.0
+            except Exception:
+                self.limit_w = None
 
     def _reasons(self):
         nv = self.nvml
@@ -225,6 +232,10 @@ class ClockSampler:
         while not self.stop.is_set():
             try:
                 self.samples.append((float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)), self._reasons()))
+            except Exception:
+                pass
+            try:
+                self.watts.append(float(nv.nvmlDeviceGetPowerUsage(self.handle)) / 1000.0)
             except Exception:
                 pass
             self.stop.wait(self.PERIOD_S)
@@ -270,8 +281,13 @@ class ClockSampler:
             if not self.samples:
                 return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
             reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(r & bit for _, r in self.samples))
-            return {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": self.max_mhz,
-                    "reasons": reasons, "samples": len(self.samples), "source": "NVML every 20 ms in the timed region"}
+            out = {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": self.max_mhz,
+                   "reasons": reasons, "samples": len(self.samples), "source": "NVML every 20 ms in the timed region"}
+            if self.watts:
+                out["power_w"] = float(np.median(self.watts))
+            if self.limit_w is not None:
+                out["power_limit_w"] = self.limit_w
+            return out
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         try:

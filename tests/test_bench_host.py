@@ -180,7 +180,9 @@ def test_clock_sampler_reads_nvml_only_inside_the_timed_region(monkeypatch):
         nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
         nvmlDeviceGetMaxClockInfo=lambda h, k: 1965,
         nvmlDeviceGetClockInfo=clock,
-        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 if reads["n"] >= 3 else 0x0)
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 if reads["n"] >= 3 else 0x0,
+        nvmlDeviceGetPowerUsage=lambda h: 998000,        # mW
+        nvmlDeviceGetEnforcedPowerLimit=lambda h: 1000000)
     monkeypatch.setitem(sys.modules, "pynvml", fake)
     import bench
     c = bench.ClockSampler(3)
@@ -193,3 +195,4 @@ def test_clock_sampler_reads_nvml_only_inside_the_timed_region(monkeypatch):
     s = c.summary()
     assert s["samples"] == n_in >= 5 and s["sm_max_mhz"] == 1965.0
     assert s["sm_mhz"] == 1900.0 and s["reasons"] == ["sw_power_cap"]
+    assert s["power_w"] == 998.0 and s["power_limit_w"] == 1000.0

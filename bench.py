@@ -227,6 +227,20 @@ class ClockSampler:
         get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
         return int(get(self.handle))
 
+    def _instant_watts(self):
+        # the instantaneous board power (NVML field POWER_INSTANT, mW): the
+        # plain power query averages over about a second, longer than the
+        # timed region, so it is not used
+        nv = self.nvml
+        try:
+            v = nv.nvmlDeviceGetFieldValues(self.handle, [nv.NVML_FI_DEV_POWER_INSTANT])[0]
+            if v.nvmlReturn != 0:
+                return None
+            kinds = {0: "dVal", 1: "uiVal", 2: "ulVal", 3: "ullVal", 4: "sllVal", 5: "siVal"}
+            return float(getattr(v.value, kinds[int(v.valueType)])) / 1000.0
+        except Exception:
+            return None
+
     def _run(self):
         nv = self.nvml
         while not self.stop.is_set():
@@ -234,10 +248,9 @@ class ClockSampler:
                 self.samples.append((float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)), self._reasons()))
             except Exception:
                 pass
-            try:
-                self.watts.append(float(nv.nvmlDeviceGetPowerUsage(self.handle)) / 1000.0)
-            except Exception:
-                pass
+            w = self._instant_watts()
+            if w is not None:
+                self.watts.append(w)
             self.stop.wait(self.PERIOD_S)
 
     def __enter__(self):
@@ -285,6 +298,8 @@ class ClockSampler:
                    "reasons": reasons, "samples": len(self.samples), "source": "NVML every 20 ms in the timed region"}
             if self.watts:
                 out["power_w"] = float(np.median(self.watts))
+                out["power_source"] = "NVML instantaneous board power, median of the samples"
+
             if self.limit_w is not None:
                 out["power_limit_w"] = self.limit_w
             return out

@@ -181,7 +181,9 @@ def test_clock_sampler_reads_nvml_only_inside_the_timed_region(monkeypatch):
         nvmlDeviceGetMaxClockInfo=lambda h, k: 1965,
         nvmlDeviceGetClockInfo=clock,
         nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 if reads["n"] >= 3 else 0x0,
-        nvmlDeviceGetPowerUsage=lambda h: 998000,        # mW
+        NVML_FI_DEV_POWER_INSTANT=186,
+        nvmlDeviceGetFieldValues=lambda h, ids: [types.SimpleNamespace(
+            nvmlReturn=0, valueType=1, value=types.SimpleNamespace(uiVal=998000))],  # mW
         nvmlDeviceGetEnforcedPowerLimit=lambda h: 1000000)
     monkeypatch.setitem(sys.modules, "pynvml", fake)
     import bench

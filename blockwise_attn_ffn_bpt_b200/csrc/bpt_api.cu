@@ -1235,11 +1235,13 @@ struct XChunks {
 // and the per-GEMM wave schedule.
 bool interleavable(int dtype, int causal, int wave_rows) { return causal && !use_chain(dtype, wave_rows); }
 
-// interleave (callers that size the workspace with layout_for(...,
-// interleavable(dtype, causal, wave_rows))): attention runs wave by wave, each
+// interleave_req, where interleavable(): attention runs wave by wave, each
 // wave's rows just before that wave's FFN side, and the first input's row
 // chunks (xc) are projected as the waves need them, so that results start to
-// come out early in the layer rather than after all of attention.
+// come out early in the layer rather than after all of attention. The caller
+// then sizes ws with layout_for(..., interleavable(dtype, causal, wave_rows)),
+// whose FFN scratch lies beside K/V; that workspace also holds the layout
+// without interleave.
 int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int ffn, int q_block, int causal,
               int wave_rows, uint8_t* ws, float* out, cudaStream_t st, int sms, const WaveHook* hook = nullptr,
               const XChunks* xc = nullptr, __nv_bfloat16* o_save = nullptr, float* lse2_save = nullptr,

@@ -217,7 +217,8 @@ def test_host_entry_equals_the_device_path(dtype):
     (1, 4096, 256, 2, 512, 512, True),    # one sequence: attention wave by wave, last wave in halves
     (3, 1000, 256, 2, 200, 125, True),    # waves and row chunks that straddle sequence boundaries
     (1, 4096, 256, 2, 512, 512, False),   # not causal: one attention launch before the waves
-], ids=["causal_b1", "causal_b3_ragged", "full_b1"])
+    (1, 6000, 256, 2, 1000, 500, True),   # waves of whole 1000-row query blocks: rows start off the 128-row tiles
+], ids=["causal_b1", "causal_b3_ragged", "full_b1", "causal_q1000"])
 def test_host_entry_pipelining_keeps_every_row_bit_equal(b, s, h, heads, q_block, kv_block, causal):
     # With causal attention the host entry runs each FFN wave's attention just
     # before the wave (launches split at sequence boundaries, the first input's
@@ -252,7 +253,8 @@ def test_host_entry_pipelining_keeps_every_row_bit_equal(b, s, h, heads, q_block
     assert op_dev <= op_host <= op_dev + 1, (k_host, k_dev)
     if b == 1:
         assert op_host == op_dev + 1, (k_host, k_dev)
-    assert_parity(got.numpy(), oracle_full(shape, inp), f"host pipeline {shape}")
+    if s * s * h <= 4096 * 4096 * 256:  # the device entry itself is checked against the oracle elsewhere
+        assert_parity(got.numpy(), oracle_full(shape, inp), f"host pipeline {shape}")
 
 
 def test_convert_rounds_to_nearest_even_like_torch():

@@ -60,6 +60,7 @@ def layer_flops(shape: bi.LayerShape) -> dict:
 def kernel_flops(shape: bi.LayerShape) -> dict:
     f = layer_flops(shape)
     f["ffn_chain"] = f["gemm_outproj"] + f["gemm_ffn_up"] + f["gemm_ffn_down"]
+    f["layer_mega"] = f["attention"] + f["ffn_chain"]  # attention and the FFN side in one launch
     return f
 
 

@@ -198,3 +198,18 @@ def test_clock_sampler_reads_nvml_only_inside_the_timed_region(monkeypatch):
     assert s["samples"] == n_in >= 5 and s["sm_max_mhz"] == 1965.0
     assert s["sm_mhz"] == 1900.0 and s["reasons"] == ["sw_power_cap"]
     assert s["power_w"] == 998.0 and s["power_limit_w"] == 1000.0
+
+
+def test_every_forward_kernel_of_each_schedule_has_its_flops():
+    # the kernels one forward launches under each FFN schedule (the library's
+    # timing-log names) all have a flop count, and the fused launches count
+    # exactly the steps they run
+    import bench
+    import bpt_inputs as bi
+    shape = bi.WORKLOADS["gpt7b_s32768_h4096"]
+    f = bench.kernel_flops(shape)
+    for name in ("gemm_qkv", "attention", "gemm_outproj", "gemm_ffn_up", "gemm_ffn_down", "ffn_chain", "layer_mega"):
+        assert f[name] > 0, name
+    assert f["ffn_chain"] == f["gemm_outproj"] + f["gemm_ffn_up"] + f["gemm_ffn_down"]
+    assert f["layer_mega"] == f["attention"] + f["ffn_chain"]
+    assert sum(bench.layer_flops(shape).values()) == f["gemm_qkv"] + f["layer_mega"]

@@ -41,7 +41,11 @@ constexpr int ATT_REGS_SOFTMAX = 216;  // warpgroups 1 and 2
 static_assert(ATT_THREADS * ATT_REGS_LAUNCH >= 128 * ATT_REGS_CONTROL + 256 * ATT_REGS_SOFTMAX,
               "register split exceeds the block's launch allocation");
 constexpr int ATT_TMEM_COLS = 512;
-constexpr int ATT_HEAD_GROUP = 4;  // heads scheduled together (see the grid order below)
+// Heads scheduled together (see the grid order below). Two: at s = 32768 a
+// group of four heads' K/V (67 MB) and the next group's exceeded L2 (DRAM
+// reads 1.48x Q + K + V); groups of two read 1.01x and ran ~1% faster, and
+// single heads ran ~1.5% slower (fewer CTAs share each K/V tile).
+constexpr int ATT_HEAD_GROUP = 2;
 // Skip rescaling O until the running max has grown by more than this (log2
 // units); P then holds values up to 2^8, well inside bf16 and fp32 range. The
 // final division by l uses the same stale max, so the result is exact.

@@ -40,7 +40,7 @@ def nvcc() -> str:
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(INCLUDE, "bpt.h")])
+                  + glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "bpt.h")])
 
 
 def up_to_date() -> bool:

@@ -36,6 +36,7 @@
 #include "ffn_chain.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "row_pieces.h"
 
 // The bf16 forward GEMMs run on SM pairs (gemm_pair.cuh) when this is 1, on
 // single SMs (gemm.cuh) when it is 0. Measured on B200 at b=1, s=32768,
@@ -1266,20 +1267,15 @@ int run_layer(int dtype, const LayerPtrs& p, int b, int s, int h, int heads, int
   const bool mega = L.mega && mega_available() && o_save == nullptr;
   const __nv_bfloat16* O = o_save != nullptr ? o_save : QO;
   const long long ldo = o_save != nullptr ? (long long)h : ldq;
-  // Attention of the flat rows [r0, r0 + m), split at sequence boundaries into
-  // launches over whole sequences or one sequence's run of rows. Every row's
-  // arithmetic is the same as in one launch over all rows.
+  // Attention of the flat rows [r0, r0 + m), one launch per piece (whole
+  // sequences, or one sequence's run of rows). Every row's arithmetic is the
+  // same as in one launch over all rows.
   auto attend_rows = [&](long long r0, long long m) -> int {
-    for (long long r = r0, end = r0 + m; r < end;) {
-      const int beta = (int)(r / s), t = (int)(r - (long long)beta * s);
-      const bool whole = t == 0 && end - r >= s;
-      const int nb = whole ? (int)std::min<long long>((end - r) / s, b - beta) : 1;
-      const int tl = whole ? s : (int)std::min<long long>(s - t, end - r);
-      BPT_TRY(launch_attention(QO, ldq, K, V, b, s, h, heads, causal, beta, nb, t, tl,
-                               const_cast<__nv_bfloat16*>(O) + r * ldo, ldo, st, status));
-      r += (long long)nb * tl;
-    }
-    return BPT_OK;
+    return for_each_row_piece(r0, m, b, s, [&](const RowPiece& pc) -> int {
+      const long long r = (long long)pc.beta * s + pc.t_start;
+      return launch_attention(QO, ldq, K, V, b, s, h, heads, causal, pc.beta, pc.n_seq, pc.t_start, pc.t_len,
+                              const_cast<__nv_bfloat16*>(O) + r * ldo, ldo, st, status);
+    });
   };
   // the first input's row chunks, projected in order up to a given row
   const bool chunked = !f32 && xc != nullptr && xc->n > 0;

@@ -88,10 +88,6 @@ __device__ __forceinline__ int a_block(const GemmArgs& a, int kb) {
   return kb - a.a_kb;
 }
 
-__device__ __forceinline__ float load_vec_elem(const void* p, int f32, long long i) {
-  return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
-}
-
 // 32 consecutive values (columns col .. col+31) of one row.
 __device__ __forceinline__ void load32(const void* p, int f32, long long off, float (&v)[32]) {
   if (f32) {
